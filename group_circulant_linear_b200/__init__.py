@@ -16,6 +16,6 @@ __all__ = ["inputs", "workloads", "eqlin"]
 
 def __getattr__(name):
     if name == "eqlin":
-        from . import eqlin as _eqlin
-        return _eqlin
+        import importlib
+        return importlib.import_module(".eqlin", __name__)
     raise AttributeError(name)

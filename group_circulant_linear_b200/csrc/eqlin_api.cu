@@ -1,0 +1,216 @@
+// eqlin_api.cu -- the C ABI: handle lifetime, argument checks, dispatch.
+//
+// Every entry point validates its arguments on the host, returns a status and
+// enqueues kernels on the caller's stream.  No entry point synchronises except
+// eqlin_get_error (which reads the device error word) and eqlin_destroy.
+#include <stdlib.h>
+#include <string.h>
+#include <new>
+
+#include "eqlin_internal.cuh"
+
+using eqlin::Handle;
+
+struct eqlin_handle {
+  Handle h;
+};
+
+namespace {
+
+size_t elem_size(eqlin_dtype_t dt) { return dt == EQLIN_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Make the handle's device current for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+void free_all(Handle& h) {
+  cudaFree(h.wf_fwd);
+  cudaFree(h.wf_bwd);
+  cudaFree(h.wt_fwd);
+  cudaFree(h.wt_bwd);
+  cudaFree(h.bias);
+  cudaFree(h.ws);
+  cudaFree(h.err);
+  h.wf_fwd = h.wf_bwd = nullptr;
+  h.wt_fwd = h.wt_bwd = nullptr;
+  h.bias = h.ws = nullptr;
+  h.err = nullptr;
+}
+
+eqlin_status_t check_io(const Handle& h, const void* a, const void* b, int64_t N) {
+  if (N < 0) return EQLIN_ERR_INVALID_ARG;
+  if (N == 0) return EQLIN_OK;
+  if (!a || !b) return EQLIN_ERR_INVALID_ARG;
+  if (!h.has_weights) return EQLIN_ERR_NO_WEIGHTS;
+  if (!aligned16(a) || !aligned16(b)) return EQLIN_ERR_MISALIGNED;
+  return EQLIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* eqlin_status_string(eqlin_status_t s) {
+  switch (s) {
+    case EQLIN_OK: return "ok";
+    case EQLIN_ERR_INVALID_ARG: return "invalid argument";
+    case EQLIN_ERR_UNSUPPORTED: return "unsupported group order or size";
+    case EQLIN_ERR_MISALIGNED: return "pointer or row not 16-byte aligned";
+    case EQLIN_ERR_CUDA: return "CUDA error";
+    case EQLIN_ERR_NO_WEIGHTS: return "weights not set";
+    case EQLIN_ERR_TIMEOUT: return "device-side wait timed out";
+    case EQLIN_ERR_OOM: return "device out of memory";
+  }
+  return "unknown status";
+}
+
+eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, eqlin_t* out) {
+  if (!out) return EQLIN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (dtype != EQLIN_F32 && dtype != EQLIN_F16 && dtype != EQLIN_BF16) return EQLIN_ERR_INVALID_ARG;
+  if (Cp < 1 || Dp < 1) return EQLIN_ERR_INVALID_ARG;
+  if (T != 1 && T != 2 && T != 4 && T != 8) return EQLIN_ERR_UNSUPPORTED;
+  if (Cp > 65536 || Dp > 65536) return EQLIN_ERR_UNSUPPORTED;
+  const size_t e = elem_size(dtype);
+  if ((Cp * T * e) % 16 || (Dp * T * e) % 16) return EQLIN_ERR_MISALIGNED;
+
+  eqlin_handle* hh = new (std::nothrow) eqlin_handle();
+  if (!hh) return EQLIN_ERR_OOM;
+  Handle& h = hh->h;
+  h.T = T;
+  h.Cp = Cp;
+  h.Dp = Dp;
+  h.dtype = dtype;
+  if (cudaGetDevice(&h.device) != cudaSuccess) { delete hh; return EQLIN_ERR_CUDA; }
+  if (cudaDeviceGetAttribute(&h.sm_count, cudaDevAttrMultiProcessorCount, h.device) != cudaSuccess) {
+    delete hh;
+    return EQLIN_ERR_CUDA;
+  }
+  const size_t planes = (size_t)T * Cp * Dp;
+  const int Q = (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
+  h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
+  bool ok = cudaMalloc(&h.wf_fwd, planes * 4) == cudaSuccess &&
+            cudaMalloc(&h.wf_bwd, planes * 4) == cudaSuccess &&
+            cudaMalloc(&h.bias, (size_t)Dp * 4) == cudaSuccess &&
+            cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
+            cudaMalloc(&h.err, sizeof(int)) == cudaSuccess;
+  if (ok && dtype != EQLIN_F32) {
+    ok = cudaMalloc(&h.wt_fwd, (size_t)Q * Cp * Dp * e) == cudaSuccess &&
+         cudaMalloc(&h.wt_bwd, (size_t)Q * Cp * Dp * e) == cudaSuccess;
+  }
+  if (ok) ok = cudaMemset(h.err, 0, sizeof(int)) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete hh;
+    return EQLIN_ERR_OOM;
+  }
+  h.backend = (dtype == EQLIN_F32) ? "simt" : (eqlin::tc_supported(h, false) ? "tcgen05" : "simt");
+  *out = hh;
+  return EQLIN_OK;
+}
+
+void eqlin_destroy(eqlin_t hh) {
+  if (!hh) return;
+  DeviceGuard g(hh->h.device);
+  cudaDeviceSynchronize();
+  free_all(hh->h);
+  delete hh;
+}
+
+eqlin_status_t eqlin_set_weights(eqlin_t hh, const void* W, const void* b, void* stream) {
+  if (!hh || !W) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  if (!aligned16(W) || (b && ((uintptr_t)b % elem_size(h.dtype)))) return EQLIN_ERR_MISALIGNED;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  cudaError_t e = eqlin::launch_pretransform(h, W, b, (cudaStream_t)stream);
+  if (e != cudaSuccess) return EQLIN_ERR_CUDA;
+  h.has_weights = true;
+  return EQLIN_OK;
+}
+
+eqlin_status_t eqlin_forward(eqlin_t hh, const void* x, void* y, int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  eqlin_status_t s = check_io(h, x, y, N);
+  if (s != EQLIN_OK || N == 0) return s;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  cudaError_t e;
+  if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, false))
+    e = eqlin::launch_tc_apply(h, false, x, y, N, (cudaStream_t)stream);
+  else
+    e = eqlin::launch_simt_apply(h, false, x, y, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_backward_dx(eqlin_t hh, const void* gy, void* dx, int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  eqlin_status_t s = check_io(h, gy, dx, N);
+  if (s != EQLIN_OK || N == 0) return s;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  cudaError_t e;
+  if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, true))
+    e = eqlin::launch_tc_apply(h, true, gy, dx, N, (cudaStream_t)stream);
+  else
+    e = eqlin::launch_simt_apply(h, true, gy, dx, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, float* dW, float* db,
+                                 int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  if (!dW || N < 0) return EQLIN_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (db && !aligned16(db))) return EQLIN_ERR_MISALIGNED;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  if (N == 0) {
+    cudaError_t e = cudaMemsetAsync(dW, 0, (size_t)h.Dp * h.Cp * h.T * 4, (cudaStream_t)stream);
+    if (e == cudaSuccess && db) e = cudaMemsetAsync(db, 0, (size_t)h.Dp * 4, (cudaStream_t)stream);
+    return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+  }
+  eqlin_status_t s = check_io(h, x, gy, N);
+  if (s != EQLIN_OK) return s;
+  cudaError_t e = eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_get_error(eqlin_t hh) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  DeviceGuard g(h.device);
+  int v = 0;
+  if (cudaMemcpy(&v, h.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return EQLIN_ERR_CUDA;
+  if (v != eqlin::DEV_OK) {
+    const int zero = 0;
+    if (cudaMemcpy(h.err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return EQLIN_ERR_CUDA;
+  }
+  return v == eqlin::DEV_OK ? EQLIN_OK : v == eqlin::DEV_TIMEOUT ? EQLIN_ERR_TIMEOUT : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_set_wait_limit(eqlin_t hh, uint32_t iterations) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  hh->h.wait_limit = iterations;
+  return EQLIN_OK;
+}
+
+const char* eqlin_backend_name(eqlin_t hh) { return hh ? hh->h.backend : "none"; }
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// eqlin_internal.cuh -- shared declarations of the Flash EQ-Linear CUDA library.
+//
+// Group-axis transforms used by every kernel ("Flash EQ-Linear", technical
+// summary, section "Abordagem Algoritmica"): with theta = 2*pi*k*t/T,
+//
+//   forward DFT   V_k = sum_t v_t (cos theta - i sin theta),   k = 0 .. floor(T/2)
+//   inverse DFT   v_s = (1/T) [ V_0 + (-1)^s V_{T/2} + 2 sum_{0<k<T/2} Re(V_k e^{+i theta_s}) ]
+//
+// Real inputs give a Hermitian spectrum, so only the half spectrum is kept
+// (item 2 of the same section).  A T-vector is held as T real "planes":
+//   plane 0             Re V_0
+//   plane 1 (T even)    Re V_{T/2}
+//   plane nreal+2(k-1)  Re V_k,  plane nreal+2(k-1)+1  Im V_k,  k = 1 .. T/2-1
+// For p4 that is [V0, V2, Re V1, Im V1], and the transforms need only adds,
+// subtracts and power-of-two scales (section "Especializacao ... p4").
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/eqlin.h"
+
+namespace eqlin {
+
+// ------------------------------------------------------------- element types
+template <typename E> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float v) { return v; }
+  static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__half> {
+  static __device__ __forceinline__ float to_f(__half v) { return __half2float(v); }
+  static __device__ __forceinline__ __half from_f(float v) { return __float2half_rn(v); }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+// --------------------------------------------------- group-axis plane tables
+// cos/sin of 2*pi*j/8; T in {1,2,4,8} reads entry (j * 8/T) mod 8.  The only
+// inexact entry is sqrt(2)/2 (T = 8), rounded once to float.
+#define EQLIN_RSQRT2 0.70710678118654752440f
+
+template <int T> struct Group {
+  static constexpr int nreal = (T == 1) ? 1 : 2;        // k = 0 and k = T/2
+  static constexpr int ncomplex = (T - nreal) / 2;      // k = 1 .. T/2-1
+  static constexpr int planes = T;                      // real planes of the half spectrum
+  // Real GEMM count R(T): one per real frequency, four per complex one.
+  static constexpr int gemms = nreal + 4 * ncomplex;
+
+  static __host__ __device__ __forceinline__ float cos8(int j) {
+    j &= 7;
+    return j == 0 ? 1.f : j == 1 ? EQLIN_RSQRT2 : j == 2 ? 0.f : j == 3 ? -EQLIN_RSQRT2
+         : j == 4 ? -1.f : j == 5 ? -EQLIN_RSQRT2 : j == 6 ? 0.f : EQLIN_RSQRT2;
+  }
+  static __host__ __device__ __forceinline__ float sin8(int j) { return cos8(j - 2); }
+  // cos / sin of 2*pi*k*t/T
+  static __host__ __device__ __forceinline__ float c(int k, int t) { return cos8(k * t * (8 / T)); }
+  static __host__ __device__ __forceinline__ float s(int k, int t) { return sin8(k * t * (8 / T)); }
+
+  // Forward real DFT of v[0..T) into planes P[0..T).
+  static __host__ __device__ __forceinline__ void dft(const float* v, float* P) {
+    float a = 0.f;
+#pragma unroll
+    for (int t = 0; t < T; ++t) a += v[t];
+    P[0] = a;
+    if (T >= 2) {
+      float h = 0.f;
+#pragma unroll
+      for (int t = 0; t < T; ++t) h += (t & 1) ? -v[t] : v[t];
+      P[1] = h;
+    }
+#pragma unroll
+    for (int k = 1; k <= ncomplex; ++k) {
+      float re = 0.f, im = 0.f;
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        const float ct = c(k, t), st = s(k, t);
+        if (ct != 0.f) re += (ct == 1.f ? v[t] : ct == -1.f ? -v[t] : ct * v[t]);
+        if (st != 0.f) im -= (st == 1.f ? v[t] : st == -1.f ? -v[t] : st * v[t]);
+      }
+      P[nreal + 2 * (k - 1)] = re;
+      P[nreal + 2 * (k - 1) + 1] = im;
+    }
+  }
+
+  // Inverse real DFT of planes P into v[0..T), including the 1/T.
+  static __host__ __device__ __forceinline__ void idft(const float* P, float* v) {
+#pragma unroll
+    for (int s_ = 0; s_ < T; ++s_) {
+      float a = P[0];
+      if (T >= 2) a += (s_ & 1) ? -P[1] : P[1];
+      float acc2 = 0.f;
+#pragma unroll
+      for (int k = 1; k <= ncomplex; ++k) {
+        const float cs = c(k, s_), sn = s(k, s_);
+        const float re = P[nreal + 2 * (k - 1)], im = P[nreal + 2 * (k - 1) + 1];
+        if (cs != 0.f) acc2 += (cs == 1.f ? re : cs == -1.f ? -re : cs * re);
+        if (sn != 0.f) acc2 -= (sn == 1.f ? im : sn == -1.f ? -im : sn * im);
+      }
+      v[s_] = (a + 2.f * acc2) * (1.f / T);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ handle
+struct Handle {
+  int T = 0;
+  int64_t Cp = 0, Dp = 0;
+  eqlin_dtype_t dtype = EQLIN_F32;
+  int device = 0;
+  int sm_count = 0;
+  bool has_weights = false;
+  // FP32 Fourier planes for the SIMT kernels: fwd [T][Cp][Dp] (row = input
+  // channel, contiguous over output channel); bwd [T][Dp][Cp], conjugated.
+  float* wf_fwd = nullptr;
+  float* wf_bwd = nullptr;
+  // Fourier planes in the handle dtype for the tensor-core kernels, K-major:
+  // fwd [Q][Dp][Cp], bwd [Q][Cp][Dp]; Q = real freqs + 3 per complex freq
+  // (-Im, Re, Im stacked so that [Re;Im] and [-Im;Re] are contiguous windows).
+  void* wt_fwd = nullptr;
+  void* wt_bwd = nullptr;
+  float* bias = nullptr;          // [Dp] float32 (zeros when no bias)
+  float* ws = nullptr;            // dW split partials
+  size_t ws_bytes = 0;
+  int* err = nullptr;             // device error word
+  uint32_t wait_limit = 0;        // 0 = default
+  const char* backend = "simt";
+};
+
+// Device error codes written into Handle::err (first writer wins).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+
+constexpr uint32_t kDefaultWaitLimit = 1u << 26;   // polls; ~seconds at worst
+
+// ------------------------------------------------------- launch wrappers
+// SIMT path (any T in {1,2,4,8}, any dtype).
+cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st);
+cudaError_t launch_simt_apply(const Handle& h, bool backward, const void* in, void* out,
+                              int64_t N, cudaStream_t st);
+cudaError_t launch_simt_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                           int64_t N, cudaStream_t st);
+size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp);
+
+// tcgen05 path (f16/bf16).  Returns cudaErrorNotSupported when the shape is
+// outside what the kernel handles, so the caller can fall back to SIMT.
+bool tc_supported(const Handle& h, bool backward);
+cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out,
+                            int64_t N, cudaStream_t st);
+
+}  // namespace eqlin

@@ -1,0 +1,442 @@
+// eqlin_simt.cu -- weight pre-transform and the SIMT (CUDA-core) kernels.
+//
+// These kernels serve every T in {1,2,4,8} and every dtype.  They are the
+// FP32 path (FFMA, FP32 accumulation) and the reference structure the
+// tensor-core kernels follow:
+//
+//   prologue  DFT of each input row along t, one T-vector per channel
+//   mainloop  per-frequency channel products on the half spectrum: one real
+//             product per real frequency, a complex product (4 real ones)
+//             per complex frequency -- R(T) real GEMMs in all
+//   epilogue  inverse DFT along the frequency axis, 1/T, bias, cast, store
+//
+// ("Flash EQ-Linear", technical summary, sections "Abordagem Algoritmica" and
+// "Implementacao": fused data flow, no intermediate global writes.)
+#include "eqlin_internal.cuh"
+
+namespace eqlin {
+
+// ========================================================== weight transform
+// One thread per (d, c): the DFT of W[d, c, 0..T) along tau, written as
+//   wf_fwd[p][c][d]  (FP32, forward planes)
+//   wf_bwd[p][d][c]  (FP32, conjugated: the dx product uses conj(W_hat))
+//   wt_fwd[q][d][c], wt_bwd[q][c][d]  (handle dtype, tensor-core operand
+//   planes; q enumerates real frequencies, then (-Im, Re, Im) triples)
+template <int T, typename E>
+__global__ void pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b,
+                                    float* __restrict__ wf_fwd, float* __restrict__ wf_bwd,
+                                    E* __restrict__ wt_fwd, E* __restrict__ wt_bwd,
+                                    float* __restrict__ bias, int Cp, int Dp) {
+  using G = Group<T>;
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)Cp * Dp;
+  if (idx < Dp) bias[idx] = b ? Elem<E>::to_f(b[idx]) : 0.f;
+  if (idx >= total) return;
+  const int d = (int)(idx % Dp), c = (int)(idx / Dp);    // d fastest: coalesced wf_fwd writes
+  float v[T], P[T];
+#pragma unroll
+  for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(W[((int64_t)d * Cp + c) * T + t]);
+  G::dft(v, P);
+  const int64_t plane = (int64_t)Cp * Dp;
+#pragma unroll
+  for (int p = 0; p < T; ++p) {
+    const bool imag = p >= G::nreal && ((p - G::nreal) & 1);
+    wf_fwd[p * plane + (int64_t)c * Dp + d] = P[p];
+    wf_bwd[p * plane + (int64_t)d * Cp + c] = imag ? -P[p] : P[p];
+  }
+  if (wt_fwd) {
+#pragma unroll
+    for (int f = 0; f < G::nreal; ++f) {
+      wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f]);
+      wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f]);
+    }
+#pragma unroll
+    for (int k = 1; k <= G::ncomplex; ++k) {
+      const float re = P[G::nreal + 2 * (k - 1)], im = P[G::nreal + 2 * (k - 1) + 1];
+      const int q = G::nreal + 3 * (k - 1);
+      // forward: (-Im, Re, Im); backward uses conj(W_hat): Im -> -Im
+      wt_fwd[(q + 0) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(-im);
+      wt_fwd[(q + 1) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(re);
+      wt_fwd[(q + 2) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(im);
+      wt_bwd[(q + 0) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(im);
+      wt_bwd[(q + 1) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(re);
+      wt_bwd[(q + 2) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(-im);
+    }
+  }
+}
+
+template <int T, typename E>
+static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b, cudaStream_t st) {
+  const int64_t total = h.Cp * h.Dp;
+  const int64_t work = total > h.Dp ? total : h.Dp;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((work + threads - 1) / threads);
+  pretransform_kernel<T, E><<<blocks, threads, 0, st>>>(
+      (const E*)W, (const E*)b, h.wf_fwd, h.wf_bwd, (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias,
+      (int)h.Cp, (int)h.Dp);
+  return cudaGetLastError();
+}
+
+template <typename E>
+static cudaError_t pretransform_e(const Handle& h, const void* W, const void* b, cudaStream_t st) {
+  switch (h.T) {
+    case 1: return pretransform_t<1, E>(h, W, b, st);
+    case 2: return pretransform_t<2, E>(h, W, b, st);
+    case 4: return pretransform_t<4, E>(h, W, b, st);
+    case 8: return pretransform_t<8, E>(h, W, b, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st) {
+  switch (h.dtype) {
+    case EQLIN_F32: return pretransform_e<float>(h, W, b, st);
+    case EQLIN_F16: return pretransform_e<__half>(h, W, b, st);
+    case EQLIN_BF16: return pretransform_e<__nv_bfloat16>(h, W, b, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ============================================================ apply (fwd/dx)
+// out[n, o*T+s] = bias[o] + IDFT_s( sum_i planes[.][i][o] (*) DFT(in[n, i*T+.]) )
+// planes [T][K][O] FP32.  Forward: in = x, K = C', O = D', forward planes.
+// dx: in = gy, K = D', O = C', conjugated planes, no bias.
+namespace simt {
+constexpr int BM = 64, BO = 32, BK = 8, THREADS = 256;
+}
+
+template <int T, typename E>
+__global__ void __launch_bounds__(simt::THREADS)
+simt_apply_kernel(const E* __restrict__ in, const float* __restrict__ planes,
+                  const float* __restrict__ bias, E* __restrict__ out, int64_t N, int K, int O) {
+  using G = Group<T>;
+  using namespace simt;
+  __shared__ float Xs[T][BK][BM];
+  __shared__ __align__(16) float Ws[T][BK][BO];
+
+  const int tid = threadIdx.x;
+  const int to = tid % 8, tn = tid / 8;              // 4 outputs x 2 tokens per thread
+  const int64_t n0 = (int64_t)blockIdx.x * BM;
+  const int o0 = blockIdx.y * BO;
+  const int64_t plane = (int64_t)K * O;
+
+  float acc[2][4][T];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int p = 0; p < T; ++p) acc[i][j][p] = 0.f;
+
+  for (int k0 = 0; k0 < K; k0 += BK) {
+    // prologue: DFT of BM x BK input T-vectors into the planes Xs
+#pragma unroll
+    for (int r = 0; r < (BM * BK) / THREADS; ++r) {
+      const int q = tid + r * THREADS;
+      const int kk = q % BK, nn = q / BK;
+      const int64_t n = n0 + nn;
+      const int k = k0 + kk;
+      float v[T], P[T];
+      if (n < N && k < K) {
+        const E* src = in + n * (int64_t)K * T + (int64_t)k * T;
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(src[t]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = 0.f;
+      }
+      G::dft(v, P);
+#pragma unroll
+      for (int p = 0; p < T; ++p) Xs[p][kk][nn] = P[p];
+    }
+    // Fourier weight planes
+    for (int q = tid; q < T * BK * BO; q += THREADS) {
+      const int oo = q % BO, kk = (q / BO) % BK, p = q / (BO * BK);
+      const int o = o0 + oo, k = k0 + kk;
+      Ws[p][kk][oo] = (o < O && k < K) ? planes[p * plane + (int64_t)k * O + o] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float xv[2][T], wv[4][T];
+#pragma unroll
+      for (int p = 0; p < T; ++p) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) xv[i][p] = Xs[p][kk][tn + 32 * i];
+        const float4 w4 = *reinterpret_cast<const float4*>(&Ws[p][kk][to * 4]);
+        wv[0][p] = w4.x; wv[1][p] = w4.y; wv[2][p] = w4.z; wv[3][p] = w4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int f = 0; f < G::nreal; ++f) acc[i][j][f] = fmaf(xv[i][f], wv[j][f], acc[i][j][f]);
+#pragma unroll
+          for (int m = 0; m < G::ncomplex; ++m) {
+            const int pr = G::nreal + 2 * m, pi = pr + 1;
+            acc[i][j][pr] = fmaf(xv[i][pr], wv[j][pr], acc[i][j][pr]);
+            acc[i][j][pr] = fmaf(-xv[i][pi], wv[j][pi], acc[i][j][pr]);
+            acc[i][j][pi] = fmaf(xv[i][pr], wv[j][pi], acc[i][j][pi]);
+            acc[i][j][pi] = fmaf(xv[i][pi], wv[j][pr], acc[i][j][pi]);
+          }
+        }
+    }
+    __syncthreads();
+  }
+  // epilogue: inverse DFT, bias, store T contiguous outputs per (n, o)
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int64_t n = n0 + tn + 32 * i;
+    if (n >= N) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int o = o0 + to * 4 + j;
+      if (o >= O) continue;
+      float v[T];
+      G::idft(acc[i][j], v);
+      const float bo = bias ? bias[o] : 0.f;
+      E* dst = out + n * (int64_t)O * T + (int64_t)o * T;
+#pragma unroll
+      for (int s = 0; s < T; ++s) dst[s] = Elem<E>::from_f(v[s] + bo);
+    }
+  }
+}
+
+template <int T, typename E>
+static cudaError_t simt_apply_t(const Handle& h, bool backward, const void* in, void* out,
+                                int64_t N, cudaStream_t st) {
+  const int K = (int)(backward ? h.Dp : h.Cp);
+  const int O = (int)(backward ? h.Cp : h.Dp);
+  const int64_t tiles_n = (N + simt::BM - 1) / simt::BM;
+  if (tiles_n > 0x7fffffff) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)tiles_n, (unsigned)((O + simt::BO - 1) / simt::BO));
+  simt_apply_kernel<T, E><<<grid, simt::THREADS, 0, st>>>(
+      (const E*)in, backward ? h.wf_bwd : h.wf_fwd, backward ? nullptr : h.bias, (E*)out, N, K, O);
+  return cudaGetLastError();
+}
+
+template <typename E>
+static cudaError_t simt_apply_e(const Handle& h, bool bwd, const void* in, void* out, int64_t N,
+                                cudaStream_t st) {
+  switch (h.T) {
+    case 1: return simt_apply_t<1, E>(h, bwd, in, out, N, st);
+    case 2: return simt_apply_t<2, E>(h, bwd, in, out, N, st);
+    case 4: return simt_apply_t<4, E>(h, bwd, in, out, N, st);
+    case 8: return simt_apply_t<8, E>(h, bwd, in, out, N, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_simt_apply(const Handle& h, bool backward, const void* in, void* out,
+                              int64_t N, cudaStream_t st) {
+  switch (h.dtype) {
+    case EQLIN_F32: return simt_apply_e<float>(h, backward, in, out, N, st);
+    case EQLIN_F16: return simt_apply_e<__half>(h, backward, in, out, N, st);
+    case EQLIN_BF16: return simt_apply_e<__nv_bfloat16>(h, backward, in, out, N, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ================================================================= dW and db
+// Fourier form of the weight gradient (derived from the definition; the
+// pages give no formula): dW_hat_k[d, c] = sum_n G_k[n, d] conj(X_k[n, c]),
+// G = DFT(gy), X = DFT(x); dW = IDFT_tau(dW_hat) with the 1/T.  db[d] =
+// sum_n G_0[n, d].  Stage 1 writes per-split partial planes; stage 2 sums the
+// splits in a fixed order and applies the inverse DFT (deterministic).
+namespace simtdw {
+constexpr int BD = 32, BC = 32, BK = 16, THREADS = 256, MAX_SPLITS = 64, TARGET_CTAS = 4 * 148;
+}
+
+static int dw_splits(int64_t Cp, int64_t Dp, int64_t N) {
+  using namespace simtdw;
+  const int64_t tiles = ((Cp + BC - 1) / BC) * ((Dp + BD - 1) / BD);
+  int64_t s = (TARGET_CTAS + tiles - 1) / tiles;
+  const int64_t max_by_n = (N + BK - 1) / BK;
+  if (s > MAX_SPLITS) s = MAX_SPLITS;
+  if (s > max_by_n) s = max_by_n;
+  return s < 1 ? 1 : (int)s;
+}
+
+size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp) {
+  const int64_t s = dw_splits(Cp, Dp, INT64_MAX / 2);
+  return (size_t)s * ((size_t)T * Cp * Dp + Dp) * sizeof(float);
+}
+
+template <int T, typename E>
+__global__ void __launch_bounds__(simtdw::THREADS)
+simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restrict__ part,
+               float* __restrict__ dbpart, int64_t N, int Cp, int Dp, int64_t tok_per_split) {
+  using G = Group<T>;
+  using namespace simtdw;
+  __shared__ float Gs[T][BK][BD];
+  __shared__ __align__(16) float Xs[T][BK][BC];
+  const int tid = threadIdx.x;
+  const int tc = tid % 8, td = tid / 8;             // 4 c x 1 d per thread
+  const int c0 = blockIdx.x * BC, d0 = blockIdx.y * BD;
+  const int z = blockIdx.z;
+  const int64_t nbeg = (int64_t)z * tok_per_split;
+  int64_t nend = nbeg + tok_per_split;
+  if (nend > N) nend = N;
+
+  float acc[4][T];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int p = 0; p < T; ++p) acc[j][p] = 0.f;
+  float dbacc = 0.f;
+
+  for (int64_t nb = nbeg; nb < nend; nb += BK) {
+#pragma unroll
+    for (int r = 0; r < (BK * BD) / THREADS; ++r) {
+      const int q = tid + r * THREADS;
+      const int dd = q % BD, nn = q / BD;
+      const int64_t n = nb + nn;
+      const int d = d0 + dd;
+      float v[T], P[T];
+      if (n < nend && d < Dp) {
+        const E* src = gy + n * (int64_t)Dp * T + (int64_t)d * T;
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(src[t]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = 0.f;
+      }
+      G::dft(v, P);
+#pragma unroll
+      for (int p = 0; p < T; ++p) Gs[p][nn][dd] = P[p];
+    }
+#pragma unroll
+    for (int r = 0; r < (BK * BC) / THREADS; ++r) {
+      const int q = tid + r * THREADS;
+      const int cc = q % BC, nn = q / BC;
+      const int64_t n = nb + nn;
+      const int c = c0 + cc;
+      float v[T], P[T];
+      if (n < nend && c < Cp) {
+        const E* src = x + n * (int64_t)Cp * T + (int64_t)c * T;
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(src[t]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < T; ++t) v[t] = 0.f;
+      }
+      G::dft(v, P);
+#pragma unroll
+      for (int p = 0; p < T; ++p) Xs[p][nn][cc] = P[p];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float gv[T], xv[4][T];
+#pragma unroll
+      for (int p = 0; p < T; ++p) {
+        gv[p] = Gs[p][kk][td];
+        const float4 x4 = *reinterpret_cast<const float4*>(&Xs[p][kk][tc * 4]);
+        xv[0][p] = x4.x; xv[1][p] = x4.y; xv[2][p] = x4.z; xv[3][p] = x4.w;
+      }
+      dbacc += gv[0];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int f = 0; f < G::nreal; ++f) acc[j][f] = fmaf(gv[f], xv[j][f], acc[j][f]);
+#pragma unroll
+        for (int m = 0; m < G::ncomplex; ++m) {
+          const int pr = G::nreal + 2 * m, pi = pr + 1;
+          // G * conj(X)
+          acc[j][pr] = fmaf(gv[pr], xv[j][pr], acc[j][pr]);
+          acc[j][pr] = fmaf(gv[pi], xv[j][pi], acc[j][pr]);
+          acc[j][pi] = fmaf(gv[pi], xv[j][pr], acc[j][pi]);
+          acc[j][pi] = fmaf(-gv[pr], xv[j][pi], acc[j][pi]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const int d = d0 + td;
+  if (d >= Dp) return;
+  const int64_t plane = (int64_t)Cp * Dp;
+  float* base = part + (int64_t)z * T * plane;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = c0 + tc * 4 + j;
+    if (c >= Cp) continue;
+#pragma unroll
+    for (int p = 0; p < T; ++p) base[p * plane + (int64_t)d * Cp + c] = acc[j][p];
+  }
+  if (blockIdx.x == 0 && tc == 0) dbpart[(int64_t)z * Dp + d] = dbacc;
+}
+
+// Sum the splits in index order, then inverse DFT along the frequency planes.
+template <int T>
+__global__ void dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart,
+                                 float* __restrict__ dW, float* __restrict__ db, int splits,
+                                 int Cp, int Dp) {
+  using G = Group<T>;
+  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t plane = (int64_t)Cp * Dp;
+  if (idx < plane) {
+    float P[T], v[T];
+#pragma unroll
+    for (int p = 0; p < T; ++p) {
+      float s = 0.f;
+      for (int z = 0; z < splits; ++z) s += part[((int64_t)z * T + p) * plane + idx];
+      P[p] = s;
+    }
+    G::idft(P, v);
+    // idx = d*Cp + c, and dW is [Dp][Cp][T]
+#pragma unroll
+    for (int t = 0; t < T; ++t) dW[idx * T + t] = v[t];
+  }
+  if (db && idx < Dp) {
+    float s = 0.f;
+    for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + idx];
+    db[idx] = s;
+  }
+}
+
+template <int T, typename E>
+static cudaError_t simt_dw_t(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                             int64_t N, cudaStream_t st) {
+  using namespace simtdw;
+  const int splits = dw_splits(h.Cp, h.Dp, N);
+  const int64_t tps = ((N + splits - 1) / splits + BK - 1) / BK * BK;
+  const int64_t plane = h.Cp * h.Dp;
+  float* part = h.ws;
+  float* dbpart = h.ws + (int64_t)splits * T * plane;
+  if ((size_t)splits * ((size_t)T * plane + h.Dp) * sizeof(float) > h.ws_bytes)
+    return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((h.Cp + BC - 1) / BC), (unsigned)((h.Dp + BD - 1) / BD), (unsigned)splits);
+  simt_dw_kernel<T, E><<<grid, THREADS, 0, st>>>((const E*)x, (const E*)gy, part, dbpart, N,
+                                                 (int)h.Cp, (int)h.Dp, tps);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t work = plane > h.Dp ? plane : h.Dp;
+  dw_reduce_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(part, dbpart, dW, db, splits,
+                                                                      (int)h.Cp, (int)h.Dp);
+  return cudaGetLastError();
+}
+
+template <typename E>
+static cudaError_t simt_dw_e(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                             int64_t N, cudaStream_t st) {
+  switch (h.T) {
+    case 1: return simt_dw_t<1, E>(h, x, gy, dW, db, N, st);
+    case 2: return simt_dw_t<2, E>(h, x, gy, dW, db, N, st);
+    case 4: return simt_dw_t<4, E>(h, x, gy, dW, db, N, st);
+    case 8: return simt_dw_t<8, E>(h, x, gy, dW, db, N, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_simt_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                           int64_t N, cudaStream_t st) {
+  switch (h.dtype) {
+    case EQLIN_F32: return simt_dw_e<float>(h, x, gy, dW, db, N, st);
+    case EQLIN_F16: return simt_dw_e<__half>(h, x, gy, dW, db, N, st);
+    case EQLIN_BF16: return simt_dw_e<__nv_bfloat16>(h, x, gy, dW, db, N, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace eqlin

@@ -1,0 +1,147 @@
+/*
+ * eqlin.h -- C ABI of the Flash EQ-Linear library for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Flash EQ-Linear: Accelerating Equivariant Linear Layers via
+ * Group-wise Discrete Fourier Transform", abstract; technical summary of the
+ * same paper, section "Insight Central") is the equivariant linear layer whose
+ * weight is a group-circulant matrix: a circular convolution along the group
+ * axis composed with a linear map along channels.  With T the order of the
+ * cyclic group (T = 4 is the rotation group p4), C' input and D' output
+ * channels per group element:
+ *
+ *   y[n, d*T+s] = b[d] + sum_{c<C'} sum_{t<T} W[d, c, (s-t) mod T] * x[n, c*T+t]
+ *
+ * The library evaluates it the way the paper's section "Abordagem
+ * Algoritmica" describes: a real DFT along t, channel GEMMs for each
+ * frequency of the non-redundant half spectrum (six real GEMMs for p4,
+ * section "Especializacao para o Grupo de Rotacao p4"), then an inverse DFT,
+ * all inside its own CUDA kernels.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Layouts are row-major and contiguous:
+ *     x  [N, C'*T]  index c*T+t        y  [N, D'*T]  index d*T+s
+ *     gy [N, D'*T]  (dL/dy)            dx [N, C'*T]  (dL/dx)
+ *     W  [D', C', T]                   b  [D']
+ *     dW [D', C', T] float32           db [D'] float32
+ * - x, y, gy, dx, W and b have the handle's dtype; dW and db are float32.
+ * - Every tensor pointer is a DEVICE pointer owned by the caller, on the
+ *   device that was current when the handle was created.  It must be 16-byte
+ *   aligned, and every row of x, y, gy and dx must be a multiple of 16 bytes
+ *   (C'*T*elemsize and D'*T*elemsize), else EQLIN_ERR_MISALIGNED.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Calls are stream-ordered and asynchronous: they enqueue kernels
+ *   and return without synchronising.  Device-side failures (a bounded wait
+ *   that ran out) are recorded in the handle and read with eqlin_get_error()
+ *   after the caller has synchronised the stream.
+ * - N = 0 is a no-op that returns EQLIN_OK (dW and db are then zeroed).
+ * - Supported T: 1, 2, 4, 8.  Other values give EQLIN_ERR_UNSUPPORTED.
+ * - Nothing is thrown across the ABI; every call returns a status.
+ * - A handle may be used from one host thread at a time.
+ */
+#ifndef EQLIN_H
+#define EQLIN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EQLIN_API __attribute__((visibility("default")))
+#else
+#define EQLIN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EQLIN_F32 = 0,   /* float32 in/out; FP32 arithmetic (FFMA) */
+    EQLIN_F16 = 1,   /* float16 in/out; tensor cores, FP32 accumulation */
+    EQLIN_BF16 = 2   /* bfloat16 in/out; tensor cores, FP32 accumulation */
+} eqlin_dtype_t;
+
+typedef enum {
+    EQLIN_OK = 0,
+    EQLIN_ERR_INVALID_ARG = -1,  /* NULL handle/pointer, negative size, bad dtype */
+    EQLIN_ERR_UNSUPPORTED = -2,  /* T not in {1,2,4,8}, or a size beyond the limits */
+    EQLIN_ERR_MISALIGNED = -3,   /* pointer or row not 16-byte aligned */
+    EQLIN_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed */
+    EQLIN_ERR_NO_WEIGHTS = -5,   /* forward/backward before eqlin_set_weights */
+    EQLIN_ERR_TIMEOUT = -6,      /* a kernel's bounded wait ran out (device-side) */
+    EQLIN_ERR_OOM = -7           /* device allocation failed */
+} eqlin_status_t;
+
+typedef struct eqlin_handle *eqlin_t;
+
+/*
+ * Create a layer handle for group order T, C' = Cp input and D' = Dp output
+ * channels per group element, and the given dtype.  Allocates the handle's
+ * device buffers (Fourier-domain weights, bias, the dW reduction workspace and
+ * an error word) on the current device.  *out receives the handle.
+ * Limits: 1 <= Cp, Dp <= 65536 and Cp*T, Dp*T rows 16-byte multiples.
+ */
+EQLIN_API eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype,
+                            eqlin_t *out);
+
+/*
+ * Load weights: W [D', C', T] and b [D'] (b may be NULL: zero bias), device
+ * pointers of the handle's dtype.  Enqueues the weight pre-transform (the DFT
+ * of W along its group axis, the paper's Fourier-domain weights) on `stream`;
+ * W and b may be freed or overwritten once that work has run.  Must be called
+ * again after every weight update.
+ */
+EQLIN_API eqlin_status_t eqlin_set_weights(eqlin_t h, const void *W, const void *b, void *stream);
+
+/* Forward: y = EQ-Linear(x) + b.  x [N, C'*T] -> y [N, D'*T]. */
+EQLIN_API eqlin_status_t eqlin_forward(eqlin_t h, const void *x, void *y, int64_t N, void *stream);
+
+/*
+ * Input gradient: dx[n, c*T+t] = sum_d sum_s W[d, c, (s-t) mod T] gy[n, d*T+s].
+ * gy [N, D'*T] -> dx [N, C'*T]; dx is overwritten.
+ */
+EQLIN_API eqlin_status_t eqlin_backward_dx(eqlin_t h, const void *gy, void *dx, int64_t N,
+                                 void *stream);
+
+/*
+ * Weight and bias gradients over the N tokens:
+ *   dW[d, c, tau] = sum_n sum_s gy[n, d*T+s] x[n, c*T + (s-tau) mod T]
+ *   db[d]         = sum_n sum_s gy[n, d*T+s]
+ * dW [D', C', T] and db [D'] are float32 and OVERWRITTEN (not accumulated);
+ * db may be NULL.  Uses the handle's workspace; the reduction is
+ * deterministic (fixed order, no atomics).
+ */
+EQLIN_API eqlin_status_t eqlin_backward_dw(eqlin_t h, const void *x, const void *gy, float *dW,
+                                 float *db, int64_t N, void *stream);
+
+/*
+ * Read and clear the handle's device-side error word.  Call after
+ * synchronising the streams the handle's kernels ran on.  Returns EQLIN_OK,
+ * EQLIN_ERR_TIMEOUT (a kernel's bounded wait ran out and the kernel returned
+ * early: its outputs are invalid) or EQLIN_ERR_CUDA.
+ */
+EQLIN_API eqlin_status_t eqlin_get_error(eqlin_t h);
+
+/*
+ * Cap, in polling iterations, on every wait inside this handle's kernels
+ * (0 restores the default).  A wait that reaches the cap records
+ * EQLIN_ERR_TIMEOUT and its kernel returns early instead of spinning.
+ */
+EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
+
+/*
+ * Which kernel family serves each call of this handle, as a short string
+ * (e.g. "tcgen05" or "simt"); for logging and tests.
+ */
+EQLIN_API const char *eqlin_backend_name(eqlin_t h);
+
+/* Static description of a status code. */
+EQLIN_API const char *eqlin_status_string(eqlin_status_t s);
+
+/* Free the handle and its device buffers (synchronises the device first).  NULL is a no-op. */
+EQLIN_API void eqlin_destroy(eqlin_t h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQLIN_H */

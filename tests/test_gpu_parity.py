@@ -1,0 +1,194 @@
+"""GPU parity: the CUDA library against the CPU oracle on the same seeded inputs.
+
+Tolerances (relative Frobenius norm of the difference, i.e. RMS(err)/RMS(ref)):
+FP32 1e-5; FP16/BF16 with FP32 accumulation 2e-2.  Integer-valued inputs
+whose every intermediate is exactly representable must match bit for bit
+(T in {1, 2, 4}: the p4 and T=2 transforms use only +-1 and +-1/2, +-1/4).
+
+Small cases span several 128-token tiles with a ragged tail; full-size cases
+use the benchmark's shapes and launch path and compare sampled rows (forward,
+dx) and sampled (d, c) weight pairs (dW) against the oracle, plus the
+equivariance property on the whole output.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_circulant_linear_b200 import eqlin, inputs, workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
+
+
+def rel_err(out, ref) -> float:
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(out - ref) / (den if den > 0 else 1.0))
+
+
+def _dev(d):
+    return {k: v.cuda() for k, v in d.items()}
+
+
+def _run_all(T, Cp, Dp, dt, inp, passes=("fwd", "dx", "dw")):
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    out = {}
+    if "fwd" in passes:
+        out["y"] = layer.forward(g["x"])
+    if "dx" in passes:
+        out["dx"] = layer.backward_dx(g["gy"])
+    if "dw" in passes:
+        out["dW"], out["db"] = layer.backward_dw(g["x"], g["gy"])
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    return layer, {k: v.float().cpu().numpy() for k, v in out.items()}
+
+
+SMALL = [  # (T, C', D', N, dtype)
+    (4, 16, 16, 256, "f32"),        # p4 tiny forward
+    (4, 96, 288, 333, "f16"),       # EQ-ViT-S qkv-like, ragged N
+    (4, 96, 96, 300, "f16"),        # EQ-ViT-S proj-like
+    (4, 192, 768, 300, "bf16"),     # EQ-ViT-B fc1-like
+    (4, 768, 192, 260, "bf16"),     # EQ-ViT-B fc2-like
+    (4, 24, 96, 1000, "f16"),       # EQ-Swin-T stage-1 fc1-like
+    (4, 96, 24, 1000, "f16"),       # EQ-Swin-T stage-1 fc2-like
+    (2, 64, 64, 257, "f32"), (4, 64, 64, 257, "f32"), (8, 32, 32, 257, "f32"),
+    (2, 64, 64, 257, "f16"), (4, 64, 64, 257, "f16"), (8, 32, 32, 257, "f16"),
+    (1, 64, 48, 200, "f32"), (1, 64, 48, 200, "bf16"),
+    (8, 64, 16, 130, "bf16"), (2, 40, 72, 129, "bf16"),
+    (4, 8, 8, 1, "f16"), (4, 200, 40, 131, "f16"),
+]
+
+
+@pytest.mark.parametrize("T,Cp,Dp,N,dt", SMALL, ids=lambda v: str(v))
+def test_small_parity(T, Cp, Dp, N, dt):
+    inp = inputs.make_inputs(T, Cp, Dp, N, dt, seed=0)
+    _, out = _run_all(T, Cp, Dp, dt, inp)
+    y = oracle.forward(inp["x"], inp["W"], inp["b"])
+    dx = oracle.backward_dx(inp["gy"], inp["W"])
+    dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
+    tol = TOL[dt]
+    assert rel_err(out["y"], y) <= tol
+    assert rel_err(out["dx"], dx) <= tol
+    assert rel_err(out["dW"], dW) <= tol
+    assert rel_err(out["db"], db) <= tol
+
+
+EXACT = [  # (T, C', D', N, dtype, amp): every intermediate exactly representable
+    (4, 64, 64, 1024, "f32", 4), (2, 64, 48, 515, "f32", 4), (1, 32, 64, 300, "f32", 4),
+    (4, 16, 16, 700, "f16", 4), (2, 16, 16, 300, "f16", 4), (4, 16, 8, 129, "f16", 4),
+    (4, 8, 8, 400, "bf16", 2), (2, 8, 8, 200, "bf16", 2),
+]
+
+
+@pytest.mark.parametrize("T,Cp,Dp,N,dt,amp", EXACT, ids=lambda v: str(v))
+def test_integer_inputs_bit_exact(T, Cp, Dp, N, dt, amp):
+    inp = inputs.make_integer_inputs(T, Cp, Dp, N, dt, seed=3, amp=amp)
+    _, out = _run_all(T, Cp, Dp, dt, inp)
+    y = oracle.forward(inp["x"], inp["W"], inp["b"])
+    dx = oracle.backward_dx(inp["gy"], inp["W"])
+    dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
+    assert np.array_equal(out["y"], y)
+    assert np.array_equal(out["dx"], dx)
+    assert np.array_equal(out["dW"], dW)
+    assert np.array_equal(out["db"], db)
+
+
+def _roll(a: torch.Tensor, ch: int, T: int, r: int) -> torch.Tensor:
+    N = a.shape[0]
+    return torch.roll(a.reshape(N, ch, T), r, dims=2).reshape(N, ch * T).contiguous()
+
+
+FULL = [(name, i) for name, layers in workloads.WORKLOADS.items() for i in range(len(layers))]
+
+
+@pytest.mark.parametrize("name,idx", FULL, ids=lambda v: str(v))
+def test_full_size_sampled(name, idx):
+    L = workloads.WORKLOADS[name][idx]
+    T, Cp, Dp, N, dt = L.T, L.Cp, L.Dp, L.N, L.dtype
+    inp = inputs.make_inputs(T, Cp, Dp, N, dt, seed=0, with_gy=("dx" in L.passes or "dw" in L.passes))
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, 62)]))
+    tol = TOL[dt]
+    y = layer.forward(g["x"])
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    assert rel_err(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
+                   oracle.forward(inp["x"], inp["W"], inp["b"], rows=rows)) <= tol
+    # equivariance on the whole output: rotate the group axis of x by one step
+    yr = layer.forward(_roll(g["x"], Cp, T, 1))
+    assert rel_err(yr.float().cpu().numpy(), _roll(y, Dp, T, 1).float().cpu().numpy()) <= tol
+    if "dx" in L.passes:
+        dx = layer.backward_dx(g["gy"])
+        torch.cuda.synchronize()
+        assert rel_err(dx[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
+                       oracle.backward_dx(inp["gy"], inp["W"], rows=rows)) <= tol
+    if "dw" in L.passes:
+        dW, db = layer.backward_dw(g["x"], g["gy"])
+        torch.cuda.synchronize()
+        pairs = np.stack([rng.integers(0, Dp, 48), rng.integers(0, Cp, 48)], 1)
+        want, want_db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp, pairs=pairs)
+        got = dW.cpu().numpy()[pairs[:, 0], pairs[:, 1]]
+        assert rel_err(got, want) <= tol
+        assert rel_err(db.cpu().numpy(), want_db) <= tol
+    assert eqlin.get_error(layer.h) == 0
+
+
+# ------------------------------------------------------------- error paths
+
+def test_error_paths():
+    T, Cp, Dp = 4, 16, 16
+    h = eqlin.create(T, Cp, Dp, "f16")
+    x = torch.zeros((10, Cp * T), dtype=torch.float16, device="cuda")
+    y = torch.zeros((10, Dp * T), dtype=torch.float16, device="cuda")
+    L = eqlin.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    vp = ctypes.c_void_p
+    # before set_weights
+    assert L.eqlin_forward(h.ptr, vp(x.data_ptr()), vp(y.data_ptr()), 10, vp(s)) == -5
+    W = torch.randn((Dp, Cp, T), device="cuda").half()
+    eqlin.set_weights(h, W, None)
+    # misaligned pointers
+    assert L.eqlin_forward(h.ptr, vp(x.data_ptr() + 2), vp(y.data_ptr()), 9, vp(s)) == -3
+    assert L.eqlin_forward(h.ptr, vp(x.data_ptr()), vp(y.data_ptr() + 8), 9, vp(s)) == -3
+    # negative N, null pointers
+    assert L.eqlin_forward(h.ptr, vp(x.data_ptr()), vp(y.data_ptr()), -1, vp(s)) == -1
+    assert L.eqlin_forward(h.ptr, None, vp(y.data_ptr()), 10, vp(s)) == -1
+    # N = 0 is a no-op; dW/db are zeroed
+    assert L.eqlin_forward(h.ptr, None, None, 0, vp(s)) == 0
+    dW = torch.full((Dp, Cp, T), 7.0, device="cuda")
+    db = torch.full((Dp,), 7.0, device="cuda")
+    assert L.eqlin_backward_dw(h.ptr, None, None, vp(dW.data_ptr()), vp(db.data_ptr()), 0, vp(s)) == 0
+    torch.cuda.synchronize()
+    assert not dW.any() and not db.any()
+    # wrong dtype / shape are rejected by the binding
+    with pytest.raises(TypeError):
+        eqlin.forward(h, x.float(), y)
+    with pytest.raises(ValueError):
+        eqlin.forward(h, x[:, :8].contiguous(), y)
+    assert eqlin.get_error(h) == 0
+    h.close()
+
+
+def test_outputs_have_no_stray_writes():
+    """Canary rows around the output stay untouched (ragged N, odd D')."""
+    T, Cp, Dp, N = 4, 96, 40, 133
+    inp = _dev(inputs.make_inputs(T, Cp, Dp, N, "bf16", seed=2))
+    layer = eqlin.EQLinear(inp["W"], inp["b"])
+    buf = torch.full((N + 64, Dp * T), 123.0, dtype=torch.bfloat16, device="cuda")
+    eqlin.forward(layer.h, inp["x"], buf[32:32 + N])
+    dxb = torch.full((N + 64, Cp * T), 123.0, dtype=torch.bfloat16, device="cuda")
+    eqlin.backward_dx(layer.h, inp["gy"], dxb[32:32 + N])
+    torch.cuda.synchronize()
+    assert (buf[:32] == 123).all() and (buf[32 + N:] == 123).all()
+    assert (dxb[:32] == 123).all() and (dxb[32 + N:] == 123).all()
+    assert not (buf[32:32 + N] == 123).all()
