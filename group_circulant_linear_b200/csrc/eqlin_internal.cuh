@@ -134,7 +134,8 @@ struct Handle {
 // Device error codes written into Handle::err (first writer wins).
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 
-constexpr uint32_t kDefaultWaitLimit = 1u << 26;   // polls; ~seconds at worst
+// Default poll cap of a wait; the wall-time cap (2 s per wait) binds first.
+constexpr uint32_t kDefaultWaitLimit = 0xFFFFFFFFu;
 
 // ------------------------------------------------------- launch wrappers
 // SIMT path (any T in {1,2,4,8}, any dtype).

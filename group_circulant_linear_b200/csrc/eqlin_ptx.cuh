@@ -45,10 +45,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed; false after `limit` polls.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Upper bound on the wall time of any single wait, whatever the poll limit.
+constexpr uint64_t kWaitTimeNs = 2000000000ull;
+
+// Wait until the phase with the given parity has completed; false after
+// `limit` polls or kWaitTimeNs, whichever comes first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
+  uint64_t t0 = 0;
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 15u) {
+      const uint64_t t = globaltimer_ns();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > kWaitTimeNs) return false;
+    }
+  }
   return false;
 }
 

@@ -192,3 +192,35 @@ def test_outputs_have_no_stray_writes():
     assert (buf[:32] == 123).all() and (buf[32 + N:] == 123).all()
     assert (dxb[:32] == 123).all() and (dxb[32 + N:] == 123).all()
     assert not (buf[32:32 + N] == 123).all()
+
+
+def test_tensor_core_backend_is_used():
+    """f16/bf16 handles with 8-aligned channel counts run the tcgen05 kernels."""
+    for dt in ("f16", "bf16"):
+        for T in (1, 2, 4, 8):
+            h = eqlin.create(T, 64, 64, dt)
+            assert h.backend() == "tcgen05", (T, dt, h.backend())
+            h.close()
+    assert eqlin.create(4, 16, 16, "f32").backend() == "simt"
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait cap of one poll makes the kernel give up, record EQLIN_ERR_TIMEOUT
+    and return; with the default cap the same handle then computes correctly."""
+    T, Cp, Dp, N = 4, 768, 192, 4096
+    inp = inputs.make_inputs(T, Cp, Dp, N, "bf16", seed=4)
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    assert layer.h.backend() == "tcgen05"
+    eqlin.set_wait_limit(layer.h, 1)
+    layer.forward(g["x"])
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == -6
+    assert eqlin.get_error(layer.h) == 0          # reading clears it
+    eqlin.set_wait_limit(layer.h, 0)
+    y = layer.forward(g["x"])
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    rows = np.arange(0, N, 97)
+    assert rel_err(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
+                   oracle.forward(inp["x"], inp["W"], inp["b"], rows=rows)) <= TOL["bf16"]
