@@ -5,11 +5,17 @@
 // eqlin_get_error (which reads the device error word) and eqlin_destroy.
 #include <stdlib.h>
 #include <string.h>
+#include <atomic>
 #include <new>
 
 #include "eqlin_internal.cuh"
 
 using eqlin::Handle;
+
+namespace eqlin {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace eqlin
 
 struct eqlin_handle {
   Handle h;
@@ -101,6 +107,10 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
   const size_t planes = (size_t)T * Cp * Dp;
   const int Q = (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
+  if (dtype != EQLIN_F32) {
+    const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
+    if (tcb > h.ws_bytes) h.ws_bytes = tcb;
+  }
   bool ok = cudaMalloc(&h.wf_fwd, planes * 4) == cudaSuccess &&
             cudaMalloc(&h.wf_bwd, planes * 4) == cudaSuccess &&
             cudaMalloc(&h.bias, (size_t)Dp * 4) == cudaSuccess &&
@@ -187,7 +197,9 @@ eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, floa
   }
   eqlin_status_t s = check_io(h, x, gy, N);
   if (s != EQLIN_OK) return s;
-  cudaError_t e = eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
+  cudaError_t e = eqlin::tc_dw_supported(h)
+                      ? eqlin::launch_tc_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
+                      : eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }
 
@@ -212,5 +224,7 @@ eqlin_status_t eqlin_set_wait_limit(eqlin_t hh, uint32_t iterations) {
 }
 
 const char* eqlin_backend_name(eqlin_t hh) { return hh ? hh->h.backend : "none"; }
+
+uint64_t eqlin_launch_count(void) { return eqlin::g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

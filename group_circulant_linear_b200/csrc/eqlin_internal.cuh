@@ -137,6 +137,9 @@ enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 // Default poll cap of a wait; the wall-time cap (2 s per wait) binds first.
 constexpr uint32_t kDefaultWaitLimit = 0xFFFFFFFFu;
 
+// Count kernels enqueued by this library (reported by eqlin_launch_count).
+void count_launches(int n);
+
 // ------------------------------------------------------- launch wrappers
 // SIMT path (any T in {1,2,4,8}, any dtype).
 cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st);
@@ -145,11 +148,19 @@ cudaError_t launch_simt_apply(const Handle& h, bool backward, const void* in, vo
 cudaError_t launch_simt_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
                            int64_t N, cudaStream_t st);
 size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp);
+// Sum per-split partial Fourier planes [splits][T][Dp][Cp] (+ db partials
+// [splits][Dp]) in split order and apply the inverse DFT -> dW [Dp][Cp][T].
+cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
+                             float* dW, float* db, cudaStream_t st);
 
 // tcgen05 path (f16/bf16).  Returns cudaErrorNotSupported when the shape is
 // outside what the kernel handles, so the caller can fall back to SIMT.
 bool tc_supported(const Handle& h, bool backward);
 cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out,
                             int64_t N, cudaStream_t st);
+bool tc_dw_supported(const Handle& h);
+size_t tc_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);
+cudaError_t launch_tc_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                         int64_t N, cudaStream_t st);
 
 }  // namespace eqlin

@@ -74,6 +74,7 @@ static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b,
   pretransform_kernel<T, E><<<blocks, threads, 0, st>>>(
       (const E*)W, (const E*)b, h.wf_fwd, h.wf_bwd, (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias,
       (int)h.Cp, (int)h.Dp);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -213,6 +214,7 @@ static cudaError_t simt_apply_t(const Handle& h, bool backward, const void* in, 
   dim3 grid((unsigned)tiles_n, (unsigned)((O + simt::BO - 1) / simt::BO));
   simt_apply_kernel<T, E><<<grid, simt::THREADS, 0, st>>>(
       (const E*)in, backward ? h.wf_bwd : h.wf_fwd, backward ? nullptr : h.bias, (E*)out, N, K, O);
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -411,10 +413,30 @@ static cudaError_t simt_dw_t(const Handle& h, const void* x, const void* gy, flo
                                                  (int)h.Cp, (int)h.Dp, tps);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  count_launches(1);
+  return launch_dw_reduce(h, splits, part, dbpart, dW, db, st);
+}
+
+template <int T>
+static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
+                               float* dW, float* db, cudaStream_t st) {
+  const int64_t plane = h.Cp * h.Dp;
   const int64_t work = plane > h.Dp ? plane : h.Dp;
   dw_reduce_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(part, dbpart, dW, db, splits,
                                                                       (int)h.Cp, (int)h.Dp);
+  count_launches(1);
   return cudaGetLastError();
+}
+
+cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
+                             float* dW, float* db, cudaStream_t st) {
+  switch (h.T) {
+    case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, st);
+    case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, st);
+    case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, st);
+    case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <typename E>

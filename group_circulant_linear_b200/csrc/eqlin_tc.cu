@@ -476,6 +476,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
   tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_w, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 

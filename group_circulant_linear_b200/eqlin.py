@@ -38,6 +38,7 @@ SIGNATURES = {
     "eqlin_set_wait_limit": ([_vp, _u32], _int),
     "eqlin_backend_name": ([_vp], ctypes.c_char_p),
     "eqlin_status_string": ([_int], ctypes.c_char_p),
+    "eqlin_launch_count": ([], ctypes.c_uint64),
     "eqlin_destroy": ([_vp], None),
 }
 
@@ -164,6 +165,11 @@ def get_error(h: Handle) -> int:
 
 def set_wait_limit(h: Handle, iterations: int):
     _check(lib().eqlin_set_wait_limit(h.ptr, int(iterations)), "eqlin_set_wait_limit")
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process (all handles)."""
+    return int(lib().eqlin_launch_count())
 
 
 def status_string(status: int) -> str:

@@ -134,6 +134,12 @@ EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
  */
 EQLIN_API const char *eqlin_backend_name(eqlin_t h);
 
+/*
+ * Number of CUDA kernels this library has enqueued in this process, over all
+ * handles (a monotonically increasing counter, for accounting).
+ */
+EQLIN_API uint64_t eqlin_launch_count(void);
+
 /* Static description of a status code. */
 EQLIN_API const char *eqlin_status_string(eqlin_status_t s);
 
