@@ -39,6 +39,7 @@ SIGNATURES = {
     "eqlin_backend_name": ([_vp], ctypes.c_char_p),
     "eqlin_status_string": ([_int], ctypes.c_char_p),
     "eqlin_launch_count": ([], ctypes.c_uint64),
+    "eqlin_backward_dw_noalloc": ([_int, _i64, _i64, _int, _vp, _vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_destroy": ([_vp], None),
 }
 
@@ -156,6 +157,19 @@ def backward_dw(h: Handle, x: torch.Tensor, gy: torch.Tensor, dW: torch.Tensor,
     pw = _dev_ptr(dW, torch.float32, (h.Dp, h.Cp, h.T), "dW")
     pb = None if db is None else _dev_ptr(db, torch.float32, (h.Dp,), "db")
     _check(lib().eqlin_backward_dw(h.ptr, px, pg, pw, pb, N, _stream(stream)), "eqlin_backward_dw")
+
+
+def backward_dw_noalloc(T: int, x: torch.Tensor, gy: torch.Tensor, dW: torch.Tensor,
+                        db: torch.Tensor | None = None, stream=None):
+    """dW/db with no handle and no device allocation (see eqlin_backward_dw_noalloc)."""
+    Dp, Cp = dW.shape[0], dW.shape[1]
+    N = x.shape[0]
+    px = _dev_ptr(x, x.dtype, (N, Cp * T), "x")
+    pg = _dev_ptr(gy, x.dtype, (N, Dp * T), "gy")
+    pw = _dev_ptr(dW, torch.float32, (Dp, Cp, T), "dW")
+    pb = None if db is None else _dev_ptr(db, torch.float32, (Dp,), "db")
+    _check(lib().eqlin_backward_dw_noalloc(T, Cp, Dp, _DT[x.dtype], px, pg, pw, pb, N, _stream(stream)),
+           "eqlin_backward_dw_noalloc")
 
 
 def get_error(h: Handle) -> int:

@@ -114,6 +114,42 @@ EQLIN_API eqlin_status_t eqlin_backward_dw(eqlin_t h, const void *x, const void 
                                  float *db, int64_t N, void *stream);
 
 /*
+ * dW and db without a handle and without any device allocation.
+ *
+ * For callers that cannot call cudaMalloc -- code that runs while another
+ * allocator owns the device memory, runtimes that forbid allocation after
+ * start-up, plug-ins inside a host that manages memory itself.  They cannot
+ * create an eqlin_t, but the weight gradient needs no weights, so this call
+ * takes the layer shape directly.  The paper has no counterpart; it is a
+ * service of this library.
+ *
+ * Same arguments and results as eqlin_backward_dw (T, C' = Cp, D' = Dp and
+ * the dtype describe the layer; x [N, C'*T], gy [N, D'*T] device pointers of
+ * that dtype; dW [D', C', T] and db [D'] float32, overwritten; db may be
+ * NULL), computed by the same tensor-core kernels.  f16 and bf16 only
+ * (EQLIN_ERR_UNSUPPORTED for f32).
+ *
+ * Scratch: a fixed 64 MiB device array inside the library, reserved on a
+ * device when the library's code first loads there and held until the
+ * process exits.  A shape whose per-chunk partial sums would not fit returns
+ * EQLIN_ERR_UNSUPPORTED (the need is splits * (T*C'*D' + D') * 4 bytes, with
+ * up to one token split per SM for a single 128 x 128 channel tile; e.g. p4
+ * with C' = D' = 1024 fits, C' = D' = 2048 does not).
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - Every call on a device shares the array, so calls that may overlap on
+ *   the GPU (different streams, or concurrent host threads) race and give
+ *   wrong results: order them on one stream.
+ * - A device-side wait that runs out (only if the GPU stalls for seconds)
+ *   leaves dW and db undefined; there is no handle to report it through.
+ * The call itself allocates nothing and frees nothing.
+ */
+EQLIN_API eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t Dp,
+                                                   eqlin_dtype_t dtype, const void *x,
+                                                   const void *gy, float *dW, float *db,
+                                                   int64_t N, void *stream);
+
+/*
  * Read and clear the handle's device-side error word.  Call after
  * synchronising the streams the handle's kernels ran on.  Returns EQLIN_OK,
  * EQLIN_ERR_TIMEOUT (a kernel's bounded wait ran out and the kernel returned
