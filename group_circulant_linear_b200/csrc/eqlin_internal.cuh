@@ -87,6 +87,27 @@ template <int T> struct Group {
     }
   }
 
+  // Inverse real DFT of planes that already carry the scales 1/T (real
+  // frequencies) and 2/T (complex ones): v_s = P0 + (-1)^s P1 + sum_k
+  // (Re_k cos - Im_k sin), plus `add` on every output.
+  static __host__ __device__ __forceinline__ void idft_scaled(const float* P, float add, float* v) {
+    const float a = P[0] + add;
+    if (T == 1) { v[0] = a; return; }
+    const float ep = a + P[1], em = a - P[1];      // even / odd s
+#pragma unroll
+    for (int s_ = 0; s_ < T; ++s_) {
+      float acc = (s_ & 1) ? em : ep;
+#pragma unroll
+      for (int k = 1; k <= ncomplex; ++k) {
+        const float cs = c(k, s_), sn = s(k, s_);
+        const float re = P[nreal + 2 * (k - 1)], im = P[nreal + 2 * (k - 1) + 1];
+        if (cs != 0.f) acc += (cs == 1.f ? re : cs == -1.f ? -re : cs * re);
+        if (sn != 0.f) acc -= (sn == 1.f ? im : sn == -1.f ? -im : sn * im);
+      }
+      v[s_] = acc;
+    }
+  }
+
   // Inverse real DFT of planes P into v[0..T), including the 1/T.
   static __host__ __device__ __forceinline__ void idft(const float* P, float* v) {
 #pragma unroll

@@ -21,7 +21,8 @@ namespace eqlin {
 //   wf_fwd[p][c][d]  (FP32, forward planes)
 //   wf_bwd[p][d][c]  (FP32, conjugated: the dx product uses conj(W_hat))
 //   wt_fwd[q][d][c], wt_bwd[q][c][d]  (handle dtype, tensor-core operand
-//   planes; q enumerates real frequencies, then (-Im, Re, Im) triples)
+//   planes scaled by 1/T (real) or 2/T (complex); q enumerates real
+//   frequencies, then (-Im, Re, Im) triples)
 template <int T, typename E>
 __global__ void pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b,
                                     float* __restrict__ wf_fwd, float* __restrict__ wf_bwd,
@@ -45,14 +46,18 @@ __global__ void pretransform_kernel(const E* __restrict__ W, const E* __restrict
     wf_bwd[p * plane + (int64_t)d * Cp + c] = imag ? -P[p] : P[p];
   }
   if (wt_fwd) {
+    // The tensor-core planes carry the inverse DFT's scales (1/T for a real
+    // frequency, 2/T for a complex one; exact powers of two), so that the
+    // kernels' epilogue is only additions.
+    const float sr = 1.f / T, sc = 2.f / T;
 #pragma unroll
     for (int f = 0; f < G::nreal; ++f) {
-      wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f]);
-      wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f]);
+      wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f] * sr);
+      wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f] * sr);
     }
 #pragma unroll
     for (int k = 1; k <= G::ncomplex; ++k) {
-      const float re = P[G::nreal + 2 * (k - 1)], im = P[G::nreal + 2 * (k - 1) + 1];
+      const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
       const int q = G::nreal + 3 * (k - 1);
       // forward: (-Im, Re, Im); backward uses conj(W_hat): Im -> -Im
       wt_fwd[(q + 0) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(-im);

@@ -2,29 +2,34 @@
 // forward pass and the input gradient, f16/bf16 in, f32 accumulation.
 //
 // One persistent CTA per SM walks output tiles of 128 tokens x BO output
-// channels (all T group positions).  Per tile and per K stage of BK input
+// channels (all T group positions).  Per tile and per K stage of 16 input
 // channels:
 //
-//   producer warp     TMA: the raw input tile [128 x BK*T] (128B swizzle) and
-//                     the Fourier weight planes of the stage
-//   transform warps   one thread per token row: DFT along t of the raw row
-//                     (adds/subtracts; +-sqrt(2)/2 for T = 8), one rounding to
-//                     the operand dtype, written as T K-major swizzled operand
-//                     planes; then a generic->async proxy fence
-//   MMA warp          one thread issues tcgen05.mma into TMEM: for each real
-//                     frequency one M=128, N=BO product; for each complex
-//                     frequency two M=128, N=2*BO products that accumulate
-//                     [Re Y | Im Y] = Re X [Re W ; Im W] + Im X [-Im W ; Re W]
-//                     -- R(T) real GEMMs, six for p4
-//   epilogue warps    tcgen05.ld of the frequency planes, inverse DFT with the
-//                     1/T, bias, cast, 16-byte stores of y[n, d*T+s]
+//   producer warp    (8)    TMA: the raw input tile of the stage [128 tokens x
+//                    16*T elements], the Fourier weight planes of the stage,
+//                    and L2 prefetches of raw tiles several stages ahead
+//   transform warps  (0-7)  one thread per (input channel, 8 tokens): read the
+//                    channel's T group values of its tokens from the raw tile,
+//                    take the group DFT (adds/subtracts on packed token pairs
+//                    for T <= 4, FP32 with the sqrt(2)/2 twiddles for T = 8)
+//                    and write the T frequency planes as token-contiguous
+//                    (MN-major, 128B-swizzled) MMA operands; then a
+//                    generic->async proxy fence
+//   MMA warp         (9)    one thread issues tcgen05.mma into TMEM: for each
+//                    real frequency one M=128, N=BO product; for each complex
+//                    frequency two M=128, N=2*BO products that accumulate
+//                    [Re Y | Im Y] = Re X [Re W ; Im W] + Im X [-Im W ; Re W]
+//                    -- R(T) real GEMMs, six for p4
+//   epilogue warps   (10-17) tcgen05.ld of the frequency planes, inverse DFT
+//                    (the weight planes carry its 1/T and 2/T scales, so this
+//                    is additions only), bias, cast into a 128B-swizzled
+//                    staging tile, TMA store of 64 output elements x 128 rows
 //
 // ("Flash EQ-Linear", technical summary, sections "Abordagem Algoritmica",
 // "Especializacao para o Grupo de Rotacao p4" and "Implementacao": fused data
-// flow, Fourier fragments kept on chip, tensor cores.)  The accumulators are
-// double-buffered in TMEM so the epilogue of one tile overlaps the main loop
-// of the next.  The input gradient uses the same kernel with the conjugated,
-// transposed weight planes and no bias.
+// flow, Fourier fragments kept on chip, tensor cores.)  The input gradient
+// runs the same kernel with the conjugated, transposed weight planes and no
+// bias.
 //
 // Every mbarrier wait is bounded.  A wait that runs out records a timeout in
 // the handle's error word, raises a CTA-wide abort flag, and the kernel
@@ -34,6 +39,7 @@
 #include <type_traits>
 
 #include "eqlin_internal.cuh"
+#include "eqlin_packed.cuh"
 #include "eqlin_ptx.cuh"
 
 namespace eqlin {
@@ -45,36 +51,44 @@ template <int T>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
-  static constexpr int RAW_EL = 128;                   // raw input elements per row per stage
-  static constexpr int BK = RAW_EL / T;                // input channels per stage
-  static constexpr int ROWB = (BK * 2 >= 128) ? 128 : BK * 2;   // operand row bytes = swizzle span
-  static constexpr int KATOMS = BK * 2 / ROWB;         // swizzle atoms along K (2 for T = 1)
-  static constexpr int KSTEPS = BK / 16;               // MMA K = 16 steps per stage
-  static constexpr int BO = (256 / T) < 128 ? (256 / T) : 128;   // output channels per tile
-  static constexpr int Q = G::nreal + 3 * G::ncomplex; // weight planes per stage
-  static constexpr int ACC_COLS = T * BO;              // f32 accumulator columns per tile
-  static constexpr int NACC = 2;                       // accumulator buffers
+  static constexpr int BK = 16;                        // input channels per stage (one MMA K step)
+  // output channels per tile and accumulator buffers: T * BO * NACC <= 512 columns
+  static constexpr int BO = T == 1 ? 256 : T == 2 ? 128 : T == 4 ? 128 : 32;
+  static constexpr int NACC = (T * BO * 2 <= 512) ? 2 : 1;
+  static constexpr int ACC_COLS = T * BO;
   static constexpr int TMEM_COLS = NACC * ACC_COLS <= 256 ? 256 : 512;
-  static constexpr int RAW_SLOTS = 2;
-  static constexpr int RAW_BOX_BYTES = BM * 128;       // one 64-element box of 128 rows
-  static constexpr int RAW_BYTES = 2 * RAW_BOX_BYTES;
-  static constexpr int A_PLANE_BYTES = BM * BK * 2;
+  static constexpr int Q = G::nreal + 3 * G::ncomplex; // weight planes per stage
+  // raw input tile of a stage: 128 tokens x (16 channels x T) elements, row-major (TMA)
+  static constexpr int RAW_ROWB = BK * T * 2;
+  static constexpr int RAW_BYTES = BM * RAW_ROWB;
+  // A: MN-major, 128B swizzle: 64-token blocks (LBO apart) of 8-channel groups (SBO apart)
+  static constexpr int A_SBO = 1024;
+  static constexpr int A_LBO = (BK / 8) * A_SBO;       // 2048
+  static constexpr int A_PLANE_BYTES = BM * BK * 2;    // 4 KB
   static constexpr int A_BYTES = T * A_PLANE_BYTES;
-  static constexpr int B_PLANE_BYTES = BO * BK * 2;
+  // B: K-major, 32-byte rows (16 channels), 32B swizzle
+  static constexpr int B_ROWB = BK * 2;
+  static constexpr int B_PLANE_BYTES = BO * B_ROWB;
   static constexpr int B_BYTES = Q * B_PLANE_BYTES;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BUDGET = 224 * 1024;
-  static constexpr int STAGES_FIT = (SMEM_BUDGET - RAW_SLOTS * RAW_BYTES - 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  static_assert(STAGES >= 2, "shared memory too small for two stages");
-  static constexpr int NBAR = 2 * RAW_SLOTS + 3 * STAGES + 2 * NACC + 1;
-  static constexpr int SMEM_BYTES =
-      RAW_SLOTS * RAW_BYTES + STAGES * STAGE_BYTES + NBAR * 8 + 16 + 1024 /*alignment slack*/;
-  // swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> SW_SHIFT) & SW_MASK)
-  static constexpr int SW_BITS = ROWB == 128 ? 3 : ROWB == 64 ? 2 : 1;
-  static constexpr int SW_SHIFT = 3 - SW_BITS;
-  static constexpr int SW_MASK = (1 << SW_BITS) - 1;
-  static constexpr int THREADS = 320;                  // producer, MMA, 4 transform, 4 epilogue warps
+  static constexpr int STAGE_BYTES = RAW_BYTES + A_BYTES + B_BYTES;
+  // output staging for the TMA stores: per epilogue half one [128 rows x 128 B] tile
+  static constexpr int OUT_EL = 64;                    // output elements per row per store
+  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2;
+  static constexpr int STAGES_FIT = (220 * 1024 - 2 * OUT_TILE_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static_assert(STAGES >= 2, "two stages must fit");
+  static constexpr int NBAR = 5 * STAGES + 2 * NACC + 1;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * OUT_TILE_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int CH = OUT_EL / T;                // output channels per store chunk
+  static constexpr int NCHUNK = BO / CH;               // store chunks per tile (even)
+  static_assert(NCHUNK % 2 == 0, "chunks alternate between the two epilogue halves");
+  // roles
+  static constexpr int TR_WARPS = 8;                   // transform: 8 tokens x 16 channels per warp-half
+  static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1, EPI0 = TR_WARPS + 2;
+  static constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter
+  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+  static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
+  static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
 };
 
 struct Params {
@@ -83,8 +97,8 @@ struct Params {
   int O;           // output channels per group element
   int n_otiles;
   int64_t n_tiles;
+  const void* in;
   const float* bias;   // nullptr: none
-  void* out;
   int* err;
   uint32_t wait_limit;
   uint32_t ab_fmt;     // 0 f16, 1 bf16
@@ -106,23 +120,27 @@ __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t l
   return false;
 }
 
-// Every lane polls (each needs the acquire); the warp agrees on the outcome so
-// that no lane leaves a loop that holds warp-synchronous operations.
+// Lane 0 waits; the warp then agrees on the outcome (and is ordered after the
+// wait), so no lane leaves a loop that holds warp-synchronous operations.
 __device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag) {
+                                      volatile int* abort_flag, int lane) {
+  int ok = 0;
+  if (lane == 0) ok = bwait(bar, parity, limit, abort_flag) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// Every lane waits (each acquires the phase, as a reader of TMA-written data
+// must); the warp agrees on the outcome.
+__device__ __forceinline__ bool wwait_all(uint64_t* bar, uint32_t parity, uint32_t limit,
+                                          volatile int* abort_flag) {
   return __all_sync(0xffffffffu, bwait(bar, parity, limit, abort_flag));
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) {
   *abort_flag = 1;
   atomicCAS(err, DEV_OK, DEV_TIMEOUT);
-}
-
-template <typename E>
-__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
-  const E* e = reinterpret_cast<const E*>(&u);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = Elem<E>::to_f(e[i]);
 }
 
 template <typename E>
@@ -134,25 +152,39 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
+// MN-major, 128B-swizzled operand descriptor (A side): leading byte offset =
+// stride between 64-element MN blocks, stride byte offset = stride between
+// 8-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;                                   // 128B swizzle
+  return d;
+}
+
 template <int T, typename E>
 __global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
-tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_w,
-                Params p) {
+tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_in,
+                const __grid_constant__ CUtensorMap map_out, Params p) {
   using C = Cfg<T>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte alignment for the 128B-swizzled tiles
+  // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* raw_buf = smem;
-  uint8_t* a_buf = raw_buf + C::RAW_SLOTS * C::RAW_BYTES;
+  uint8_t* a_buf = smem;
   uint8_t* b_buf = a_buf + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_buf + C::STAGES * C::B_BYTES);
-  uint64_t* raw_full = bars;
-  uint64_t* raw_empty = raw_full + C::RAW_SLOTS;
-  uint64_t* a_full = raw_empty + C::RAW_SLOTS;
+  uint8_t* raw_buf = b_buf + C::STAGES * C::B_BYTES;
+  uint8_t* o_buf = raw_buf + C::STAGES * C::RAW_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_buf + 2 * C::OUT_TILE_BYTES);
+  uint64_t* a_full = bars;
   uint64_t* b_full = a_full + C::STAGES;
   uint64_t* ab_empty = b_full + C::STAGES;
-  uint64_t* acc_full = ab_empty + C::STAGES;
+  uint64_t* raw_full = ab_empty + C::STAGES;
+  uint64_t* raw_empty = raw_full + C::STAGES;
+  uint64_t* acc_full = raw_empty + C::STAGES;
   uint64_t* acc_empty = acc_full + C::NACC;
   uint64_t* drain_bar = acc_empty + C::NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -161,22 +193,29 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t limit = p.wait_limit;
   const int nk = (p.K + C::BK - 1) / C::BK;
+  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int64_t my_tiles = p.n_tiles > blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::RAW_SLOTS; ++i) { mbar_init(&raw_full[i], 1); mbar_init(&raw_empty[i], 4); }
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&a_full[i], 4);
+      mbar_init(&a_full[i], C::TR_WARPS);
       mbar_init(&b_full[i], 1);
       mbar_init(&ab_empty[i], 1);
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], C::TR_WARPS);
     }
-    for (int i = 0; i < C::NACC; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 128); }
+    for (int i = 0; i < C::NACC; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::EPI_WARPS * 32);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&map_in);
     prefetch_tensormap(&map_w);
+    prefetch_tensormap(&map_in);
+    prefetch_tensormap(&map_out);
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -185,57 +224,135 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < C::TR_WARPS) {
+    // ----------------------------------------------------- transform warps
+    // thread: channel c of the stage (16 per stage), 8 consecutive tokens
+    const int c = lane & 15;
+    const int m = warp * 16 + 8 * (lane >> 4);       // first of its 8 tokens in the tile
+    // MN-major placement of the 8 tokens for K row c of a plane
+    const uint32_t a_off = (uint32_t)((m >> 6) * C::A_LBO + (c >> 3) * C::A_SBO + (c & 7) * 128 +
+                                      ((((m & 63) >> 3) ^ (c & 7)) << 4));
+    const uint32_t raw_off = (uint32_t)(m * C::RAW_ROWB + c * T * 2);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int64_t it = 0; it < my_tiles * nk; ++it) {
+      if (!wwait_all(&raw_full[s], ph, limit, abort_flag) ||
+          !wwait(&ab_empty[s], ph ^ 1, limit, abort_flag, lane)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* raw = raw_buf + s * C::RAW_BYTES + raw_off;
+      uint32_t wv[8][C::W];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint8_t* src = raw + j * C::RAW_ROWB;
+        if constexpr (C::W == 4) {
+          const uint4 u = *reinterpret_cast<const uint4*>(src);
+          wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
+        } else if constexpr (C::W == 2) {
+          const uint2 u = *reinterpret_cast<const uint2*>(src);
+          wv[j][0] = u.x; wv[j][1] = u.y;
+        } else if constexpr (T == 2) {
+          wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
+        } else {
+          wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[s]);       // the raw slot may be refilled
+      uint32_t Pw[T][4];
+      if constexpr (T <= 4) {
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+          uint32_t P[T];
+          packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
+#pragma unroll
+          for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
+        }
+      } else {
+        // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+          float Pa[T], Pb[T], va[T], vb[T];
+          const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
+          const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
+#pragma unroll
+          for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
+          G::dft(va, Pa);
+          G::dft(vb, Pb);
+#pragma unroll
+          for (int q = 0; q < T; ++q) {
+            E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
+            Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
+          }
+        }
+      }
+      uint8_t* a_st = a_buf + s * C::A_BYTES + a_off;
+#pragma unroll
+      for (int q = 0; q < T; ++q)
+        *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES) = make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[s]);
+      if (++s == C::STAGES) { s = 0; ph ^= 1; }
+    }
+    if (!ok) raise_abort(abort_flag, p.err);
+  } else if (warp == C::PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int rs = 0, s = 0;
-      uint32_t rph = 0, ph = 0;
-      int64_t n_raw = 0, n_b = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t n_b = 0, n_raw = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-        const int m0 = (int)(tile / p.n_otiles) * C::BM;
-        const int o0 = (int)(tile % p.n_otiles) * C::BO;
+      // L2 prefetch of the raw input tiles PF_STAGES stages ahead of their loads
+      int64_t pf_ti = 0;
+      int pf_kb = 0;
+      auto prefetch_next = [&]() {
+        if (pf_ti >= my_tiles) return;
+        const int tile = (int)(blockIdx.x + pf_ti * gridDim.x);
+        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, (tile / p.n_otiles) * C::BM);
+        if (++pf_kb == nk) { pf_kb = 0; ++pf_ti; }
+      };
+      for (int i = 0; i < C::PF_STAGES; ++i) prefetch_next();
+      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
+        const int tile = (int)(blockIdx.x + ti * gridDim.x);
+        const int m0 = (tile / p.n_otiles) * C::BM;
+        const int o0 = (tile % p.n_otiles) * C::BO;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&raw_empty[rs], rph ^ 1, limit, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&raw_full[rs], C::RAW_BYTES);
-          uint8_t* dst = raw_buf + rs * C::RAW_BYTES;
-          tma_load_2d(dst, &map_in, kb * C::RAW_EL, m0, &raw_full[rs]);
-          tma_load_2d(dst + C::RAW_BOX_BYTES, &map_in, kb * C::RAW_EL + 64, m0, &raw_full[rs]);
+          prefetch_next();
+          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
+          tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
           ++n_raw;
-          if (++rs == C::RAW_SLOTS) { rs = 0; rph ^= 1; }
-
           if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&b_full[s], C::B_BYTES);
           uint8_t* bdst = b_buf + s * C::B_BYTES;
 #pragma unroll
           for (int q = 0; q < C::Q; ++q)
-#pragma unroll
-            for (int a = 0; a < C::KATOMS; ++a)
-              tma_load_3d(bdst + q * C::B_PLANE_BYTES + a * (C::BO * 128), &map_w,
-                          kb * C::BK + a * 64, o0, q, &b_full[s]);
+            tma_load_3d(bdst + q * C::B_PLANE_BYTES, &map_w, kb * C::BK, o0, q, &b_full[s]);
           ++n_b;
           if (++s == C::STAGES) { s = 0; ph ^= 1; }
         }
       }
       if (!ok) raise_abort(abort_flag, p.err);
-      {
-        // drain: every issued TMA copy must land before the CTA exits (a
-        // no-op on the normal path, where the consumers already waited)
-        for (int i = 0; i < C::RAW_SLOTS; ++i)
-          if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::RAW_SLOTS) & 1), kDefaultWaitLimit);
-        for (int i = 0; i < C::STAGES; ++i)
-          if (n_b > i) mbar_wait(&b_full[i], (uint32_t)(((n_b - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
+      // every issued TMA copy must land before the CTA exits (a no-op on the
+      // normal path, where the MMA thread already waited for them)
+      for (int i = 0; i < C::STAGES; ++i) {
+        if (n_b > i) mbar_wait(&b_full[i], (uint32_t)(((n_b - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
+        if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == C::MMA_WARP) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       int s = 0, ab = 0;
       uint32_t ph = 0, aph = 0;
       bool ok = true;
-      const uint32_t id_real = idesc_f16(p.ab_fmt, C::BO);
-      const uint32_t id_cplx = idesc_f16(p.ab_fmt, 2 * C::BO);
-      for (int64_t tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+      // A is MN-major (bit 15), B K-major
+      const uint32_t id_real = idesc_f16(p.ab_fmt, C::BO) | (1u << 15);
+      const uint32_t id_cplx = idesc_f16(p.ab_fmt, 2 * C::BO) | (1u << 15);
+      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         if (!bwait(&acc_empty[ab], aph ^ 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
@@ -247,28 +364,25 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           tc_fence_after();
           const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
           const uint32_t b_st = smem_u32(b_buf + s * C::B_BYTES);
-#pragma unroll
-          for (int ks = 0; ks < C::KSTEPS; ++ks) {
-            const int atom = (ks * 32) / C::ROWB;
-            const uint32_t koff = (ks * 32) % C::ROWB;
-            const uint32_t a_k = a_st + atom * (C::BM * 128) + koff;
-            const uint32_t b_k = b_st + atom * (C::BO * 128) + koff;
-            const uint32_t first = (kb > 0 || ks > 0) ? 1u : 0u;
+          {
+            const uint32_t a_k = a_st;
+            const uint32_t b_k = b_st;
+            const uint32_t first = kb > 0 ? 1u : 0u;
 #pragma unroll
             for (int f = 0; f < G::nreal; ++f)
-              mma_f16_ss(acc + f * C::BO, smem_desc(a_k + f * C::A_PLANE_BYTES, C::ROWB),
-                         smem_desc(b_k + f * C::B_PLANE_BYTES, C::ROWB), id_real, first);
+              mma_f16_ss(acc + f * C::BO, smem_desc_mn(a_k + f * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
+                         smem_desc(b_k + f * C::B_PLANE_BYTES, C::B_ROWB), id_real, first);
 #pragma unroll
             for (int k = 1; k <= G::ncomplex; ++k) {
               const int pr = G::nreal + 2 * (k - 1);
               const int q = G::nreal + 3 * (k - 1);
               const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO;
               // [Re Y | Im Y] += Re X [Re W ; Im W]
-              mma_f16_ss(col, smem_desc(a_k + pr * C::A_PLANE_BYTES, C::ROWB),
-                         smem_desc(b_k + (q + 1) * C::B_PLANE_BYTES, C::ROWB), id_cplx, first);
+              mma_f16_ss(col, smem_desc_mn(a_k + pr * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
+                         smem_desc(b_k + (q + 1) * C::B_PLANE_BYTES, C::B_ROWB), id_cplx, first);
               // [Re Y | Im Y] += Im X [-Im W ; Re W]
-              mma_f16_ss(col, smem_desc(a_k + (pr + 1) * C::A_PLANE_BYTES, C::ROWB),
-                         smem_desc(b_k + q * C::B_PLANE_BYTES, C::ROWB), id_cplx, 1u);
+              mma_f16_ss(col, smem_desc_mn(a_k + (pr + 1) * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
+                         smem_desc(b_k + q * C::B_PLANE_BYTES, C::B_ROWB), id_cplx, 1u);
             }
           }
           mma_commit(&ab_empty[s]);
@@ -282,123 +396,90 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       mma_commit(drain_bar);              // arrives once every issued MMA has completed
       mbar_wait(drain_bar, 0, kDefaultWaitLimit);
     }
-  } else if (warp < 6) {
-    // ----------------------------------------------------- transform warps
-    const int r = (warp - 2) * 32 + lane;            // token row within the tile
-    int rs = 0, s = 0;
-    uint32_t rph = 0, ph = 0;
-    bool ok = true;
-    const int swz = (r >> C::SW_SHIFT) & C::SW_MASK;
-    for (int64_t tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < nk; ++kb) {
-        if (!wwait(&raw_full[rs], rph, limit, abort_flag) || !wwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* rrow = raw_buf + rs * C::RAW_BYTES + r * 128;
-        uint8_t* a_st = a_buf + s * C::A_BYTES;
-        // 8 channels (one 16-byte operand chunk per plane) at a time
-#pragma unroll
-        for (int g = 0; g < C::BK / 8; ++g) {
-          float v[8 * T];
-#pragma unroll
-          for (int cch = 0; cch < T; ++cch) {
-            const int chunk = g * T + cch;           // 16-byte chunk of the 256-byte raw row
-            const int box = chunk >> 3, j = chunk & 7;
-            const uint4 u = *reinterpret_cast<const uint4*>(rrow + box * C::RAW_BOX_BYTES + ((j ^ (r & 7)) << 4));
-            unpack8<E>(u, v + 8 * cch);
-          }
-          float P[T][8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float Pc[T];
-            G::dft(v + c * T, Pc);
-#pragma unroll
-            for (int q = 0; q < T; ++q) P[q][c] = Pc[q];
-          }
-          const int atom = (g * 16) / C::ROWB;
-          const int j = g % (C::ROWB / 16);
-#pragma unroll
-          for (int q = 0; q < T; ++q) {
-            uint8_t* dst = a_st + q * C::A_PLANE_BYTES + atom * (C::BM * 128) + r * C::ROWB +
-                           ((j ^ swz) << 4);
-            *reinterpret_cast<uint4*>(dst) = pack8<E>(P[q]);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&raw_empty[rs]);
-          mbar_arrive(&a_full[s]);
-        }
-        if (++rs == C::RAW_SLOTS) { rs = 0; rph ^= 1; }
-        if (++s == C::STAGES) { s = 0; ph ^= 1; }
-      }
-    }
-    if (!ok) raise_abort(abort_flag, p.err);
   } else {
     // ------------------------------------------------------ epilogue warps
+    // Two halves of four warps (one per TMEM lane quarter); half h takes the
+    // store chunks h, h+2, ...  Each chunk is 64 output elements of all 128
+    // rows: TMEM -> registers -> inverse DFT + bias -> 128B-swizzled staging
+    // tile -> one TMA store.
+    const int e = warp - C::EPI0;
+    const int half = e >> 2;
     const int quarter = warp & 3;                    // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const bool issuer = (e & 3) == 0 && lane == 0;
+    uint8_t* stage_tile = o_buf + half * C::OUT_TILE_BYTES;
+    uint8_t* my_row = stage_tile + r * 128;
     int ab = 0;
     uint32_t aph = 0;
     bool ok = true;
-    E* out = reinterpret_cast<E*>(p.out);
-    for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
-      if (!wwait(&acc_full[ab], aph, limit, abort_flag)) { ok = false; break; }
+    for (int64_t ti = 0; ti < my_tiles; ++ti) {
+      const int tile = (int)(blockIdx.x + ti * gridDim.x);
+      // the four warps of a half share named barriers, so they decide together
+      const bool got = named_bar_and(1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane));
+      if (!got) { ok = false; break; }
       tc_fence_after();
-      const int64_t row = (tile / p.n_otiles) * C::BM + r;
-      const int o0 = (int)(tile % p.n_otiles) * C::BO;
+      const int m0 = (tile / p.n_otiles) * C::BM;
+      const int o0 = (tile % p.n_otiles) * C::BO;
       const uint32_t acc = tmem_base + lane_addr + ab * C::ACC_COLS;
 #pragma unroll 1
-      for (int oc = 0; oc < C::BO; oc += 8) {
-        uint32_t rg[T][8];
+      for (int ci = half; ci < C::NCHUNK; ci += 2) {
+        // the previous TMA store from this staging tile must have read it
+        if (issuer) bulk_wait_read<0>();
+        named_bar_sync(1 + half, 128);
 #pragma unroll
-        for (int f = 0; f < G::nreal; ++f) tmem_ld_32x32b_x8(acc + f * C::BO + oc, rg[f]);
+        for (int sub = 0; sub < C::CH / 8; ++sub) {
+          const int oc = ci * C::CH + sub * 8;       // channel offset within the tile
+          uint32_t rg[T][8];
 #pragma unroll
-        for (int k = 1; k <= G::ncomplex; ++k) {
-          const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO + oc;
-          tmem_ld_32x32b_x8(col, rg[G::nreal + 2 * (k - 1)]);
-          tmem_ld_32x32b_x8(col + C::BO, rg[G::nreal + 2 * (k - 1) + 1]);
+          for (int f = 0; f < G::nreal; ++f) tmem_ld_32x32b_x8(acc + f * C::BO + oc, rg[f]);
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO + oc;
+            tmem_ld_32x32b_x8(col, rg[G::nreal + 2 * (k - 1)]);
+            tmem_ld_32x32b_x8(col + C::BO, rg[G::nreal + 2 * (k - 1) + 1]);
+          }
+          tmem_wait_ld();
+          if (ci + 2 >= C::NCHUNK && sub == C::CH / 8 - 1) {
+            // last TMEM read of this tile by this thread: release the accumulator
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);
+          }
+          const int o = o0 + oc;
+          // 8 channels x T outputs = T 16-byte chunks of this row's 128 bytes;
+          // chunk v holds the outputs of channels v*8/T .. (v+1)*8/T - 1
+#pragma unroll
+          for (int v = 0; v < T; ++v) {
+            float vals[8];
+#pragma unroll
+            for (int cc = 0; cc < 8 / T; ++cc) {
+              const int c = v * (8 / T) + cc;
+              const float bo = (p.bias && o + c < p.O) ? __ldg(p.bias + o + c) : 0.f;
+              float Pc[T];
+#pragma unroll
+              for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][c]);
+              G::idft_scaled(Pc, bo, vals + cc * T);
+            }
+            const int j = sub * T + v;
+            *reinterpret_cast<uint4*>(my_row + ((j ^ (r & 7)) << 4)) = pack8<E>(vals);
+          }
         }
-        tmem_wait_ld();
-        const int o = o0 + oc;
-        if (row < p.N && o < p.O) {
-          float vals[8 * T];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float Pc[T], yc[T];
-#pragma unroll
-            for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][c]);
-            G::idft(Pc, yc);
-            const float bo = (p.bias && o + c < p.O) ? __ldg(p.bias + o + c) : 0.f;
-#pragma unroll
-            for (int s_ = 0; s_ < T; ++s_) vals[c * T + s_] = yc[s_] + bo;
-          }
-          E* dst = out + row * (int64_t)p.O * T + (int64_t)o * T;
-          if (o + 8 <= p.O) {
-#pragma unroll
-            for (int v = 0; v < T; ++v)
-              reinterpret_cast<uint4*>(dst)[v] = pack8<E>(vals + 8 * v);
-          } else {
-            const int nvalid = (p.O - o) * T;
-#pragma unroll
-            for (int i = 0; i < 8 * T; ++i)
-              if (i < nvalid) dst[i] = Elem<E>::from_f(vals[i]);
-          }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + half, 128);
+        if (issuer) {
+          tma_store_2d(&map_out, stage_tile, (o0 + ci * C::CH) * T, m0);
+          bulk_commit();
         }
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[ab]);
       if (++ab == C::NACC) { ab = 0; aph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
+    if (issuer) bulk_wait<0>();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
@@ -417,11 +498,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-static CUtensorMapSwizzle swz_enum(int row_bytes) {
-  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-       : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-}
-
 template <int T, typename E>
 static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, int64_t N,
                             cudaStream_t st) {
@@ -432,25 +508,37 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   const int O = (int)(backward ? h.Cp : h.Dp);
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap map_in, map_w;
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)K * T, (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)K * T * 2};
-    cuuint32_t box[2] = {64, C::BM};
-    cuuint32_t es[2] = {1, 1};
-    if (enc(&map_in, dt, 2, const_cast<void*>(in), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
+  CUtensorMap map_w;
   {
     cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)O, (cuuint64_t)C::Q};
     cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)K * O * 2};
-    cuuint32_t box[3] = {(cuuint32_t)(C::ROWB / 2), (cuuint32_t)C::BO, 1};
+    cuuint32_t box[3] = {(cuuint32_t)C::BK, (cuuint32_t)C::BO, 1};
     cuuint32_t es[3] = {1, 1, 1};
     void* wptr = backward ? h.wt_bwd : h.wt_fwd;
     if (enc(&map_w, dt, 3, wptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swz_enum(C::ROWB), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  CUtensorMap map_in;      // raw input tiles: 16 channels x T elements x 128 tokens
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K * T, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)K * T * 2};
+    cuuint32_t box[2] = {(cuuint32_t)(C::BK * T), (cuuint32_t)C::BM};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&map_in, dt, 2, const_cast<void*>(in), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  CUtensorMap map_out;     // TMA stores of the output tile, 64 elements x 128 rows, 128B swizzle
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)O * T, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)O * T * 2};
+    cuuint32_t box[2] = {(cuuint32_t)C::OUT_EL, (cuuint32_t)C::BM};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&map_out, dt, 2, out, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
@@ -460,8 +548,8 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.O = O;
   p.n_otiles = (O + C::BO - 1) / C::BO;
   p.n_tiles = ((N + C::BM - 1) / C::BM) * p.n_otiles;
+  p.in = in;
   p.bias = backward ? nullptr : h.bias;
-  p.out = out;
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
@@ -475,7 +563,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_w, p);
+  tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_w, map_in, map_out, p);
   count_launches(1);
   return cudaGetLastError();
 }

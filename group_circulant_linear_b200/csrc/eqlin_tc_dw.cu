@@ -15,18 +15,24 @@
 // contiguous chunk of tokens.  Roles:
 //   warps 0-3  (one thread per d)  load gy[n, d*T .. d*T+T) straight from
 //              global memory -- a warp reads 256 contiguous bytes per token --,
-//              take the DFT in FP32, keep sum_n G_0 for db, round once to the
-//              operand type and write the K-major (token-contiguous) planes;
+//              one stage ahead of use (double-buffered in registers), take the
+//              DFT on packed pairs of tokens (T <= 4; FP32 with one rounding
+//              for T = 8), keep sum_n G_0 in FP32 for db and write the K-major
+//              (token-contiguous) operand planes;
 //              after the main loop they read the accumulators out of TMEM
 //   warps 4-7  (one thread per c)  the same for x, writing the B planes
 //              (real frequencies, then Im X, Re X, -Im X per complex one)
-//   warp 8     allocates TMEM; one thread issues the MMAs
+//   warp 8     allocates TMEM; one thread issues the MMAs and, several
+//              stages ahead, L2 prefetches (TMA) of the gy and x rows
 // The per-chunk partial planes go to the handle's workspace; a second kernel
 // sums the chunks in a fixed order and applies the inverse DFT
 // (deterministic, no atomics).  All waits are bounded as in eqlin_tc.cu.
+#include <cudaTypedefs.h>
+
 #include <type_traits>
 
 #include "eqlin_internal.cuh"
+#include "eqlin_packed.cuh"
 #include "eqlin_ptx.cuh"
 
 namespace eqlin {
@@ -53,6 +59,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NBAR * 8 + 16 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
   static constexpr int THREADS = 288;
+  static constexpr int PF_STAGES = 8;                     // L2 prefetch distance (stages)
 };
 
 struct Params {
@@ -133,7 +140,8 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
 
 template <int T, typename E>
 __global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
-tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, Params p) {
+tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_constant__ CUtensorMap map_x,
+             const __grid_constant__ CUtensorMap map_gy, Params p) {
   using C = Cfg<T>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
@@ -185,61 +193,145 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, Params p) {
     const bool valid = active && ch < nch;
     const E* src = (is_a ? gy : x) + (int64_t)(valid ? ch : 0) * T;
     const int64_t pitch = (int64_t)nch * T;
+    constexpr int W = packed::Words<T>::n;                // 32-bit words per token and channel
+    constexpr int TOK = C::BKN;
     float dbacc = 0.f;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int st = 0; st < nst; ++st) {
-      if (!wwait(&op_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+
+    // Raw words of one stage: one vector load per token, issued ahead of use.
+    auto load_stage = [&](uint32_t (&buf)[TOK][W], int st) {
+      const int64_t n_st = nbeg + (int64_t)st * TOK;
+#pragma unroll
+      for (int j = 0; j < TOK; ++j) {
+        const int64_t n = n_st + j;
+        if (valid && st < nst && n < nend) {
+          packed::load_words<T>(src + n * pitch, buf[j]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < W; ++w) buf[j][w] = 0u;
+        }
+      }
+    };
+
+    // Write the plane words of one group of 8 tokens (g) into the stage slot.
+    auto store_group = [&](uint32_t (&Pw)[T][4], int g, uint8_t* a_st, uint8_t* b_st) {
+      const uint32_t off = kmajor_off(r, g);
+      if (is_a) {
+#pragma unroll
+        for (int q = 0; q < T; ++q)
+          *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
+              make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+      } else {
+#pragma unroll
+        for (int f = 0; f < G::nreal; ++f)
+          *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
+              make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
+#pragma unroll
+        for (int k = 1; k <= G::ncomplex; ++k) {
+          const int pr = G::nreal + 2 * (k - 1);
+          const int q = G::nreal + 3 * (k - 1);
+          const uint32_t* re = Pw[pr];
+          const uint32_t* im = Pw[pr + 1];
+          *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(im[0], im[1], im[2], im[3]);
+          *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(re[0], re[1], re[2], re[3]);
+          *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
+              make_uint4(packed::neg2(im[0]), packed::neg2(im[1]), packed::neg2(im[2]), packed::neg2(im[3]));
+        }
+      }
+    };
+
+    // One stage: wait for the slot, transform the buffered tokens, publish.
+    auto run_stage = [&](const uint32_t (&buf)[TOK][W]) -> bool {
+      if (!wwait(&op_empty[s], ph ^ 1, limit, abort_flag)) return false;
       if (active) {
         uint8_t* a_st = a_buf + s * C::A_BYTES;
         uint8_t* b_st = b_buf + s * C::B_BYTES;
-        const int64_t n_st = nbeg + (int64_t)st * C::BKN;
 #pragma unroll
-        for (int g = 0; g < C::BKN / 8; ++g) {
-          float P[T][8];
+        for (int g = 0; g < TOK / 8; ++g) {
+          uint32_t Pw[T][4];
+          if constexpr (T <= 4) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int64_t n = n_st + g * 8 + j;
-            float v[T], Pj[T];
-            if (valid && n < nend) {
-              load_group<T, E>(src + n * pitch, v);
-            } else {
+            for (int pr = 0; pr < 4; ++pr) {
+              uint32_t P[T];
+              packed::dft_pair<T, E>(buf[g * 8 + 2 * pr], buf[g * 8 + 2 * pr + 1], P);
 #pragma unroll
-              for (int t = 0; t < T; ++t) v[t] = 0.f;
-            }
-            G::dft(v, Pj);
-#pragma unroll
-            for (int q = 0; q < T; ++q) P[q][j] = Pj[q];
-            dbacc += Pj[0];
-          }
-          const uint32_t off = kmajor_off(r, g);
-          if (is_a) {
-#pragma unroll
-            for (int q = 0; q < T; ++q)
-              *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) = pack8<E>(P[q]);
-          } else {
-#pragma unroll
-            for (int f = 0; f < G::nreal; ++f)
-              *reinterpret_cast<uint4*>(b_st + f * b_plane + off) = pack8<E>(P[f]);
-#pragma unroll
-            for (int k = 1; k <= G::ncomplex; ++k) {
-              const int pr = G::nreal + 2 * (k - 1);
-              const int q = G::nreal + 3 * (k - 1);
-              float ni[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) ni[j] = -P[pr + 1][j];
-              *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = pack8<E>(P[pr + 1]);
-              *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = pack8<E>(P[pr]);
-              *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) = pack8<E>(ni);
+              for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
+              if (is_a) {
+                const float2 f = packed::Pair<E>::to_f2(P[0]);
+                dbacc += f.x + f.y;
+              }
             }
           }
+          store_group(Pw, g, a_st, b_st);
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&op_full[s]);
       if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      return true;
+    };
+
+    if constexpr (T <= 4) {
+      // double-buffered: the next stage's loads are in flight while this one is transformed
+      uint32_t bufA[TOK][W], bufB[TOK][W];
+      load_stage(bufA, 0);
+      for (int st = 0; st < nst; st += 2) {
+        load_stage(bufB, st + 1);
+        if (!run_stage(bufA)) { ok = false; break; }
+        if (st + 1 >= nst) break;
+        load_stage(bufA, st + 2);
+        if (!run_stage(bufB)) { ok = false; break; }
+      }
+    } else {
+      // T = 8: FP32 butterflies with the sqrt(2)/2 twiddles; loads per group of 8 tokens
+      for (int st = 0; st < nst; ++st) {
+        if (!wwait(&op_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+        if (active) {
+          uint8_t* a_st = a_buf + s * C::A_BYTES;
+          uint8_t* b_st = b_buf + s * C::B_BYTES;
+          const int64_t n_st = nbeg + (int64_t)st * TOK;
+#pragma unroll 1
+          for (int g = 0; g < TOK / 8; ++g) {
+            uint32_t raw[8][W];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int64_t n = n_st + g * 8 + j;
+              if (valid && n < nend) {
+                packed::load_words<T>(src + n * pitch, raw[j]);
+              } else {
+#pragma unroll
+                for (int w = 0; w < W; ++w) raw[j][w] = 0u;
+              }
+            }
+            float Pf[T][8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const E* e = reinterpret_cast<const E*>(raw[j]);
+              float v[T], Pj[T];
+#pragma unroll
+              for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(e[t]);
+              G::dft(v, Pj);
+#pragma unroll
+              for (int q = 0; q < T; ++q) Pf[q][j] = Pj[q];
+              dbacc += Pj[0];
+            }
+            uint32_t Pw[T][4];
+#pragma unroll
+            for (int q = 0; q < T; ++q) {
+              const uint4 u = pack8<E>(Pf[q]);
+              Pw[q][0] = u.x; Pw[q][1] = u.y; Pw[q][2] = u.z; Pw[q][3] = u.w;
+            }
+            store_group(Pw, g, a_st, b_st);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&op_full[s]);
+        if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      }
     }
     if (!ok) raise_abort(abort_flag, p.err);
 
@@ -295,7 +387,16 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, Params p) {
     bool ok = true;
     const uint32_t id_real = idesc_f16(p.ab_fmt, (uint32_t)BC);
     const uint32_t id_cplx = idesc_f16(p.ab_fmt, (uint32_t)(2 * BC));
+    // L2 prefetch of the gy and x rows of stage `ps` (this CTA's d and c range)
+    auto prefetch = [&](int ps) {
+      if (ps >= nst) return;
+      const int n = (int)(nbeg + (int64_t)ps * C::BKN);
+      for (int xb = 0; xb < C::BM * T; xb += 256) tma_prefetch_2d(&map_gy, d0 * T + xb, n);
+      for (int xb = 0; xb < BC * T; xb += 256) tma_prefetch_2d(&map_x, c0 * T + xb, n);
+    };
+    for (int i = 0; i < C::PF_STAGES; ++i) prefetch(i);
     for (int st = 0; st < nst; ++st) {
+      prefetch(st + C::PF_STAGES);
       if (!bwait(&op_full[s], ph, limit, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
@@ -387,6 +488,32 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
+  // tensor maps used only for L2 prefetches of the token chunks
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return cudaErrorNotSupported;
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap map_x, map_gy;
+  const void* srcs[2] = {x, gy};
+  const int64_t widths[2] = {h.Cp * T, h.Dp * T};
+  CUtensorMap* maps[2] = {&map_x, &map_gy};
+  for (int i = 0; i < 2; ++i) {
+    cuuint64_t dims[2] = {(cuuint64_t)widths[i], (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)widths[i] * 2};
+    cuuint32_t box[2] = {(cuuint32_t)(widths[i] < 256 ? widths[i] : 256), (cuuint32_t)C::BKN};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(maps[i], dt, 2, const_cast<void*>(srcs[i]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(tc_dw_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -395,7 +522,7 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
     attr_set = true;
   }
   const unsigned grid = (unsigned)(pl.n_dt * pl.n_ct * pl.splits);
-  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>((const E*)x, (const E*)gy, p);
+  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>((const E*)x, (const E*)gy, map_x, map_gy, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);
