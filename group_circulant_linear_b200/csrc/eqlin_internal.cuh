@@ -169,10 +169,11 @@ cudaError_t launch_simt_apply(const Handle& h, bool backward, const void* in, vo
 cudaError_t launch_simt_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
                            int64_t N, cudaStream_t st);
 size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp);
-// Sum per-split partial Fourier planes [splits][T][Dp][Cp] (+ db partials
-// [splits][Dp]) in split order and apply the inverse DFT -> dW [Dp][Cp][T].
+// Sum per-split partial Fourier planes ([splits][T][Dp][Cp], or
+// [splits][T][Cp][Dp] when cd_layout) and db partials [splits][Dp] in split
+// order and apply the inverse DFT -> dW [Dp][Cp][T].
 cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
-                             float* dW, float* db, cudaStream_t st);
+                             float* dW, float* db, bool cd_layout, cudaStream_t st);
 
 // tcgen05 path (f16/bf16).  Returns cudaErrorNotSupported when the shape is
 // outside what the kernel handles, so the caller can fall back to SIMT.

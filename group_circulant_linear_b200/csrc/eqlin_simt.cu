@@ -375,10 +375,12 @@ simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restr
 }
 
 // Sum the splits in index order, then inverse DFT along the frequency planes.
+// Partials are [splits][T][Dp][Cp] (cd_layout false) or [splits][T][Cp][Dp]
+// (cd_layout true); threads walk the partials' contiguous index.
 template <int T>
 __global__ void dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart,
                                  float* __restrict__ dW, float* __restrict__ db, int splits,
-                                 int Cp, int Dp) {
+                                 int Cp, int Dp, bool cd_layout) {
   using G = Group<T>;
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t plane = (int64_t)Cp * Dp;
@@ -391,9 +393,11 @@ __global__ void dw_reduce_kernel(const float* __restrict__ part, const float* __
       P[p] = s;
     }
     G::idft(P, v);
-    // idx = d*Cp + c, and dW is [Dp][Cp][T]
+    const int64_t d = cd_layout ? idx % Dp : idx / Cp;
+    const int64_t c = cd_layout ? idx / Dp : idx % Cp;
+    // dW is [Dp][Cp][T]
 #pragma unroll
-    for (int t = 0; t < T; ++t) dW[idx * T + t] = v[t];
+    for (int t = 0; t < T; ++t) dW[(d * Cp + c) * T + t] = v[t];
   }
   if (db && idx < Dp) {
     float s = 0.f;
@@ -419,27 +423,27 @@ static cudaError_t simt_dw_t(const Handle& h, const void* x, const void* gy, flo
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);
-  return launch_dw_reduce(h, splits, part, dbpart, dW, db, st);
+  return launch_dw_reduce(h, splits, part, dbpart, dW, db, /*cd_layout=*/false, st);
 }
 
 template <int T>
 static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
-                               float* dW, float* db, cudaStream_t st) {
+                               float* dW, float* db, bool cd_layout, cudaStream_t st) {
   const int64_t plane = h.Cp * h.Dp;
   const int64_t work = plane > h.Dp ? plane : h.Dp;
   dw_reduce_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(part, dbpart, dW, db, splits,
-                                                                      (int)h.Cp, (int)h.Dp);
+                                                                      (int)h.Cp, (int)h.Dp, cd_layout);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
-                             float* dW, float* db, cudaStream_t st) {
+                             float* dW, float* db, bool cd_layout, cudaStream_t st) {
   switch (h.T) {
-    case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, st);
-    case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, st);
-    case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, st);
-    case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, st);
+    case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, cd_layout, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -12,21 +12,22 @@
 // so p4 again needs six real GEMMs.
 //
 // Work unit of one CTA: 128 output channels d x BC input channels c x one
-// contiguous chunk of tokens.  Roles:
-//   warps 0-3  (one thread per d)  load gy[n, d*T .. d*T+T) straight from
-//              global memory -- a warp reads 256 contiguous bytes per token --,
-//              one stage ahead of use (double-buffered in registers), take the
-//              DFT on packed pairs of tokens (T <= 4; FP32 with one rounding
+// contiguous chunk of tokens, in stages of 16 tokens.  Roles:
+//   warp 8     (producer)  TMA: the stage's gy rows of the 128 d channels and
+//              x rows of the BC c channels into shared memory, and L2
+//              prefetches of later stages
+//   warps 0-3  (one thread per d)  read the channel's T group values of the 16
+//              tokens, take the group DFT (packed token pairs for T <= 4, FP32
 //              for T = 8), keep sum_n G_0 in FP32 for db and write the K-major
-//              (token-contiguous) operand planes;
-//              after the main loop they read the accumulators out of TMEM
+//              (token-contiguous) A planes; after the main loop they read the
+//              accumulators out of TMEM
 //   warps 4-7  (one thread per c)  the same for x, writing the B planes
 //              (real frequencies, then Im X, Re X, -Im X per complex one)
-//   warp 8     allocates TMEM; one thread issues the MMAs and, several
-//              stages ahead, L2 prefetches (TMA) of the gy and x rows
-// The per-chunk partial planes go to the handle's workspace; a second kernel
-// sums the chunks in a fixed order and applies the inverse DFT
-// (deterministic, no atomics).  All waits are bounded as in eqlin_tc.cu.
+//   warp 9     allocates TMEM; one thread issues the MMAs
+// The per-chunk partial planes go to the handle's workspace as
+// [chunk][plane][c][d]; a second kernel sums the chunks in a fixed order and
+// applies the inverse DFT (deterministic, no atomics).  All waits are bounded
+// as in eqlin_tc.cu.
 #include <cudaTypedefs.h>
 
 #include <type_traits>
@@ -44,22 +45,29 @@ template <int T>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                          // output channels d per tile (MMA M)
-  static constexpr int BKN = 32;                          // tokens per stage (MMA K = 2 x 16)
-  static constexpr int ROWB = BKN * 2;                    // 64-byte K-major rows, 64B swizzle
+  static constexpr int BKN = 16;                          // tokens per stage (one MMA K step)
+  static constexpr int ROWB = BKN * 2;                    // 32-byte K-major rows, 32B swizzle
   static constexpr int BC_MAX = (512 / T) < 128 ? (512 / T) : 128;
   static constexpr int Q = G::nreal + 3 * G::ncomplex;    // B planes
   static constexpr int A_PLANE_BYTES = BM * ROWB;
   static constexpr int A_BYTES = T * A_PLANE_BYTES;
   static constexpr int B_BYTES = Q * BC_MAX * ROWB;       // plane stride is BC * ROWB at run time
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  // raw tiles of a stage (TMA, row-major): gy [16 tokens][128 d x T], x [16 tokens][BC x T]
+  static constexpr int GY_ROWB = BM * T * 2;
+  static constexpr int X_ROWB_MAX = BC_MAX * T * 2;
+  static constexpr int RAW_BYTES = BKN * (GY_ROWB + X_ROWB_MAX);
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
   static constexpr int STAGES_FIT = (220 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(STAGES >= 2, "two stages must fit");
-  static constexpr int NBAR = 2 * STAGES + 2;
+  static constexpr int NBAR = 4 * STAGES + 2;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NBAR * 8 + 16 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
-  static constexpr int THREADS = 288;
-  static constexpr int PF_STAGES = 8;                     // L2 prefetch distance (stages)
+  static constexpr int PRODUCER = 8, MMA_WARP = 9;
+  static constexpr int THREADS = 320;
+  static constexpr int PF_STAGES = 12;                    // L2 prefetch distance (stages)
+  static constexpr int GY_BOX = BM * T <= 256 ? BM * T : 256;   // gy TMA box width (elements)
+  static constexpr int W = packed::Words<T>::n;
 };
 
 struct Params {
@@ -68,7 +76,8 @@ struct Params {
   int BC;                 // input channels per tile (multiple of 16)
   int n_dt, n_ct;         // d tiles, c tiles
   int64_t chunk;          // tokens per split (multiple of BKN)
-  float* part;            // [splits][T][Dp][Cp]
+  int x_box;              // x TMA box width (elements), divides BC * T
+  float* part;            // [splits][T][Cp][Dp]
   float* dbpart;          // [splits][Dp]
   int* err;
   uint32_t wait_limit;
@@ -90,38 +99,25 @@ __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t l
   return false;
 }
 
-__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag) {
+// every lane waits (readers of TMA-written data); the warp agrees on the outcome
+__device__ __forceinline__ bool wwait_all(uint64_t* bar, uint32_t parity, uint32_t limit,
+                                          volatile int* abort_flag) {
   return __all_sync(0xffffffffu, bwait(bar, parity, limit, abort_flag));
+}
+
+// lane 0 waits, the warp follows (slot reuse)
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit,
+                                      volatile int* abort_flag, int lane) {
+  int ok = 0;
+  if (lane == 0) ok = bwait(bar, parity, limit, abort_flag) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) {
   *abort_flag = 1;
   atomicCAS(err, DEV_OK, DEV_TIMEOUT);
-}
-
-// Load the T group values of one channel of one token (T*2 bytes, one vector load).
-template <int T, typename E>
-__device__ __forceinline__ void load_group(const E* p, float* v) {
-  if constexpr (T == 8) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const E* e = reinterpret_cast<const E*>(&u);
-#pragma unroll
-    for (int t = 0; t < 8; ++t) v[t] = Elem<E>::to_f(e[t]);
-  } else if constexpr (T == 4) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const E* e = reinterpret_cast<const E*>(&u);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) v[t] = Elem<E>::to_f(e[t]);
-  } else if constexpr (T == 2) {
-    const unsigned u = __ldg(reinterpret_cast<const unsigned*>(p));
-    const E* e = reinterpret_cast<const E*>(&u);
-    v[0] = Elem<E>::to_f(e[0]);
-    v[1] = Elem<E>::to_f(e[1]);
-  } else {
-    const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
-    v[0] = Elem<E>::to_f(*reinterpret_cast<const E*>(&u));
-  }
 }
 
 template <typename E>
@@ -133,23 +129,25 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
-// Byte offset of the 16-byte chunk j (8 tokens) of row r in a 64B-swizzled K-major plane.
+// Byte offset of the 16-byte chunk j (8 tokens) of row r in a 32B-swizzled K-major plane.
 __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
-  return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+  return (uint32_t)(r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
 }
 
 template <int T, typename E>
 __global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
-tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_constant__ CUtensorMap map_x,
-             const __grid_constant__ CUtensorMap map_gy, Params p) {
+tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy, Params p) {
   using C = Cfg<T>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* a_buf = smem;
   uint8_t* b_buf = a_buf + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_buf + C::STAGES * C::B_BYTES);
-  uint64_t* op_full = bars;                       // 8 transform warps arrive
+  uint8_t* raw_buf = b_buf + C::STAGES * C::B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw_buf + C::STAGES * C::RAW_BYTES);
+  uint64_t* raw_full = bars;                      // TMA
+  uint64_t* raw_empty = raw_full + C::STAGES;     // 8 transform warps
+  uint64_t* op_full = raw_empty + C::STAGES;      // 8 transform warps
   uint64_t* op_empty = op_full + C::STAGES;       // MMA commit
   uint64_t* acc_full = op_empty + C::STAGES;
   uint64_t* drain_bar = acc_full + 1;
@@ -166,15 +164,23 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
   const uint32_t limit = p.wait_limit;
   const int BC = p.BC;
   const uint32_t b_plane = (uint32_t)BC * C::ROWB;
+  const int x_rowb = BC * T * 2;                  // raw x row bytes of this tile
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&op_full[i], 8); mbar_init(&op_empty[i], 1); }
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 8);
+      mbar_init(&op_full[i], 8);
+      mbar_init(&op_empty[i], 1);
+    }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_gy);
   }
-  if (warp == 8) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -187,75 +193,52 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
     // --------------------------------------------------- transform warps
     const bool is_a = warp < 4;
     const int r = (warp & 3) * 32 + lane;                 // operand row: d (A) or c (B)
-    const int ch = is_a ? d0 + r : c0 + r;                // channel index in the tensor
-    const int nch = is_a ? p.Dp : p.Cp;
     const bool active = is_a || r < BC;
-    const bool valid = active && ch < nch;
-    const E* src = (is_a ? gy : x) + (int64_t)(valid ? ch : 0) * T;
-    const int64_t pitch = (int64_t)nch * T;
-    constexpr int W = packed::Words<T>::n;                // 32-bit words per token and channel
-    constexpr int TOK = C::BKN;
+    // this thread's channel in the raw tile rows
+    const uint32_t raw_col = is_a ? (uint32_t)((r / (C::GY_BOX / T)) * C::BKN * C::GY_BOX * 2 +
+                                               (r % (C::GY_BOX / T)) * T * 2)
+                                  : (uint32_t)((r * T / p.x_box) * C::BKN * p.x_box * 2 +
+                                               ((r * T) % p.x_box) * 2);
+    const uint32_t raw_rowb = is_a ? (uint32_t)(C::GY_BOX * 2) : (uint32_t)(p.x_box * 2);
+    const uint32_t raw_base = is_a ? 0u : (uint32_t)(C::BKN * C::GY_ROWB);
     float dbacc = 0.f;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-
-    // Raw words of one stage: one vector load per token, issued ahead of use.
-    auto load_stage = [&](uint32_t (&buf)[TOK][W], int st) {
-      const int64_t n_st = nbeg + (int64_t)st * TOK;
-#pragma unroll
-      for (int j = 0; j < TOK; ++j) {
-        const int64_t n = n_st + j;
-        if (valid && st < nst && n < nend) {
-          packed::load_words<T>(src + n * pitch, buf[j]);
-        } else {
-#pragma unroll
-          for (int w = 0; w < W; ++w) buf[j][w] = 0u;
-        }
+    for (int st = 0; st < nst; ++st) {
+      if (!wwait_all(&raw_full[s], ph, limit, abort_flag) ||
+          !wwait(&op_empty[s], ph ^ 1, limit, abort_flag, lane)) {
+        ok = false;
+        break;
       }
-    };
-
-    // Write the plane words of one group of 8 tokens (g) into the stage slot.
-    auto store_group = [&](uint32_t (&Pw)[T][4], int g, uint8_t* a_st, uint8_t* b_st) {
-      const uint32_t off = kmajor_off(r, g);
-      if (is_a) {
-#pragma unroll
-        for (int q = 0; q < T; ++q)
-          *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
-              make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
-      } else {
-#pragma unroll
-        for (int f = 0; f < G::nreal; ++f)
-          *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
-              make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
-#pragma unroll
-        for (int k = 1; k <= G::ncomplex; ++k) {
-          const int pr = G::nreal + 2 * (k - 1);
-          const int q = G::nreal + 3 * (k - 1);
-          const uint32_t* re = Pw[pr];
-          const uint32_t* im = Pw[pr + 1];
-          *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(im[0], im[1], im[2], im[3]);
-          *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(re[0], re[1], re[2], re[3]);
-          *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
-              make_uint4(packed::neg2(im[0]), packed::neg2(im[1]), packed::neg2(im[2]), packed::neg2(im[3]));
-        }
-      }
-    };
-
-    // One stage: wait for the slot, transform the buffered tokens, publish.
-    auto run_stage = [&](const uint32_t (&buf)[TOK][W]) -> bool {
-      if (!wwait(&op_empty[s], ph ^ 1, limit, abort_flag)) return false;
       if (active) {
+        const uint8_t* raw = raw_buf + s * C::RAW_BYTES + raw_base + raw_col;
         uint8_t* a_st = a_buf + s * C::A_BYTES;
         uint8_t* b_st = b_buf + s * C::B_BYTES;
 #pragma unroll
-        for (int g = 0; g < TOK / 8; ++g) {
+        for (int g = 0; g < C::BKN / 8; ++g) {
+          uint32_t wv[8][C::W];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint8_t* src = raw + (g * 8 + j) * raw_rowb;
+            if constexpr (C::W == 4) {
+              const uint4 u = *reinterpret_cast<const uint4*>(src);
+              wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
+            } else if constexpr (C::W == 2) {
+              const uint2 u = *reinterpret_cast<const uint2*>(src);
+              wv[j][0] = u.x; wv[j][1] = u.y;
+            } else if constexpr (T == 2) {
+              wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
+            } else {
+              wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+            }
+          }
           uint32_t Pw[T][4];
           if constexpr (T <= 4) {
 #pragma unroll
             for (int pr = 0; pr < 4; ++pr) {
               uint32_t P[T];
-              packed::dft_pair<T, E>(buf[g * 8 + 2 * pr], buf[g * 8 + 2 * pr + 1], P);
+              packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
 #pragma unroll
               for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
               if (is_a) {
@@ -263,88 +246,71 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
                 dbacc += f.x + f.y;
               }
             }
+          } else {
+            // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
+#pragma unroll
+            for (int pr = 0; pr < 4; ++pr) {
+              float Pa[T], Pb[T], va[T], vb[T];
+              const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
+              const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
+#pragma unroll
+              for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
+              G::dft(va, Pa);
+              G::dft(vb, Pb);
+              dbacc += Pa[0] + Pb[0];
+#pragma unroll
+              for (int q = 0; q < T; ++q) {
+                E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
+                Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
+              }
+            }
           }
-          store_group(Pw, g, a_st, b_st);
+          const uint32_t off = kmajor_off(r, g);
+          if (is_a) {
+#pragma unroll
+            for (int q = 0; q < T; ++q)
+              *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
+                  make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+          } else {
+#pragma unroll
+            for (int f = 0; f < G::nreal; ++f)
+              *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
+                  make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
+#pragma unroll
+            for (int k = 1; k <= G::ncomplex; ++k) {
+              const int pr = G::nreal + 2 * (k - 1);
+              const int q = G::nreal + 3 * (k - 1);
+              const uint32_t* re = Pw[pr];
+              const uint32_t* im = Pw[pr + 1];
+              *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(im[0], im[1], im[2], im[3]);
+              *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(re[0], re[1], re[2], re[3]);
+              *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
+                  make_uint4(packed::neg2(im[0]), packed::neg2(im[1]), packed::neg2(im[2]), packed::neg2(im[3]));
+            }
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[s]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&op_full[s]);
       if (++s == C::STAGES) { s = 0; ph ^= 1; }
-      return true;
-    };
-
-    if constexpr (T <= 4) {
-      // double-buffered: the next stage's loads are in flight while this one is transformed
-      uint32_t bufA[TOK][W], bufB[TOK][W];
-      load_stage(bufA, 0);
-      for (int st = 0; st < nst; st += 2) {
-        load_stage(bufB, st + 1);
-        if (!run_stage(bufA)) { ok = false; break; }
-        if (st + 1 >= nst) break;
-        load_stage(bufA, st + 2);
-        if (!run_stage(bufB)) { ok = false; break; }
-      }
-    } else {
-      // T = 8: FP32 butterflies with the sqrt(2)/2 twiddles; loads per group of 8 tokens
-      for (int st = 0; st < nst; ++st) {
-        if (!wwait(&op_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
-        if (active) {
-          uint8_t* a_st = a_buf + s * C::A_BYTES;
-          uint8_t* b_st = b_buf + s * C::B_BYTES;
-          const int64_t n_st = nbeg + (int64_t)st * TOK;
-#pragma unroll 1
-          for (int g = 0; g < TOK / 8; ++g) {
-            uint32_t raw[8][W];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int64_t n = n_st + g * 8 + j;
-              if (valid && n < nend) {
-                packed::load_words<T>(src + n * pitch, raw[j]);
-              } else {
-#pragma unroll
-                for (int w = 0; w < W; ++w) raw[j][w] = 0u;
-              }
-            }
-            float Pf[T][8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const E* e = reinterpret_cast<const E*>(raw[j]);
-              float v[T], Pj[T];
-#pragma unroll
-              for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(e[t]);
-              G::dft(v, Pj);
-#pragma unroll
-              for (int q = 0; q < T; ++q) Pf[q][j] = Pj[q];
-              dbacc += Pj[0];
-            }
-            uint32_t Pw[T][4];
-#pragma unroll
-            for (int q = 0; q < T; ++q) {
-              const uint4 u = pack8<E>(Pf[q]);
-              Pw[q][0] = u.x; Pw[q][1] = u.y; Pw[q][2] = u.z; Pw[q][3] = u.w;
-            }
-            store_group(Pw, g, a_st, b_st);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&op_full[s]);
-        if (++s == C::STAGES) { s = 0; ph ^= 1; }
-      }
     }
     if (!ok) raise_abort(abort_flag, p.err);
 
     if (is_a) {
       // ------------------------------------------------------- epilogue
+      // partial planes [z][T][Cp][Dp]: a warp stores 32 consecutive d of one c
       const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-      bool got = ok && wwait(acc_full, 0, limit, abort_flag);
+      bool got = ok && wwait_all(acc_full, 0, limit, abort_flag);
       if (!got && ok) raise_abort(abort_flag, p.err);
       if (got) {
         tc_fence_after();
-        const bool row_ok = d0 + r < p.Dp;
+        const int d = d0 + r;
+        const bool row_ok = d < p.Dp;
         const int64_t plane = (int64_t)p.Cp * p.Dp;
-        float* base = p.part + (int64_t)z * T * plane + (int64_t)(d0 + r) * p.Cp;
+        float* base = p.part + (int64_t)z * T * plane + d;
 #pragma unroll 1
         for (int cc = 0; cc < BC; cc += 8) {
           uint32_t rg[T][8];
@@ -357,28 +323,51 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
             tmem_ld_32x32b_x8(col + BC, rg[G::nreal + 2 * (k - 1) + 1]);
           }
           tmem_wait_ld();
-          const int c = c0 + cc;
-          if (row_ok && c < p.Cp) {
+          if (row_ok) {
 #pragma unroll
-            for (int q = 0; q < T; ++q) {
-              float* dst = base + q * plane + c;
-              if (c + 8 <= p.Cp) {
-                reinterpret_cast<float4*>(dst)[0] =
-                    make_float4(__uint_as_float(rg[q][0]), __uint_as_float(rg[q][1]),
-                                __uint_as_float(rg[q][2]), __uint_as_float(rg[q][3]));
-                reinterpret_cast<float4*>(dst)[1] =
-                    make_float4(__uint_as_float(rg[q][4]), __uint_as_float(rg[q][5]),
-                                __uint_as_float(rg[q][6]), __uint_as_float(rg[q][7]));
-              } else {
+            for (int q = 0; q < T; ++q)
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  if (c + i < p.Cp) dst[i] = __uint_as_float(rg[q][i]);
+              for (int i = 0; i < 8; ++i) {
+                const int c = c0 + cc + i;
+                if (c < p.Cp) base[q * plane + (int64_t)c * p.Dp] = __uint_as_float(rg[q][i]);
               }
-            }
           }
         }
-        if (c0 == 0 && row_ok) p.dbpart[(int64_t)z * p.Dp + d0 + r] = dbacc;
+        if (c0 == 0 && row_ok) p.dbpart[(int64_t)z * p.Dp + d] = dbacc;
       }
+    }
+  } else if (warp == C::PRODUCER) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t n_raw = 0;
+      bool ok = true;
+      const uint32_t tx = (uint32_t)(C::BKN * (C::GY_ROWB + x_rowb));
+      auto prefetch = [&](int ps) {
+        if (ps >= nst) return;
+        const int n = (int)(nbeg + (int64_t)ps * C::BKN);
+        for (int xb = 0; xb < C::BM * T; xb += C::GY_BOX) tma_prefetch_2d(&map_gy, d0 * T + xb, n);
+        for (int xb = 0; xb < BC * T; xb += p.x_box) tma_prefetch_2d(&map_x, c0 * T + xb, n);
+      };
+      for (int i = 0; i < C::PF_STAGES; ++i) prefetch(i);
+      for (int st = 0; st < nst; ++st) {
+        prefetch(st + C::PF_STAGES);
+        if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&raw_full[s], tx);
+        const int n = (int)(nbeg + (int64_t)st * C::BKN);
+        uint8_t* dst = raw_buf + s * C::RAW_BYTES;
+        for (int b = 0; b < C::BM * T / C::GY_BOX; ++b)
+          tma_load_2d(dst + b * C::BKN * C::GY_BOX * 2, &map_gy, d0 * T + b * C::GY_BOX, n, &raw_full[s]);
+        dst += C::BKN * C::GY_ROWB;
+        for (int b = 0; b < BC * T / p.x_box; ++b)
+          tma_load_2d(dst + b * C::BKN * p.x_box * 2, &map_x, c0 * T + b * p.x_box, n, &raw_full[s]);
+        ++n_raw;
+        if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      }
+      if (!ok) raise_abort(abort_flag, p.err);
+      for (int i = 0; i < C::STAGES; ++i)
+        if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
     }
   } else if (lane == 0) {
     // -------------------------------------------------------------- MMA
@@ -387,40 +376,27 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
     bool ok = true;
     const uint32_t id_real = idesc_f16(p.ab_fmt, (uint32_t)BC);
     const uint32_t id_cplx = idesc_f16(p.ab_fmt, (uint32_t)(2 * BC));
-    // L2 prefetch of the gy and x rows of stage `ps` (this CTA's d and c range)
-    auto prefetch = [&](int ps) {
-      if (ps >= nst) return;
-      const int n = (int)(nbeg + (int64_t)ps * C::BKN);
-      for (int xb = 0; xb < C::BM * T; xb += 256) tma_prefetch_2d(&map_gy, d0 * T + xb, n);
-      for (int xb = 0; xb < BC * T; xb += 256) tma_prefetch_2d(&map_x, c0 * T + xb, n);
-    };
-    for (int i = 0; i < C::PF_STAGES; ++i) prefetch(i);
     for (int st = 0; st < nst; ++st) {
-      prefetch(st + C::PF_STAGES);
       if (!bwait(&op_full[s], ph, limit, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
       const uint32_t b_st = smem_u32(b_buf + s * C::B_BYTES);
+      const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
-      for (int ks = 0; ks < C::BKN / 16; ++ks) {
-        const uint32_t koff = ks * 32;
-        const uint32_t first = (st > 0 || ks > 0) ? 1u : 0u;
+      for (int f = 0; f < G::nreal; ++f)
+        mma_f16_ss(tmem_base + f * BC, smem_desc(a_st + f * C::A_PLANE_BYTES, C::ROWB),
+                   smem_desc(b_st + f * b_plane, C::ROWB), id_real, first);
 #pragma unroll
-        for (int f = 0; f < G::nreal; ++f)
-          mma_f16_ss(tmem_base + f * BC, smem_desc(a_st + f * C::A_PLANE_BYTES + koff, C::ROWB),
-                     smem_desc(b_st + f * b_plane + koff, C::ROWB), id_real, first);
-#pragma unroll
-        for (int k = 1; k <= G::ncomplex; ++k) {
-          const int pr = G::nreal + 2 * (k - 1);
-          const int q = G::nreal + 3 * (k - 1);
-          const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
-          // [Re | Im] += Re G [Re X ; -Im X]
-          mma_f16_ss(col, smem_desc(a_st + pr * C::A_PLANE_BYTES + koff, C::ROWB),
-                     smem_desc(b_st + (q + 1) * b_plane + koff, C::ROWB), id_cplx, first);
-          // [Re | Im] += Im G [Im X ; Re X]
-          mma_f16_ss(col, smem_desc(a_st + (pr + 1) * C::A_PLANE_BYTES + koff, C::ROWB),
-                     smem_desc(b_st + q * b_plane + koff, C::ROWB), id_cplx, 1u);
-        }
+      for (int k = 1; k <= G::ncomplex; ++k) {
+        const int pr = G::nreal + 2 * (k - 1);
+        const int q = G::nreal + 3 * (k - 1);
+        const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
+        // [Re | Im] += Re G [Re X ; -Im X]
+        mma_f16_ss(col, smem_desc(a_st + pr * C::A_PLANE_BYTES, C::ROWB),
+                   smem_desc(b_st + (q + 1) * b_plane, C::ROWB), id_cplx, first);
+        // [Re | Im] += Im G [Im X ; Re X]
+        mma_f16_ss(col, smem_desc(a_st + (pr + 1) * C::A_PLANE_BYTES, C::ROWB),
+                   smem_desc(b_st + q * b_plane, C::ROWB), id_cplx, 1u);
       }
       mma_commit(&op_empty[s]);
       if (++s == C::STAGES) { s = 0; ph ^= 1; }
@@ -433,7 +409,7 @@ tc_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, const __grid_con
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
@@ -488,7 +464,6 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
-  // tensor maps used only for L2 prefetches of the token chunks
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   if (!enc) {
     cudaDriverEntryPointQueryResult q;
@@ -500,20 +475,25 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   }
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // x box: the largest power-of-two width <= 256 elements that divides BC * T
+  int x_box = 256;
+  while ((pl.BC * T) % x_box) x_box >>= 1;
   CUtensorMap map_x, map_gy;
   const void* srcs[2] = {x, gy};
   const int64_t widths[2] = {h.Cp * T, h.Dp * T};
+  const int boxes[2] = {x_box, C::GY_BOX};
   CUtensorMap* maps[2] = {&map_x, &map_gy};
   for (int i = 0; i < 2; ++i) {
     cuuint64_t dims[2] = {(cuuint64_t)widths[i], (cuuint64_t)N};
     cuuint64_t strides[1] = {(cuuint64_t)widths[i] * 2};
-    cuuint32_t box[2] = {(cuuint32_t)(widths[i] < 256 ? widths[i] : 256), (cuuint32_t)C::BKN};
+    cuuint32_t box[2] = {(cuuint32_t)boxes[i], (cuuint32_t)C::BKN};
     cuuint32_t es[2] = {1, 1};
     if (enc(maps[i], dt, 2, const_cast<void*>(srcs[i]), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  p.x_box = x_box;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(tc_dw_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -522,11 +502,11 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
     attr_set = true;
   }
   const unsigned grid = (unsigned)(pl.n_dt * pl.n_ct * pl.splits);
-  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>((const E*)x, (const E*)gy, map_x, map_gy, p);
+  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(map_x, map_gy, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);
-  return launch_dw_reduce(h, pl.splits, p.part, p.dbpart, dW, db, st);
+  return launch_dw_reduce(h, pl.splits, p.part, p.dbpart, dW, db, /*cd_layout=*/true, st);
 }
 
 template <typename E>
