@@ -128,6 +128,8 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
     return EQLIN_ERR_OOM;
   }
   h.backend = (dtype == EQLIN_F32) ? "simt" : (eqlin::tc_supported(h, false) ? "tcgen05" : "simt");
+  h.need_simt_fwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, false);
+  h.need_simt_bwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, true);
   *out = hh;
   return EQLIN_OK;
 }

@@ -144,6 +144,8 @@ struct Handle {
   // (-Im, Re, Im stacked so that [Re;Im] and [-Im;Re] are contiguous windows).
   void* wt_fwd = nullptr;
   void* wt_bwd = nullptr;
+  bool need_simt_fwd = true;      // FP32 planes needed (SIMT serves forward / dx)
+  bool need_simt_bwd = true;
   float* bias = nullptr;          // [Dp] float32 (zeros when no bias)
   float* ws = nullptr;            // dW split partials
   size_t ws_bytes = 0;

@@ -54,6 +54,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Upper bound on the wall time of any single wait, whatever the poll limit.
 constexpr uint64_t kWaitTimeNs = 2000000000ull;
 
+// Non-blocking check that the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed; false after
 // `limit` polls or kWaitTimeNs, whichever comes first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {

@@ -17,68 +17,104 @@
 namespace eqlin {
 
 // ========================================================== weight transform
-// One thread per (d, c): the DFT of W[d, c, 0..T) along tau, written as
-//   wf_fwd[p][c][d]  (FP32, forward planes)
+// One 32 (c) x 32 (d) tile per block: the DFT of W[d, c, 0..T) along tau,
+// written as
+//   wf_fwd[p][c][d]  (FP32, forward planes; SIMT kernels only)
 //   wf_bwd[p][d][c]  (FP32, conjugated: the dx product uses conj(W_hat))
 //   wt_fwd[q][d][c], wt_bwd[q][c][d]  (handle dtype, tensor-core operand
 //   planes scaled by 1/T (real) or 2/T (complex); q enumerates real
 //   frequencies, then (-Im, Re, Im) triples)
+// Every output row is written with consecutive threads on consecutive
+// addresses; the transposed planes go through a shared-memory tile.
+namespace pt {
+constexpr int TILE = 32, ROWS = 8;   // block = 32 x 8 threads
+}
+
 template <int T, typename E>
-__global__ void pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b,
-                                    float* __restrict__ wf_fwd, float* __restrict__ wf_bwd,
-                                    E* __restrict__ wt_fwd, E* __restrict__ wt_bwd,
-                                    float* __restrict__ bias, int Cp, int Dp) {
+__global__ void __launch_bounds__(pt::TILE * pt::ROWS)
+pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __restrict__ wf_fwd,
+                    float* __restrict__ wf_bwd, E* __restrict__ wt_fwd, E* __restrict__ wt_bwd,
+                    float* __restrict__ bias, int Cp, int Dp) {
   using G = Group<T>;
-  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)Cp * Dp;
-  if (idx < Dp) bias[idx] = b ? Elem<E>::to_f(b[idx]) : 0.f;
-  if (idx >= total) return;
-  const int d = (int)(idx % Dp), c = (int)(idx / Dp);    // d fastest: coalesced wf_fwd writes
-  float v[T], P[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(W[((int64_t)d * Cp + c) * T + t]);
-  G::dft(v, P);
+  using namespace pt;
+  constexpr int Q = G::nreal + 3 * G::ncomplex;
+  __shared__ float sP[T][TILE][TILE + 1];        // planes of the tile, [p][d][c]
+  const int c0 = blockIdx.x * TILE, d0 = blockIdx.y * TILE;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  if (blockIdx.x == 0 && ty == 0)
+    for (int d = d0 + tx; d < d0 + TILE && d < Dp; d += TILE) bias[d] = b ? Elem<E>::to_f(b[d]) : 0.f;
   const int64_t plane = (int64_t)Cp * Dp;
+  // pass 1: thread (tx = c, rows d): DFT, write the [d][c]-ordered planes
 #pragma unroll
-  for (int p = 0; p < T; ++p) {
-    const bool imag = p >= G::nreal && ((p - G::nreal) & 1);
-    wf_fwd[p * plane + (int64_t)c * Dp + d] = P[p];
-    wf_bwd[p * plane + (int64_t)d * Cp + c] = imag ? -P[p] : P[p];
-  }
-  if (wt_fwd) {
-    // The tensor-core planes carry the inverse DFT's scales (1/T for a real
-    // frequency, 2/T for a complex one; exact powers of two), so that the
-    // kernels' epilogue is only additions.
-    const float sr = 1.f / T, sc = 2.f / T;
+  for (int i = 0; i < TILE / ROWS; ++i) {
+    const int dl = ty + i * ROWS, d = d0 + dl, c = c0 + tx;
+    float v[T], P[T];
+    const bool ok = d < Dp && c < Cp;
 #pragma unroll
-    for (int f = 0; f < G::nreal; ++f) {
-      wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f] * sr);
-      wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f] * sr);
+    for (int t = 0; t < T; ++t) v[t] = ok ? Elem<E>::to_f(W[((int64_t)d * Cp + c) * T + t]) : 0.f;
+    G::dft(v, P);
+#pragma unroll
+    for (int q = 0; q < T; ++q) sP[q][dl][tx] = P[q];
+    if (!ok) continue;
+    if (wf_bwd) {
+#pragma unroll
+      for (int q = 0; q < T; ++q) {
+        const bool imag = q >= G::nreal && ((q - G::nreal) & 1);
+        wf_bwd[q * plane + (int64_t)d * Cp + c] = imag ? -P[q] : P[q];
+      }
     }
+    if (wt_fwd) {
+      const float sr = 1.f / T, sc = 2.f / T;
 #pragma unroll
-    for (int k = 1; k <= G::ncomplex; ++k) {
-      const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
-      const int q = G::nreal + 3 * (k - 1);
-      // forward: (-Im, Re, Im); backward uses conj(W_hat): Im -> -Im
-      wt_fwd[(q + 0) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(-im);
-      wt_fwd[(q + 1) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(re);
-      wt_fwd[(q + 2) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(im);
-      wt_bwd[(q + 0) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(im);
-      wt_bwd[(q + 1) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(re);
-      wt_bwd[(q + 2) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(-im);
+      for (int f = 0; f < G::nreal; ++f) wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f] * sr);
+#pragma unroll
+      for (int k = 1; k <= G::ncomplex; ++k) {
+        const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
+        const int q = G::nreal + 3 * (k - 1);
+        wt_fwd[(q + 0) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(-im);
+        wt_fwd[(q + 1) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(re);
+        wt_fwd[(q + 2) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(im);
+      }
     }
   }
+  __syncthreads();
+  // pass 2: thread (tx = d, rows c): the [c][d]-ordered planes
+#pragma unroll
+  for (int i = 0; i < TILE / ROWS; ++i) {
+    const int cl = ty + i * ROWS, c = c0 + cl, d = d0 + tx;
+    if (d >= Dp || c >= Cp) continue;
+    float P[T];
+#pragma unroll
+    for (int q = 0; q < T; ++q) P[q] = sP[q][tx][cl];
+    if (wf_fwd) {
+#pragma unroll
+      for (int q = 0; q < T; ++q) wf_fwd[q * plane + (int64_t)c * Dp + d] = P[q];
+    }
+    if (wt_bwd) {
+      const float sr = 1.f / T, sc = 2.f / T;
+#pragma unroll
+      for (int f = 0; f < G::nreal; ++f) wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f] * sr);
+#pragma unroll
+      for (int k = 1; k <= G::ncomplex; ++k) {
+        const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
+        const int q = G::nreal + 3 * (k - 1);
+        // the input gradient uses conj(W_hat): Im -> -Im
+        wt_bwd[(q + 0) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(im);
+        wt_bwd[(q + 1) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(re);
+        wt_bwd[(q + 2) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(-im);
+      }
+    }
+  }
+  (void)Q;
 }
 
 template <int T, typename E>
 static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b, cudaStream_t st) {
-  const int64_t total = h.Cp * h.Dp;
-  const int64_t work = total > h.Dp ? total : h.Dp;
-  const int threads = 256;
-  const unsigned blocks = (unsigned)((work + threads - 1) / threads);
-  pretransform_kernel<T, E><<<blocks, threads, 0, st>>>(
-      (const E*)W, (const E*)b, h.wf_fwd, h.wf_bwd, (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias,
-      (int)h.Cp, (int)h.Dp);
+  dim3 grid((unsigned)((h.Cp + pt::TILE - 1) / pt::TILE), (unsigned)((h.Dp + pt::TILE - 1) / pt::TILE));
+  dim3 block(pt::TILE, pt::ROWS);
+  pretransform_kernel<T, E><<<grid, block, 0, st>>>(
+      (const E*)W, (const E*)b, h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr,
+      (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -376,34 +412,80 @@ simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restr
 
 // Sum the splits in index order, then inverse DFT along the frequency planes.
 // Partials are [splits][T][Dp][Cp] (cd_layout false) or [splits][T][Cp][Dp]
-// (cd_layout true); threads walk the partials' contiguous index.
+// (cd_layout true).  One block per 32 x 32 (d, c) tile: threads read the
+// partials along their contiguous index, sum the splits in index order, take
+// the inverse DFT and stage the tile in shared memory so that dW [Dp][Cp][T]
+// is written row by row.
 template <int T>
-__global__ void dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart,
-                                 float* __restrict__ dW, float* __restrict__ db, int splits,
-                                 int Cp, int Dp, bool cd_layout) {
+__global__ void __launch_bounds__(256)
+dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart, float* __restrict__ dW,
+                 float* __restrict__ db, int splits, int Cp, int Dp, bool cd_layout) {
   using G = Group<T>;
-  const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  __shared__ float sV[32][32 * T + 1];            // [d][c*T + t] of the tile
+  const int c0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;   // 32 x 8
   const int64_t plane = (int64_t)Cp * Dp;
-  if (idx < plane) {
-    float P[T], v[T];
 #pragma unroll
-    for (int p = 0; p < T; ++p) {
-      float s = 0.f;
-      for (int z = 0; z < splits; ++z) s += part[((int64_t)z * T + p) * plane + idx];
-      P[p] = s;
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty + 8 * i;
+    // contiguous index along tx: d for the [c][d] layout, c for [d][c]
+    const int d = cd_layout ? d0 + tx : d0 + r;
+    const int c = cd_layout ? c0 + r : c0 + tx;
+    float P[T], v[T];
+    if (d < Dp && c < Cp) {
+      const int64_t idx = cd_layout ? (int64_t)c * Dp + d : (int64_t)d * Cp + c;
+#pragma unroll
+      for (int q = 0; q < T; ++q) {
+        float s = 0.f;
+        for (int z = 0; z < splits; ++z) s += part[((int64_t)z * T + q) * plane + idx];
+        P[q] = s;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < T; ++q) P[q] = 0.f;
     }
     G::idft(P, v);
-    const int64_t d = cd_layout ? idx % Dp : idx / Cp;
-    const int64_t c = cd_layout ? idx / Dp : idx % Cp;
-    // dW is [Dp][Cp][T]
+    const int dl = d - d0, cl = c - c0;
 #pragma unroll
-    for (int t = 0; t < T; ++t) dW[(d * Cp + c) * T + t] = v[t];
+    for (int t = 0; t < T; ++t) sV[dl][cl * T + t] = v[t];
   }
-  if (db && idx < Dp) {
-    float s = 0.f;
-    for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + idx];
-    db[idx] = s;
+  __syncthreads();
+  // write: for each d row of the tile, 32*T contiguous floats
+  const int ncol = min(32, Cp - c0) * T;
+  for (int r = ty; r < 32; r += 8) {
+    const int d = d0 + r;
+    if (d >= Dp) continue;
+    float* dst = dW + ((int64_t)d * Cp + c0) * T;
+    for (int j = tx; j < ncol; j += 32) dst[j] = sV[r][j];
   }
+  if (db && blockIdx.x == 0 && ty == 0) {
+    const int d = d0 + tx;
+    if (d < Dp) {
+      float s = 0.f;
+      for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + d];
+      db[d] = s;
+    }
+  }
+}
+
+template <int T>
+static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
+                               float* dW, float* db, bool cd_layout, cudaStream_t st) {
+  dim3 grid((unsigned)((h.Cp + 31) / 32), (unsigned)((h.Dp + 31) / 32));
+  dw_reduce_kernel<T><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp, cd_layout);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
+                             float* dW, float* db, bool cd_layout, cudaStream_t st) {
+  switch (h.T) {
+    case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, cd_layout, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int T, typename E>
@@ -424,28 +506,6 @@ static cudaError_t simt_dw_t(const Handle& h, const void* x, const void* gy, flo
   if (e != cudaSuccess) return e;
   count_launches(1);
   return launch_dw_reduce(h, splits, part, dbpart, dW, db, /*cd_layout=*/false, st);
-}
-
-template <int T>
-static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
-                               float* dW, float* db, bool cd_layout, cudaStream_t st) {
-  const int64_t plane = h.Cp * h.Dp;
-  const int64_t work = plane > h.Dp ? plane : h.Dp;
-  dw_reduce_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(part, dbpart, dW, db, splits,
-                                                                      (int)h.Cp, (int)h.Dp, cd_layout);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
-                             float* dW, float* db, bool cd_layout, cudaStream_t st) {
-  switch (h.T) {
-    case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, cd_layout, st);
-    case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, cd_layout, st);
-    case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, cd_layout, st);
-    case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, cd_layout, st);
-  }
-  return cudaErrorInvalidValue;
 }
 
 template <typename E>

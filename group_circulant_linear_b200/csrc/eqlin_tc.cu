@@ -73,12 +73,12 @@ struct Cfg {
   static constexpr int STAGE_BYTES = RAW_BYTES + A_BYTES + B_BYTES;
   // output staging for the TMA stores: per epilogue half one [128 rows x 128 B] tile
   static constexpr int OUT_EL = 64;                    // output elements per row per store
-  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2;
-  static constexpr int STAGES_FIT = (220 * 1024 - 2 * OUT_TILE_BYTES) / STAGE_BYTES;
+  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2; // two per epilogue half (double buffer)
+  static constexpr int STAGES_FIT = (220 * 1024 - 4 * OUT_TILE_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(STAGES >= 2, "two stages must fit");
-  static constexpr int NBAR = 5 * STAGES + 2 * NACC + 1;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * OUT_TILE_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int NBAR = 4 * STAGES + 2 * NACC + 1;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * OUT_TILE_BYTES + NBAR * 8 + 16 + 1024;
   static constexpr int CH = OUT_EL / T;                // output channels per store chunk
   static constexpr int NCHUNK = BO / CH;               // store chunks per tile (even)
   static_assert(NCHUNK % 2 == 0, "chunks alternate between the two epilogue halves");
@@ -107,6 +107,7 @@ struct Params {
 // Bounded wait that also gives up as soon as another role raised the abort flag.
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t limit,
                                       volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;     // already complete: no suspension
   uint64_t t0 = 0;
   for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -178,10 +179,10 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
   uint8_t* b_buf = a_buf + C::STAGES * C::A_BYTES;
   uint8_t* raw_buf = b_buf + C::STAGES * C::B_BYTES;
   uint8_t* o_buf = raw_buf + C::STAGES * C::RAW_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(o_buf + 2 * C::OUT_TILE_BYTES);
-  uint64_t* a_full = bars;
-  uint64_t* b_full = a_full + C::STAGES;
-  uint64_t* ab_empty = b_full + C::STAGES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_buf + 4 * C::OUT_TILE_BYTES);
+  // stage_full: the 8 transform warps' A planes and the producer's B planes (tx)
+  uint64_t* stage_full = bars;
+  uint64_t* ab_empty = stage_full + C::STAGES;
   uint64_t* raw_full = ab_empty + C::STAGES;
   uint64_t* raw_empty = raw_full + C::STAGES;
   uint64_t* acc_full = raw_empty + C::STAGES;
@@ -198,8 +199,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&a_full[i], C::TR_WARPS);
-      mbar_init(&b_full[i], 1);
+      mbar_init(&stage_full[i], C::TR_WARPS + 1);
       mbar_init(&ab_empty[i], 1);
       mbar_init(&raw_full[i], 1);
       mbar_init(&raw_empty[i], C::TR_WARPS);
@@ -237,11 +237,9 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
     uint32_t ph = 0;
     bool ok = true;
     for (int64_t it = 0; it < my_tiles * nk; ++it) {
-      if (!wwait_all(&raw_full[s], ph, limit, abort_flag) ||
-          !wwait(&ab_empty[s], ph ^ 1, limit, abort_flag, lane)) {
-        ok = false;
-        break;
-      }
+      // raw_full also means A slot s is free: the producer loads raw[s] only
+      // after the MMAs that read A[s] have completed
+      if (!wwait_all(&raw_full[s], ph, limit, abort_flag)) { ok = false; break; }
       const uint8_t* raw = raw_buf + s * C::RAW_BYTES + raw_off;
       uint32_t wv[8][C::W];
 #pragma unroll
@@ -294,7 +292,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
         *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES) = make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[s]);
+      if (lane == 0) mbar_arrive(&stage_full[s]);
       if (++s == C::STAGES) { s = 0; ph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
@@ -321,17 +319,20 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
         const int o0 = (tile % p.n_otiles) * C::BO;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
-          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
-          tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
-          ++n_raw;
-          if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&b_full[s], C::B_BYTES);
+          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag) ||
+              !bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&stage_full[s], C::B_BYTES);
           uint8_t* bdst = b_buf + s * C::B_BYTES;
 #pragma unroll
           for (int q = 0; q < C::Q; ++q)
-            tma_load_3d(bdst + q * C::B_PLANE_BYTES, &map_w, kb * C::BK, o0, q, &b_full[s]);
+            tma_load_3d(bdst + q * C::B_PLANE_BYTES, &map_w, kb * C::BK, o0, q, &stage_full[s]);
           ++n_b;
+          mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
+          tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
+          ++n_raw;
           if (++s == C::STAGES) { s = 0; ph ^= 1; }
         }
       }
@@ -339,7 +340,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
       // every issued TMA copy must land before the CTA exits (a no-op on the
       // normal path, where the MMA thread already waited for them)
       for (int i = 0; i < C::STAGES; ++i) {
-        if (n_b > i) mbar_wait(&b_full[i], (uint32_t)(((n_b - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
+        if (n_b > i) mbar_wait(&stage_full[i], (uint32_t)(((n_b - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
         if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
       }
     }
@@ -357,10 +358,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&a_full[s], ph, limit, abort_flag) || !bwait(&b_full[s], ph, limit, abort_flag)) {
-            ok = false;
-            break;
-          }
+          if (!bwait(&stage_full[s], ph, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
           const uint32_t b_st = smem_u32(b_buf + s * C::B_BYTES);
@@ -408,8 +406,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const bool issuer = (e & 3) == 0 && lane == 0;
-    uint8_t* stage_tile = o_buf + half * C::OUT_TILE_BYTES;
-    uint8_t* my_row = stage_tile + r * 128;
+    int sb = 0;                                      // staging buffer of this half (0/1)
     int ab = 0;
     uint32_t aph = 0;
     bool ok = true;
@@ -424,8 +421,10 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
       const uint32_t acc = tmem_base + lane_addr + ab * C::ACC_COLS;
 #pragma unroll 1
       for (int ci = half; ci < C::NCHUNK; ci += 2) {
-        // the previous TMA store from this staging tile must have read it
-        if (issuer) bulk_wait_read<0>();
+        uint8_t* stage_tile = o_buf + (half * 2 + sb) * C::OUT_TILE_BYTES;
+        uint8_t* my_row = stage_tile + r * 128;
+        // the TMA store issued from this staging tile two chunks ago must have read it
+        if (issuer) bulk_wait_read<1>();
         named_bar_sync(1 + half, 128);
 #pragma unroll
         for (int sub = 0; sub < C::CH / 8; ++sub) {
@@ -446,6 +445,16 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
             mbar_arrive(&acc_empty[ab]);
           }
           const int o = o0 + oc;
+          float bo8[8];
+          if (p.bias && o + 8 <= p.O) {
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + o));
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + o) + 1);
+            bo8[0] = b0.x; bo8[1] = b0.y; bo8[2] = b0.z; bo8[3] = b0.w;
+            bo8[4] = b1.x; bo8[5] = b1.y; bo8[6] = b1.z; bo8[7] = b1.w;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) bo8[c] = (p.bias && o + c < p.O) ? __ldg(p.bias + o + c) : 0.f;
+          }
           // 8 channels x T outputs = T 16-byte chunks of this row's 128 bytes;
           // chunk v holds the outputs of channels v*8/T .. (v+1)*8/T - 1
 #pragma unroll
@@ -454,7 +463,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
 #pragma unroll
             for (int cc = 0; cc < 8 / T; ++cc) {
               const int c = v * (8 / T) + cc;
-              const float bo = (p.bias && o + c < p.O) ? __ldg(p.bias + o + c) : 0.f;
+              const float bo = bo8[c];
               float Pc[T];
 #pragma unroll
               for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][c]);
@@ -470,6 +479,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
           tma_store_2d(&map_out, stage_tile, (o0 + ci * C::CH) * T, m0);
           bulk_commit();
         }
+        sb ^= 1;
       }
       if (++ab == C::NACC) { ab = 0; aph ^= 1; }
     }
