@@ -31,7 +31,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from group_circulant_linear_b200 import inputs, workloads  # noqa: E402
+from group_circulant_linear_b200 import dp, inputs, workloads  # noqa: E402
 
 METRIC = "EQ-Linear p4 fwd+bwd TFLOP/s (dense-equiv) & fraction of tensor-pipe roofline"
 UNIT = "TFLOP/s"
@@ -272,8 +272,7 @@ def main():
                 else:
                     fn()
             if dist:
-                torch.distributed.all_reduce(s["dW"])
-                torch.distributed.all_reduce(s["db"])
+                dp.allreduce_grads((s["dW"], s["db"]))
 
     def barrier():
         if dist:
@@ -360,8 +359,7 @@ def main():
                 eqlin.backward_dx(s["h"], db_["gy"], s["dx"])
                 eqlin.backward_dw(s["h"], db_["x"], db_["gy"], s["dW"], s["db"])
                 if dist:
-                    torch.distributed.all_reduce(s["dW"])
-                    torch.distributed.all_reduce(s["db"])
+                    dp.allreduce_grads((s["dW"], s["db"]))
                 for k in ("y", "dx", "dW", "db"):
                     hb[k].copy_(s[k], non_blocking=True)
 
