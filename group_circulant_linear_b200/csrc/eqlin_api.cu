@@ -105,7 +105,6 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
     return EQLIN_ERR_CUDA;
   }
   const size_t planes = (size_t)T * Cp * Dp;
-  const int Q = (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
   if (dtype != EQLIN_F32) {
     const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
@@ -117,8 +116,10 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
             cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
             cudaMalloc(&h.err, sizeof(int)) == cudaSuccess;
   if (ok && dtype != EQLIN_F32) {
-    ok = cudaMalloc(&h.wt_fwd, (size_t)Q * Cp * Dp * e) == cudaSuccess &&
-         cudaMalloc(&h.wt_bwd, (size_t)Q * Cp * Dp * e) == cudaSuccess;
+    const size_t nf = (size_t)eqlin::wtile_elems(T, Dp, Cp), nb = (size_t)eqlin::wtile_elems(T, Cp, Dp);
+    ok = cudaMalloc(&h.wt_fwd, nf * e) == cudaSuccess && cudaMalloc(&h.wt_bwd, nb * e) == cudaSuccess;
+    // padding rows and K columns of the tiles stay zero
+    if (ok) ok = cudaMemset(h.wt_fwd, 0, nf * e) == cudaSuccess && cudaMemset(h.wt_bwd, 0, nb * e) == cudaSuccess;
   }
   if (ok) ok = cudaMemset(h.err, 0, sizeof(int)) == cudaSuccess;
   if (!ok) {

@@ -127,6 +127,32 @@ template <int T> struct Group {
   }
 };
 
+// --------------------------------------------- tensor-core weight tiles
+// The tensor-core kernels read the Fourier weight planes as tiles of BO
+// output rows x 16 K (input channels), one per (output tile, K stage) and
+// plane, stored in the exact 32-byte-swizzled image the MMA reads from shared
+// memory, so that one contiguous bulk copy fetches a stage.  For K-major rows
+// of 32 bytes, 16-byte chunk j of row r sits at chunk j ^ ((r >> 2) & 1).
+constexpr int TC_BK = 16;
+__host__ __device__ constexpr int tc_bo(int T) { return T == 1 ? 256 : T == 2 ? 128 : T == 4 ? 128 : 32; }
+__host__ __device__ constexpr int tc_planes(int T) {
+  return (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
+}
+// Element index of (row, k, plane q) in a tiled weight buffer with n_kb K stages.
+__host__ __device__ inline int64_t wtile_index(int T, int64_t n_kb, int64_t row, int64_t k, int q) {
+  const int bo = tc_bo(T), Q = tc_planes(T);
+  const int64_t ot = row / bo, kb = k / TC_BK;
+  const int r = (int)(row % bo), kk = (int)(k % TC_BK);
+  const int64_t tile = (ot * n_kb + kb) * Q + q;
+  const int64_t byte = tile * bo * 32 + r * 32 + ((((kk >> 3) ^ ((r >> 2) & 1))) << 4) + (kk & 7) * 2;
+  return byte / 2;
+}
+// Elements of a tiled buffer for `rows` output rows and K = `kdim`.
+__host__ __device__ inline int64_t wtile_elems(int T, int64_t rows, int64_t kdim) {
+  const int bo = tc_bo(T);
+  return ((rows + bo - 1) / bo) * ((kdim + TC_BK - 1) / TC_BK) * tc_planes(T) * bo * TC_BK;
+}
+
 // ------------------------------------------------------------------ handle
 struct Handle {
   int T = 0;
@@ -139,9 +165,10 @@ struct Handle {
   // channel, contiguous over output channel); bwd [T][Dp][Cp], conjugated.
   float* wf_fwd = nullptr;
   float* wf_bwd = nullptr;
-  // Fourier planes in the handle dtype for the tensor-core kernels, K-major:
-  // fwd [Q][Dp][Cp], bwd [Q][Cp][Dp]; Q = real freqs + 3 per complex freq
-  // (-Im, Re, Im stacked so that [Re;Im] and [-Im;Re] are contiguous windows).
+  // Fourier planes in the handle dtype for the tensor-core kernels, tiled as
+  // above: fwd rows D' x K C', bwd rows C' x K D' (conjugated); Q = real
+  // freqs + 3 per complex freq (-Im, Re, Im stacked so that [Re;Im] and
+  // [-Im;Re] are contiguous windows of a stage).
   void* wt_fwd = nullptr;
   void* wt_bwd = nullptr;
   bool need_simt_fwd = true;      // FP32 planes needed (SIMT serves forward / dx)

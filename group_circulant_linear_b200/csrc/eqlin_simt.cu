@@ -21,11 +21,11 @@ namespace eqlin {
 // written as
 //   wf_fwd[p][c][d]  (FP32, forward planes; SIMT kernels only)
 //   wf_bwd[p][d][c]  (FP32, conjugated: the dx product uses conj(W_hat))
-//   wt_fwd[q][d][c], wt_bwd[q][c][d]  (handle dtype, tensor-core operand
-//   planes scaled by 1/T (real) or 2/T (complex); q enumerates real
-//   frequencies, then (-Im, Re, Im) triples)
-// Every output row is written with consecutive threads on consecutive
-// addresses; the transposed planes go through a shared-memory tile.
+//   wt_fwd (rows d, K c), wt_bwd (rows c, K d): handle dtype, tensor-core
+//   operand tiles (see wtile_index) scaled by 1/T (real) or 2/T (complex);
+//   q enumerates real frequencies, then (-Im, Re, Im) triples
+// The FP32 planes are written with consecutive threads on consecutive
+// addresses; the transposed ones go through a shared-memory tile.
 namespace pt {
 constexpr int TILE = 32, ROWS = 8;   // block = 32 x 8 threads
 }
@@ -64,16 +64,18 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
       }
     }
     if (wt_fwd) {
+      // forward tiles: rows d, K = c
       const float sr = 1.f / T, sc = 2.f / T;
+      const int64_t nkb = (Cp + TC_BK - 1) / TC_BK;
 #pragma unroll
-      for (int f = 0; f < G::nreal; ++f) wt_fwd[f * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(P[f] * sr);
+      for (int f = 0; f < G::nreal; ++f) wt_fwd[wtile_index(T, nkb, d, c, f)] = Elem<E>::from_f(P[f] * sr);
 #pragma unroll
       for (int k = 1; k <= G::ncomplex; ++k) {
         const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
         const int q = G::nreal + 3 * (k - 1);
-        wt_fwd[(q + 0) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(-im);
-        wt_fwd[(q + 1) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(re);
-        wt_fwd[(q + 2) * plane + (int64_t)d * Cp + c] = Elem<E>::from_f(im);
+        wt_fwd[wtile_index(T, nkb, d, c, q + 0)] = Elem<E>::from_f(-im);
+        wt_fwd[wtile_index(T, nkb, d, c, q + 1)] = Elem<E>::from_f(re);
+        wt_fwd[wtile_index(T, nkb, d, c, q + 2)] = Elem<E>::from_f(im);
       }
     }
   }
@@ -91,17 +93,18 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
       for (int q = 0; q < T; ++q) wf_fwd[q * plane + (int64_t)c * Dp + d] = P[q];
     }
     if (wt_bwd) {
+      // input-gradient tiles: rows c, K = d; conj(W_hat): Im -> -Im
       const float sr = 1.f / T, sc = 2.f / T;
+      const int64_t nkb = (Dp + TC_BK - 1) / TC_BK;
 #pragma unroll
-      for (int f = 0; f < G::nreal; ++f) wt_bwd[f * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(P[f] * sr);
+      for (int f = 0; f < G::nreal; ++f) wt_bwd[wtile_index(T, nkb, c, d, f)] = Elem<E>::from_f(P[f] * sr);
 #pragma unroll
       for (int k = 1; k <= G::ncomplex; ++k) {
         const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
         const int q = G::nreal + 3 * (k - 1);
-        // the input gradient uses conj(W_hat): Im -> -Im
-        wt_bwd[(q + 0) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(im);
-        wt_bwd[(q + 1) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(re);
-        wt_bwd[(q + 2) * plane + (int64_t)c * Dp + d] = Elem<E>::from_f(-im);
+        wt_bwd[wtile_index(T, nkb, c, d, q + 0)] = Elem<E>::from_f(im);
+        wt_bwd[wtile_index(T, nkb, c, d, q + 1)] = Elem<E>::from_f(re);
+        wt_bwd[wtile_index(T, nkb, c, d, q + 2)] = Elem<E>::from_f(-im);
       }
     }
   }
@@ -412,58 +415,64 @@ simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restr
 
 // Sum the splits in index order, then inverse DFT along the frequency planes.
 // Partials are [splits][T][Dp][Cp] (cd_layout false) or [splits][T][Cp][Dp]
-// (cd_layout true).  One block per 32 x 32 (d, c) tile: threads read the
-// partials along their contiguous index, sum the splits in index order, take
-// the inverse DFT and stage the tile in shared memory so that dW [Dp][Cp][T]
-// is written row by row.
+// (cd_layout true).  One block of 32 x 8 threads per 32 (d) x 8 (c) tile,
+// one element per thread: it sums the splits in index order (four partial
+// sums kept apart, combined in a fixed order), takes the inverse DFT and
+// stages the tile in shared memory so that dW [Dp][Cp][T] is written row by
+// row.
 template <int T>
 __global__ void __launch_bounds__(256)
 dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart, float* __restrict__ dW,
                  float* __restrict__ db, int splits, int Cp, int Dp, bool cd_layout) {
   using G = Group<T>;
-  __shared__ float sV[32][32 * T + 1];            // [d][c*T + t] of the tile
-  const int c0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;   // 32 x 8
+  __shared__ float sV[32][8 * T + 1];             // [d][c*T + t] of the tile
+  const int c0 = blockIdx.x * 8, d0 = blockIdx.y * 32;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
   const int64_t plane = (int64_t)Cp * Dp;
+  // thread -> (d, c): the partials' contiguous index runs along tx
+  int d, c;
+  if (cd_layout) { d = d0 + tx; c = c0 + ty; }
+  else { d = d0 + (threadIdx.x >> 3); c = c0 + (threadIdx.x & 7); }
+  float P[T], v[T];
+  if (d < Dp && c < Cp) {
+    const int64_t idx = cd_layout ? (int64_t)c * Dp + d : (int64_t)d * Cp + c;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty + 8 * i;
-    // contiguous index along tx: d for the [c][d] layout, c for [d][c]
-    const int d = cd_layout ? d0 + tx : d0 + r;
-    const int c = cd_layout ? c0 + r : c0 + tx;
-    float P[T], v[T];
-    if (d < Dp && c < Cp) {
-      const int64_t idx = cd_layout ? (int64_t)c * Dp + d : (int64_t)d * Cp + c;
-#pragma unroll
-      for (int q = 0; q < T; ++q) {
-        float s = 0.f;
-        for (int z = 0; z < splits; ++z) s += part[((int64_t)z * T + q) * plane + idx];
-        P[q] = s;
+    for (int q = 0; q < T; ++q) {
+      const float* src = part + (int64_t)q * plane + idx;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      int z = 0;
+      for (; z + 4 <= splits; z += 4) {
+        s0 += src[(int64_t)(z + 0) * T * plane];
+        s1 += src[(int64_t)(z + 1) * T * plane];
+        s2 += src[(int64_t)(z + 2) * T * plane];
+        s3 += src[(int64_t)(z + 3) * T * plane];
       }
-    } else {
-#pragma unroll
-      for (int q = 0; q < T; ++q) P[q] = 0.f;
+      for (; z < splits; ++z) s0 += src[(int64_t)z * T * plane];
+      P[q] = (s0 + s1) + (s2 + s3);
     }
-    G::idft(P, v);
-    const int dl = d - d0, cl = c - c0;
+  } else {
 #pragma unroll
-    for (int t = 0; t < T; ++t) sV[dl][cl * T + t] = v[t];
+    for (int q = 0; q < T; ++q) P[q] = 0.f;
   }
+  G::idft(P, v);
+  const int dl = d - d0, cl = c - c0;
+#pragma unroll
+  for (int t = 0; t < T; ++t) sV[dl][cl * T + t] = v[t];
   __syncthreads();
-  // write: for each d row of the tile, 32*T contiguous floats
-  const int ncol = min(32, Cp - c0) * T;
+  // each warp writes rows of 8*T contiguous floats
+  const int ncol = min(8, Cp - c0) * T;
   for (int r = ty; r < 32; r += 8) {
-    const int d = d0 + r;
-    if (d >= Dp) continue;
-    float* dst = dW + ((int64_t)d * Cp + c0) * T;
+    const int dd = d0 + r;
+    if (dd >= Dp) continue;
+    float* dst = dW + ((int64_t)dd * Cp + c0) * T;
     for (int j = tx; j < ncol; j += 32) dst[j] = sV[r][j];
   }
   if (db && blockIdx.x == 0 && ty == 0) {
-    const int d = d0 + tx;
-    if (d < Dp) {
+    const int dd = d0 + tx;
+    if (dd < Dp) {
       float s = 0.f;
-      for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + d];
-      db[d] = s;
+      for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + dd];
+      db[dd] = s;
     }
   }
 }
@@ -471,7 +480,7 @@ dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpar
 template <int T>
 static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
                                float* dW, float* db, bool cd_layout, cudaStream_t st) {
-  dim3 grid((unsigned)((h.Cp + 31) / 32), (unsigned)((h.Dp + 31) / 32));
+  dim3 grid((unsigned)((h.Cp + 7) / 8), (unsigned)((h.Dp + 31) / 32));
   dw_reduce_kernel<T><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp, cd_layout);
   count_launches(1);
   return cudaGetLastError();

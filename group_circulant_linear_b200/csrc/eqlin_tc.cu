@@ -6,8 +6,9 @@
 // channels:
 //
 //   producer warp    (8)    TMA: the raw input tile of the stage [128 tokens x
-//                    16*T elements], the Fourier weight planes of the stage,
-//                    and L2 prefetches of raw tiles several stages ahead
+//                    16*T elements]; one bulk copy of the stage's Fourier
+//                    weight planes (stored pre-swizzled per stage); L2
+//                    prefetches of raw tiles several stages ahead
 //   transform warps  (0-7)  one thread per (input channel, 8 tokens): read the
 //                    channel's T group values of its tokens from the raw tile,
 //                    take the group DFT (adds/subtracts on packed token pairs
@@ -51,9 +52,9 @@ template <int T>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
-  static constexpr int BK = 16;                        // input channels per stage (one MMA K step)
+  static constexpr int BK = TC_BK;                     // input channels per stage (one MMA K step)
   // output channels per tile and accumulator buffers: T * BO * NACC <= 512 columns
-  static constexpr int BO = T == 1 ? 256 : T == 2 ? 128 : T == 4 ? 128 : 32;
+  static constexpr int BO = tc_bo(T);
   static constexpr int NACC = (T * BO * 2 <= 512) ? 2 : 1;
   static constexpr int ACC_COLS = T * BO;
   static constexpr int TMEM_COLS = NACC * ACC_COLS <= 256 ? 256 : 512;
@@ -98,6 +99,7 @@ struct Params {
   int n_otiles;
   int64_t n_tiles;
   const void* in;
+  const void* wtiles;  // tensor-core weight tiles (rows O, K) of this pass
   const float* bias;   // nullptr: none
   int* err;
   uint32_t wait_limit;
@@ -168,8 +170,8 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
 
 template <int T, typename E>
 __global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
-tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_in,
-                const __grid_constant__ CUtensorMap map_out, Params p) {
+tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
+                Params p) {
   using C = Cfg<T>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
@@ -211,7 +213,6 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&map_w);
     prefetch_tensormap(&map_in);
     prefetch_tensormap(&map_out);
   }
@@ -316,7 +317,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
         const int m0 = (tile / p.n_otiles) * C::BM;
-        const int o0 = (tile % p.n_otiles) * C::BO;
+        const int ot = tile % p.n_otiles;
+        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)ot * nk * C::B_BYTES;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
           if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag) ||
@@ -324,11 +326,9 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant
             ok = false;
             break;
           }
+          // the stage's Q weight planes are one contiguous, pre-swizzled tile
           mbar_arrive_expect_tx(&stage_full[s], C::B_BYTES);
-          uint8_t* bdst = b_buf + s * C::B_BYTES;
-#pragma unroll
-          for (int q = 0; q < C::Q; ++q)
-            tma_load_3d(bdst + q * C::B_PLANE_BYTES, &map_w, kb * C::BK, o0, q, &stage_full[s]);
+          bulk_load(b_buf + s * C::B_BYTES, wt + (int64_t)kb * C::B_BYTES, C::B_BYTES, &stage_full[s]);
           ++n_b;
           mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
           tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
@@ -518,18 +518,6 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   const int O = (int)(backward ? h.Cp : h.Dp);
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap map_w;
-  {
-    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)O, (cuuint64_t)C::Q};
-    cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)K * O * 2};
-    cuuint32_t box[3] = {(cuuint32_t)C::BK, (cuuint32_t)C::BO, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    void* wptr = backward ? h.wt_bwd : h.wt_fwd;
-    if (enc(&map_w, dt, 3, wptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
   CUtensorMap map_in;      // raw input tiles: 16 channels x T elements x 128 tokens
   {
     cuuint64_t dims[2] = {(cuuint64_t)K * T, (cuuint64_t)N};
@@ -559,6 +547,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.n_otiles = (O + C::BO - 1) / C::BO;
   p.n_tiles = ((N + C::BM - 1) / C::BM) * p.n_otiles;
   p.in = in;
+  p.wtiles = backward ? h.wt_bwd : h.wt_fwd;
   p.bias = backward ? nullptr : h.bias;
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
@@ -573,7 +562,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_w, map_in, map_out, p);
+  tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_out, p);
   count_launches(1);
   return cudaGetLastError();
 }
