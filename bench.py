@@ -202,14 +202,14 @@ def kernel_src_sha(name: str) -> str:
 
 
 def profiled_traffic(kernel_key: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    """DRAM bytes per launch from a committed ncu summary, if every source it
+    was taken on is unchanged; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         e = d[kernel_key]
-        if e.get("src_sha") == kernel_src_sha(e["src"]):
+        if [kernel_src_sha(s) for s in e["srcs"]] == list(e["src_sha"]):
             return float(e["bytes_per_launch"])
     except Exception:
         pass
