@@ -116,7 +116,10 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
             cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
             cudaMalloc(&h.err, sizeof(int)) == cudaSuccess;
   if (ok && dtype != EQLIN_F32) {
-    const size_t nf = (size_t)eqlin::wtile_elems(T, Dp, Cp), nb = (size_t)eqlin::wtile_elems(T, Cp, Dp);
+    h.bo_fwd = eqlin::tc_pick_bo(T, Dp);
+    h.bo_bwd = eqlin::tc_pick_bo(T, Cp);
+    const size_t nf = (size_t)eqlin::wtile_elems(T, h.bo_fwd, Dp, Cp);
+    const size_t nb = (size_t)eqlin::wtile_elems(T, h.bo_bwd, Cp, Dp);
     ok = cudaMalloc(&h.wt_fwd, nf * e) == cudaSuccess && cudaMalloc(&h.wt_bwd, nb * e) == cudaSuccess;
     // padding rows and K columns of the tiles stay zero
     if (ok) ok = cudaMemset(h.wt_fwd, 0, nf * e) == cudaSuccess && cudaMemset(h.wt_bwd, 0, nb * e) == cudaSuccess;

@@ -133,14 +133,34 @@ template <int T> struct Group {
 // plane, stored in the exact 32-byte-swizzled image the MMA reads from shared
 // memory, so that one contiguous bulk copy fetches a stage.  For K-major rows
 // of 32 bytes, 16-byte chunk j of row r sits at chunk j ^ ((r >> 2) & 1).
+//
+// BO, the output channels of a tile, is chosen per pass from the pass's
+// output width O.  The accumulator of a tile takes T * BO TMEM columns (of
+// 512), a complex frequency's block product is an N = 2 * BO MMA (N <= 256),
+// and the epilogue stores 64 / T channels per chunk in an even number of
+// chunks.  For T = 4 the candidates are 128, 96, 64 and 32: the one that pads
+// O least, the wider on a tie (fewer output tiles, so fewer repeats of the
+// input transform).  Other T use one width.
 constexpr int TC_BK = 16;
-__host__ __device__ constexpr int tc_bo(int T) { return T == 1 ? 256 : T == 2 ? 128 : T == 4 ? 128 : 32; }
 __host__ __device__ constexpr int tc_planes(int T) {
   return (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
 }
-// Element index of (row, k, plane q) in a tiled weight buffer with n_kb K stages.
-__host__ __device__ inline int64_t wtile_index(int T, int64_t n_kb, int64_t row, int64_t k, int q) {
-  const int bo = tc_bo(T), Q = tc_planes(T);
+inline int tc_pick_bo(int T, int64_t O) {
+  if (T == 1) return 256;
+  if (T == 2) return 128;
+  if (T == 8) return 32;
+  int best = 128;
+  int64_t best_pad = (O + 127) / 128 * 128;
+  for (int bo : {96, 64, 32}) {
+    const int64_t pad = (O + bo - 1) / bo * bo;
+    if (pad < best_pad) { best = bo; best_pad = pad; }
+  }
+  return best;
+}
+// Element index of (row, k, plane q) in a tiled weight buffer with tile width
+// bo and n_kb K stages.
+__host__ __device__ inline int64_t wtile_index(int T, int bo, int64_t n_kb, int64_t row, int64_t k, int q) {
+  const int Q = tc_planes(T);
   const int64_t ot = row / bo, kb = k / TC_BK;
   const int r = (int)(row % bo), kk = (int)(k % TC_BK);
   const int64_t tile = (ot * n_kb + kb) * Q + q;
@@ -148,8 +168,7 @@ __host__ __device__ inline int64_t wtile_index(int T, int64_t n_kb, int64_t row,
   return byte / 2;
 }
 // Elements of a tiled buffer for `rows` output rows and K = `kdim`.
-__host__ __device__ inline int64_t wtile_elems(int T, int64_t rows, int64_t kdim) {
-  const int bo = tc_bo(T);
+__host__ __device__ inline int64_t wtile_elems(int T, int bo, int64_t rows, int64_t kdim) {
   return ((rows + bo - 1) / bo) * ((kdim + TC_BK - 1) / TC_BK) * tc_planes(T) * bo * TC_BK;
 }
 
@@ -171,6 +190,7 @@ struct Handle {
   // [-Im;Re] are contiguous windows of a stage).
   void* wt_fwd = nullptr;
   void* wt_bwd = nullptr;
+  int bo_fwd = 0, bo_bwd = 0;     // tile widths (output channels) of the two layouts
   bool need_simt_fwd = true;      // FP32 planes needed (SIMT serves forward / dx)
   bool need_simt_bwd = true;
   float* bias = nullptr;          // [Dp] float32 (zeros when no bias)

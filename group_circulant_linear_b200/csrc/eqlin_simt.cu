@@ -34,7 +34,7 @@ template <int T, typename E>
 __global__ void __launch_bounds__(pt::TILE * pt::ROWS)
 pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __restrict__ wf_fwd,
                     float* __restrict__ wf_bwd, E* __restrict__ wt_fwd, E* __restrict__ wt_bwd,
-                    float* __restrict__ bias, int Cp, int Dp) {
+                    float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b) {
   using G = Group<T>;
   using namespace pt;
   constexpr int Q = G::nreal + 3 * G::ncomplex;
@@ -68,14 +68,14 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
       const float sr = 1.f / T, sc = 2.f / T;
       const int64_t nkb = (Cp + TC_BK - 1) / TC_BK;
 #pragma unroll
-      for (int f = 0; f < G::nreal; ++f) wt_fwd[wtile_index(T, nkb, d, c, f)] = Elem<E>::from_f(P[f] * sr);
+      for (int f = 0; f < G::nreal; ++f) wt_fwd[wtile_index(T, bo_f, nkb, d, c, f)] = Elem<E>::from_f(P[f] * sr);
 #pragma unroll
       for (int k = 1; k <= G::ncomplex; ++k) {
         const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
         const int q = G::nreal + 3 * (k - 1);
-        wt_fwd[wtile_index(T, nkb, d, c, q + 0)] = Elem<E>::from_f(-im);
-        wt_fwd[wtile_index(T, nkb, d, c, q + 1)] = Elem<E>::from_f(re);
-        wt_fwd[wtile_index(T, nkb, d, c, q + 2)] = Elem<E>::from_f(im);
+        wt_fwd[wtile_index(T, bo_f, nkb, d, c, q + 0)] = Elem<E>::from_f(-im);
+        wt_fwd[wtile_index(T, bo_f, nkb, d, c, q + 1)] = Elem<E>::from_f(re);
+        wt_fwd[wtile_index(T, bo_f, nkb, d, c, q + 2)] = Elem<E>::from_f(im);
       }
     }
   }
@@ -97,14 +97,14 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
       const float sr = 1.f / T, sc = 2.f / T;
       const int64_t nkb = (Dp + TC_BK - 1) / TC_BK;
 #pragma unroll
-      for (int f = 0; f < G::nreal; ++f) wt_bwd[wtile_index(T, nkb, c, d, f)] = Elem<E>::from_f(P[f] * sr);
+      for (int f = 0; f < G::nreal; ++f) wt_bwd[wtile_index(T, bo_b, nkb, c, d, f)] = Elem<E>::from_f(P[f] * sr);
 #pragma unroll
       for (int k = 1; k <= G::ncomplex; ++k) {
         const float re = P[G::nreal + 2 * (k - 1)] * sc, im = P[G::nreal + 2 * (k - 1) + 1] * sc;
         const int q = G::nreal + 3 * (k - 1);
-        wt_bwd[wtile_index(T, nkb, c, d, q + 0)] = Elem<E>::from_f(im);
-        wt_bwd[wtile_index(T, nkb, c, d, q + 1)] = Elem<E>::from_f(re);
-        wt_bwd[wtile_index(T, nkb, c, d, q + 2)] = Elem<E>::from_f(-im);
+        wt_bwd[wtile_index(T, bo_b, nkb, c, d, q + 0)] = Elem<E>::from_f(im);
+        wt_bwd[wtile_index(T, bo_b, nkb, c, d, q + 1)] = Elem<E>::from_f(re);
+        wt_bwd[wtile_index(T, bo_b, nkb, c, d, q + 2)] = Elem<E>::from_f(-im);
       }
     }
   }
@@ -117,7 +117,7 @@ static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b,
   dim3 block(pt::TILE, pt::ROWS);
   pretransform_kernel<T, E><<<grid, block, 0, st>>>(
       (const E*)W, (const E*)b, h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr,
-      (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp);
+      (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
   count_launches(1);
   return cudaGetLastError();
 }

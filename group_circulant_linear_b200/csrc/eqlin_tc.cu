@@ -5,26 +5,33 @@
 // channels (all T group positions).  Per tile and per K stage of 16 input
 // channels:
 //
-//   producer warp    (8)    TMA: the raw input tile of the stage [128 tokens x
-//                    16*T elements]; one bulk copy of the stage's Fourier
-//                    weight planes (stored pre-swizzled per stage); L2
-//                    prefetches of raw tiles several stages ahead
-//   transform warps  (0-7)  one thread per (input channel, 8 tokens): read the
+//   raw producer     (8)    TMA: the raw input tile of the stage [128 tokens x
+//                    16*T elements] into the raw ring; L2 prefetches of raw
+//                    tiles several stages ahead
+//   weight producer  (9)    one bulk copy of the stage's Fourier weight planes
+//                    (stored pre-swizzled per stage) into the operand ring
+//   transform warps  (0-7)  two groups of four warps on alternate stages; one
+//                    thread per (input channel, 16 tokens): read the
 //                    channel's T group values of its tokens from the raw tile,
 //                    take the group DFT (adds/subtracts on packed token pairs
 //                    for T <= 4, FP32 with the sqrt(2)/2 twiddles for T = 8)
 //                    and write the T frequency planes as token-contiguous
 //                    (MN-major, 128B-swizzled) MMA operands; then a
 //                    generic->async proxy fence
-//   MMA warp         (9)    one thread issues tcgen05.mma into TMEM: for each
+//   MMA warp         (10)   one thread issues tcgen05.mma into TMEM: for each
 //                    real frequency one M=128, N=BO product; for each complex
 //                    frequency two M=128, N=2*BO products that accumulate
 //                    [Re Y | Im Y] = Re X [Re W ; Im W] + Im X [-Im W ; Re W]
 //                    -- R(T) real GEMMs, six for p4
-//   epilogue warps   (10-17) tcgen05.ld of the frequency planes, inverse DFT
+//   epilogue warps   (11-18) tcgen05.ld of the frequency planes, inverse DFT
 //                    (the weight planes carry its 1/T and 2/T scales, so this
 //                    is additions only), bias, cast into a 128B-swizzled
 //                    staging tile, TMA store of 64 output elements x 128 rows
+//
+// The two rings are independent: a raw slot is refilled as soon as the
+// transform warps have read it, and an operand slot (the stage's A planes and
+// weight planes) once the MMAs that read it have completed; so loads run
+// ahead of the tensor core by the whole raw ring.
 //
 // ("Flash EQ-Linear", technical summary, sections "Abordagem Algoritmica",
 // "Especializacao para o Grupo de Rotacao p4" and "Implementacao": fused data
@@ -48,13 +55,14 @@ namespace tc {
 
 using namespace ptx;
 
-template <int T>
+template <int T, int BO_>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
   static constexpr int BK = TC_BK;                     // input channels per stage (one MMA K step)
   // output channels per tile and accumulator buffers: T * BO * NACC <= 512 columns
-  static constexpr int BO = tc_bo(T);
+  static constexpr int BO = BO_;
+  static_assert(T * BO <= 512 && (Group<T>::ncomplex == 0 || 2 * BO <= 256), "TMEM columns, MMA N");
   static constexpr int NACC = (T * BO * 2 <= 512) ? 2 : 1;
   static constexpr int ACC_COLS = T * BO;
   static constexpr int TMEM_COLS = NACC * ACC_COLS <= 256 ? 256 : 512;
@@ -71,21 +79,34 @@ struct Cfg {
   static constexpr int B_ROWB = BK * 2;
   static constexpr int B_PLANE_BYTES = BO * B_ROWB;
   static constexpr int B_BYTES = Q * B_PLANE_BYTES;
-  static constexpr int STAGE_BYTES = RAW_BYTES + A_BYTES + B_BYTES;
-  // output staging for the TMA stores: per epilogue half one [128 rows x 128 B] tile
+  // output staging for the TMA stores: per epilogue half two [128 rows x 128 B] tiles
   static constexpr int OUT_EL = 64;                    // output elements per row per store
-  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2; // two per epilogue half (double buffer)
-  static constexpr int STAGES_FIT = (220 * 1024 - 4 * OUT_TILE_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static_assert(STAGES >= 2, "two stages must fit");
-  static constexpr int NBAR = 4 * STAGES + 2 * NACC + 1;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * OUT_TILE_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2;
+  static constexpr int STAGING = 4 * OUT_TILE_BYTES;
+  // ring depths: operand slots (the A planes of a stage and its weight
+  // planes share one slot and one pair of barriers, so the MMA thread waits
+  // and commits once per stage): three where three raw slots still fit (the
+  // transform writes stage k + 2 while the MMAs of k and k + 1 are in
+  // flight), else two; the rest of the budget for raw slots (memory latency)
+  static constexpr int BUDGET = 224 * 1024;
+  static constexpr int AB_ST = (BUDGET - STAGING - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 3 ? 3 : 2;
+  static constexpr int RAW_FIT = (BUDGET - STAGING - AB_ST * (A_BYTES + B_BYTES)) / RAW_BYTES;
+  static constexpr int RAW_ST = RAW_FIT > 8 ? 8 : RAW_FIT;
+  static_assert(RAW_ST >= 2 && AB_ST >= 2, "two slots per ring (the transform groups take alternate stages)");
+  static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + 1;
+  // per epilogue half, the bias of the tile's BO channels (FP32)
+  static constexpr int BIAS_BYTES = 2 * BO * 4;
+  static constexpr int SMEM_BYTES = RAW_ST * RAW_BYTES + AB_ST * (A_BYTES + B_BYTES) + STAGING +
+                                    BIAS_BYTES + NBAR * 8 + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
   static constexpr int CH = OUT_EL / T;                // output channels per store chunk
   static constexpr int NCHUNK = BO / CH;               // store chunks per tile (even)
   static_assert(NCHUNK % 2 == 0, "chunks alternate between the two epilogue halves");
   // roles
-  static constexpr int TR_WARPS = 8;                   // transform: 8 tokens x 16 channels per warp-half
-  static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1, EPI0 = TR_WARPS + 2;
+  static constexpr int TR_WARPS = 8;                   // transform: two groups of four warps
+  static constexpr int GRP_WARPS = TR_WARPS / 2;       // warps per stage (16 tokens x 16 channels per warp-half)
+  static constexpr int RAW_PRODUCER = TR_WARPS, B_PRODUCER = TR_WARPS + 1;
+  static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = TR_WARPS + 3;
   static constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
@@ -146,13 +167,20 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) 
   atomicCAS(err, DEV_OK, DEV_TIMEOUT);
 }
 
+// Eight floats to eight 16-bit values (round to nearest even), two per conversion.
+template <typename E>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (std::is_same<E, __half>::value) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
 template <typename E>
 __device__ __forceinline__ uint4 pack8(const float* f) {
-  uint4 u;
-  E* e = reinterpret_cast<E*>(&u);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) e[i] = Elem<E>::from_f(f[i]);
-  return u;
+  return make_uint4(pack2<E>(f[0], f[1]), pack2<E>(f[2], f[3]), pack2<E>(f[4], f[5]), pack2<E>(f[6], f[7]));
 }
 
 // MN-major, 128B-swizzled operand descriptor (A side): leading byte offset =
@@ -168,26 +196,28 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
   return d;
 }
 
-template <int T, typename E>
-__global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
+template <int T, int BO, typename E>
+__global__ void __launch_bounds__(Cfg<T, BO>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
                 Params p) {
-  using C = Cfg<T>;
+  using C = Cfg<T, BO>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* a_buf = smem;
-  uint8_t* b_buf = a_buf + C::STAGES * C::A_BYTES;
-  uint8_t* raw_buf = b_buf + C::STAGES * C::B_BYTES;
-  uint8_t* o_buf = raw_buf + C::STAGES * C::RAW_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(o_buf + 4 * C::OUT_TILE_BYTES);
-  // stage_full: the 8 transform warps' A planes and the producer's B planes (tx)
-  uint64_t* stage_full = bars;
-  uint64_t* ab_empty = stage_full + C::STAGES;
-  uint64_t* raw_full = ab_empty + C::STAGES;
-  uint64_t* raw_empty = raw_full + C::STAGES;
-  uint64_t* acc_full = raw_empty + C::STAGES;
+  uint8_t* a_buf = smem;                                   // [AB_ST][T planes]
+  uint8_t* b_buf = a_buf + C::AB_ST * C::A_BYTES;          // [AB_ST][Q planes]
+  uint8_t* raw_buf = b_buf + C::AB_ST * C::B_BYTES;        // [RAW_ST][raw tile]
+  uint8_t* o_buf = raw_buf + C::RAW_ST * C::RAW_BYTES;     // 4 staging tiles
+  float* s_bias = reinterpret_cast<float*>(o_buf + C::STAGING);      // [2][BO]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_buf + C::STAGING + C::BIAS_BYTES);
+  uint64_t* raw_full = bars;                   // TMA bytes landed
+  uint64_t* raw_empty = raw_full + C::RAW_ST;  // the 8 transform warps have read the slot
+  // ab_full: the 8 transform warps have written the A planes and the weight
+  // planes' bulk-copy bytes have landed; ab_empty: MMA commit
+  uint64_t* ab_full = raw_empty + C::RAW_ST;
+  uint64_t* ab_empty = ab_full + C::AB_ST;
+  uint64_t* acc_full = ab_empty + C::AB_ST;
   uint64_t* acc_empty = acc_full + C::NACC;
   uint64_t* drain_bar = acc_empty + C::NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -200,11 +230,13 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   const int64_t my_tiles = p.n_tiles > blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&stage_full[i], C::TR_WARPS + 1);
-      mbar_init(&ab_empty[i], 1);
+    for (int i = 0; i < C::RAW_ST; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], C::TR_WARPS);
+      mbar_init(&raw_empty[i], C::GRP_WARPS);
+    }
+    for (int i = 0; i < C::AB_ST; ++i) {
+      mbar_init(&ab_full[i], C::GRP_WARPS + 1);
+      mbar_init(&ab_empty[i], 1);
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -227,82 +259,110 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
 
   if (warp < C::TR_WARPS) {
     // ----------------------------------------------------- transform warps
-    // thread: channel c of the stage (16 per stage), 8 consecutive tokens
+    // Two groups of four warps take alternate stages, so two stages are in
+    // flight.  Thread: channel c of the stage (16 per stage) and 16
+    // consecutive tokens (two blocks of 8).
+    const int grp = warp / C::GRP_WARPS;
     const int c = lane & 15;
-    const int m = warp * 16 + 8 * (lane >> 4);       // first of its 8 tokens in the tile
-    // MN-major placement of the 8 tokens for K row c of a plane
-    const uint32_t a_off = (uint32_t)((m >> 6) * C::A_LBO + (c >> 3) * C::A_SBO + (c & 7) * 128 +
-                                      ((((m & 63) >> 3) ^ (c & 7)) << 4));
+    const int m = (warp % C::GRP_WARPS) * 32 + 16 * (lane >> 4);   // first of its 16 tokens
+    // MN-major placement of 8 tokens (block b) for K row c of a plane
+    uint32_t a_off[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int mb = m + 8 * b;
+      a_off[b] = (uint32_t)((mb >> 6) * C::A_LBO + (c >> 3) * C::A_SBO + (c & 7) * 128 +
+                            ((((mb & 63) >> 3) ^ (c & 7)) << 4));
+    }
     const uint32_t raw_off = (uint32_t)(m * C::RAW_ROWB + c * T * 2);
-    int s = 0;
-    uint32_t ph = 0;
+    // ring positions of stage `grp`, then advanced by two stages per step
+    int rs = grp % C::RAW_ST, as = grp % C::AB_ST;
+    uint32_t rph = 0, aph = 0;
     bool ok = true;
-    for (int64_t it = 0; it < my_tiles * nk; ++it) {
-      // raw_full also means A slot s is free: the producer loads raw[s] only
-      // after the MMAs that read A[s] have completed
-      if (!wwait_all(&raw_full[s], ph, limit, abort_flag)) { ok = false; break; }
-      const uint8_t* raw = raw_buf + s * C::RAW_BYTES + raw_off;
-      uint32_t wv[8][C::W];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint8_t* src = raw + j * C::RAW_ROWB;
-        if constexpr (C::W == 4) {
-          const uint4 u = *reinterpret_cast<const uint4*>(src);
-          wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
-        } else if constexpr (C::W == 2) {
-          const uint2 u = *reinterpret_cast<const uint2*>(src);
-          wv[j][0] = u.x; wv[j][1] = u.y;
-        } else if constexpr (T == 2) {
-          wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
-        } else {
-          wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&raw_empty[s]);       // the raw slot may be refilled
-      uint32_t Pw[T][4];
+    for (int64_t it = grp; it < my_tiles * nk; it += 2) {
+      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag)) { ok = false; break; }
+      const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_off;
+      uint32_t Pw[2][T][4];
       if constexpr (T <= 4) {
+        // all 16 tokens' words first, so the raw slot is released early
+        uint32_t wv[16][C::W];
 #pragma unroll
-        for (int pr = 0; pr < 4; ++pr) {
-          uint32_t P[T];
-          packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
-#pragma unroll
-          for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
-        }
-      } else {
-        // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
-#pragma unroll
-        for (int pr = 0; pr < 4; ++pr) {
-          float Pa[T], Pb[T], va[T], vb[T];
-          const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
-          const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
-#pragma unroll
-          for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
-          G::dft(va, Pa);
-          G::dft(vb, Pb);
-#pragma unroll
-          for (int q = 0; q < T; ++q) {
-            E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
-            Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
+        for (int j = 0; j < 16; ++j) {
+          const uint8_t* src = raw + j * C::RAW_ROWB;
+          if constexpr (C::W == 2) {
+            const uint2 u = *reinterpret_cast<const uint2*>(src);
+            wv[j][0] = u.x; wv[j][1] = u.y;
+          } else if constexpr (T == 2) {
+            wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
+          } else {
+            wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
           }
         }
-      }
-      uint8_t* a_st = a_buf + s * C::A_BYTES + a_off;
+        // the raw slot may be refilled by TMA (async proxy) once these generic
+        // reads are ordered before it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
 #pragma unroll
-      for (int q = 0; q < T; ++q)
-        *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES) = make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) {
+            uint32_t P[T];
+            packed::dft_pair<T, E>(wv[8 * b + 2 * pr], wv[8 * b + 2 * pr + 1], P);
+#pragma unroll
+            for (int q = 0; q < T; ++q) Pw[b][q][pr] = P[q];
+          }
+      } else {
+        // T = 8: one block of 8 tokens at a time (registers), FP32 butterflies
+        // with the sqrt(2)/2 twiddles, one rounding per value
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          uint32_t wv[8][C::W];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 u = *reinterpret_cast<const uint4*>(raw + (8 * b + j) * C::RAW_ROWB);
+            wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
+          }
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) {
+            float Pa[T], Pb[T], va[T], vb[T];
+            const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
+            const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
+#pragma unroll
+            for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
+            G::dft(va, Pa);
+            G::dft(vb, Pb);
+#pragma unroll
+            for (int q = 0; q < T; ++q) Pw[b][q][pr] = pack2<E>(Pa[q], Pb[q]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
+      }
+      rs += 2;
+      if (rs >= C::RAW_ST) { rs -= C::RAW_ST; rph ^= 1; }
+      // the operand slot must have been consumed by the MMAs issued from it
+      if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane)) { ok = false; break; }
+      uint8_t* a_st = a_buf + as * C::A_BYTES;
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int q = 0; q < T; ++q)
+          *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + a_off[b]) =
+              make_uint4(Pw[b][q][0], Pw[b][q][1], Pw[b][q][2], Pw[b][q][3]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&stage_full[s]);
-      if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      if (lane == 0) mbar_arrive(&ab_full[as]);
+      as += 2;
+      if (as >= C::AB_ST) { as -= C::AB_ST; aph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
-  } else if (warp == C::PRODUCER) {
-    // ------------------------------------------------------------ producer
+  } else if (warp == C::RAW_PRODUCER) {
+    // -------------------------------------------------------- raw producer
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      int64_t n_b = 0, n_raw = 0;
+      int64_t n_raw = 0;
       bool ok = true;
       // L2 prefetch of the raw input tiles PF_STAGES stages ahead of their loads
       int64_t pf_ti = 0;
@@ -317,78 +377,93 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
         const int m0 = (tile / p.n_otiles) * C::BM;
-        const int ot = tile % p.n_otiles;
-        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)ot * nk * C::B_BYTES;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
-          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag) ||
-              !bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) {
-            ok = false;
-            break;
-          }
-          // the stage's Q weight planes are one contiguous, pre-swizzled tile
-          mbar_arrive_expect_tx(&stage_full[s], C::B_BYTES);
-          bulk_load(b_buf + s * C::B_BYTES, wt + (int64_t)kb * C::B_BYTES, C::B_BYTES, &stage_full[s]);
-          ++n_b;
+          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
           tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
           ++n_raw;
-          if (++s == C::STAGES) { s = 0; ph ^= 1; }
+          if (++s == C::RAW_ST) { s = 0; ph ^= 1; }
         }
       }
       if (!ok) raise_abort(abort_flag, p.err);
       // every issued TMA copy must land before the CTA exits (a no-op on the
-      // normal path, where the MMA thread already waited for them)
-      for (int i = 0; i < C::STAGES; ++i) {
-        if (n_b > i) mbar_wait(&stage_full[i], (uint32_t)(((n_b - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
-        if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
+      // normal path, where the transform warps already waited for them)
+      for (int i = 0; i < C::RAW_ST; ++i)
+        if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::RAW_ST) & 1), kDefaultWaitLimit);
+    }
+  } else if (warp == C::B_PRODUCER) {
+    // ----------------------------------------------------- weight producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t n_b = 0;
+      bool ok = true;
+      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
+        const int tile = (int)(blockIdx.x + ti * gridDim.x);
+        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)(tile % p.n_otiles) * nk * C::B_BYTES;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+          // the stage's Q weight planes are one contiguous, pre-swizzled tile
+          mbar_arrive_expect_tx(&ab_full[s], C::B_BYTES);
+          bulk_load(b_buf + s * C::B_BYTES, wt + (int64_t)kb * C::B_BYTES, C::B_BYTES, &ab_full[s]);
+          ++n_b;
+          if (++s == C::AB_ST) { s = 0; ph ^= 1; }
+        }
       }
+      if (!ok) raise_abort(abort_flag, p.err);
+      // the weight copies must land before the CTA exits.  A slot's phase
+      // completes with its bytes and the transform warps' arrivals; if an
+      // aborted run never makes those, the wait gives up after its wall-time
+      // cap, long after any copy has landed.
+      for (int i = 0; i < C::AB_ST; ++i)
+        if (n_b > i) mbar_wait(&ab_full[i], (uint32_t)(((n_b - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
   } else if (warp == C::MMA_WARP) {
     // -------------------------------------------------------------- MMA
     if (lane == 0) {
       int s = 0, ab = 0;
-      uint32_t ph = 0, aph = 0;
+      uint32_t ph = 0, acph = 0;
       bool ok = true;
       // A is MN-major (bit 15), B K-major
       const uint32_t id_real = idesc_f16(p.ab_fmt, C::BO) | (1u << 15);
       const uint32_t id_cplx = idesc_f16(p.ab_fmt, 2 * C::BO) | (1u << 15);
+      // Descriptors of slot 0; a byte offset d inside shared memory (< 256 KB)
+      // moves the 14-bit start-address field by d >> 4 without a carry out.
+      const uint64_t a_desc0 = smem_desc_mn(smem_u32(a_buf), C::A_LBO, C::A_SBO);
+      const uint64_t b_desc0 = smem_desc(smem_u32(b_buf), C::B_ROWB);
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        if (!bwait(&acc_empty[ab], aph ^ 1, limit, abort_flag)) { ok = false; break; }
+        if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&stage_full[s], ph, limit, abort_flag)) { ok = false; break; }
+          if (!bwait(&ab_full[s], ph, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
-          const uint32_t b_st = smem_u32(b_buf + s * C::B_BYTES);
-          {
-            const uint32_t a_k = a_st;
-            const uint32_t b_k = b_st;
-            const uint32_t first = kb > 0 ? 1u : 0u;
+          const uint64_t a_d = a_desc0 + (uint64_t)((s * C::A_BYTES) >> 4);
+          const uint64_t b_d = b_desc0 + (uint64_t)((s * C::B_BYTES) >> 4);
+          const uint32_t first = kb > 0 ? 1u : 0u;
 #pragma unroll
-            for (int f = 0; f < G::nreal; ++f)
-              mma_f16_ss(acc + f * C::BO, smem_desc_mn(a_k + f * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
-                         smem_desc(b_k + f * C::B_PLANE_BYTES, C::B_ROWB), id_real, first);
+          for (int f = 0; f < G::nreal; ++f)
+            mma_f16_ss(acc + f * C::BO, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + ((f * C::B_PLANE_BYTES) >> 4),
+                       id_real, first);
 #pragma unroll
-            for (int k = 1; k <= G::ncomplex; ++k) {
-              const int pr = G::nreal + 2 * (k - 1);
-              const int q = G::nreal + 3 * (k - 1);
-              const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO;
-              // [Re Y | Im Y] += Re X [Re W ; Im W]
-              mma_f16_ss(col, smem_desc_mn(a_k + pr * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
-                         smem_desc(b_k + (q + 1) * C::B_PLANE_BYTES, C::B_ROWB), id_cplx, first);
-              // [Re Y | Im Y] += Im X [-Im W ; Re W]
-              mma_f16_ss(col, smem_desc_mn(a_k + (pr + 1) * C::A_PLANE_BYTES, C::A_LBO, C::A_SBO),
-                         smem_desc(b_k + q * C::B_PLANE_BYTES, C::B_ROWB), id_cplx, 1u);
-            }
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const int pr = G::nreal + 2 * (k - 1);
+            const int q = G::nreal + 3 * (k - 1);
+            const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO;
+            // [Re Y | Im Y] += Re X [Re W ; Im W]
+            mma_f16_ss(col, a_d + ((pr * C::A_PLANE_BYTES) >> 4), b_d + (((q + 1) * C::B_PLANE_BYTES) >> 4),
+                       id_cplx, first);
+            // [Re Y | Im Y] += Im X [-Im W ; Re W]
+            mma_f16_ss(col, a_d + (((pr + 1) * C::A_PLANE_BYTES) >> 4), b_d + ((q * C::B_PLANE_BYTES) >> 4),
+                       id_cplx, 1u);
           }
           mma_commit(&ab_empty[s]);
-          if (++s == C::STAGES) { s = 0; ph ^= 1; }
+          if (++s == C::AB_ST) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
         mma_commit(&acc_full[ab]);
-        if (++ab == C::NACC) { ab = 0; aph ^= 1; }
+        if (++ab == C::NACC) { ab = 0; acph ^= 1; }
       }
       if (!ok) raise_abort(abort_flag, p.err);
       mma_commit(drain_bar);              // arrives once every issued MMA has completed
@@ -412,6 +487,13 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     bool ok = true;
     for (int64_t ti = 0; ti < my_tiles; ++ti) {
       const int tile = (int)(blockIdx.x + ti * gridDim.x);
+      // this half's copy of the tile's bias, loaded while the MMAs run (the
+      // half's previous tile has finished reading it)
+      {
+        const int ob = (tile % p.n_otiles) * C::BO;
+        for (int i = (e & 3) * 32 + lane; i < C::BO; i += 128)
+          s_bias[half * C::BO + i] = (p.bias && ob + i < p.O) ? __ldg(p.bias + ob + i) : 0.f;
+      }
       // the four warps of a half share named barriers, so they decide together
       const bool got = named_bar_and(1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane));
       if (!got) { ok = false; break; }
@@ -426,34 +508,36 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         // the TMA store issued from this staging tile two chunks ago must have read it
         if (issuer) bulk_wait_read<1>();
         named_bar_sync(1 + half, 128);
+        // the chunk's T planes x CH channels (64 values) in one batch of TMEM loads
+        uint32_t rg[T][C::CH];
+#pragma unroll
+        for (int q = 0; q < T; ++q) {
+          const int k = q < G::nreal ? 0 : 1 + (q - G::nreal) / 2;
+          const uint32_t col = acc + ci * C::CH +
+                               (q < G::nreal ? q * C::BO
+                                             : G::nreal * C::BO + (k - 1) * 2 * C::BO + ((q - G::nreal) & 1) * C::BO);
+          if constexpr (C::CH == 8) {
+            tmem_ld_32x32b_x8(col, *reinterpret_cast<uint32_t(*)[8]>(&rg[q][0]));
+          } else {
+#pragma unroll
+            for (int h = 0; h < C::CH / 16; ++h) tmem_ld_32x32b_x16(col + 16 * h, &rg[q][16 * h]);
+          }
+        }
+        tmem_wait_ld();
+        if (ci + 2 >= C::NCHUNK) {
+          // last TMEM read of this tile by this thread: release the accumulator
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+        }
 #pragma unroll
         for (int sub = 0; sub < C::CH / 8; ++sub) {
           const int oc = ci * C::CH + sub * 8;       // channel offset within the tile
-          uint32_t rg[T][8];
-#pragma unroll
-          for (int f = 0; f < G::nreal; ++f) tmem_ld_32x32b_x8(acc + f * C::BO + oc, rg[f]);
-#pragma unroll
-          for (int k = 1; k <= G::ncomplex; ++k) {
-            const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO + oc;
-            tmem_ld_32x32b_x8(col, rg[G::nreal + 2 * (k - 1)]);
-            tmem_ld_32x32b_x8(col + C::BO, rg[G::nreal + 2 * (k - 1) + 1]);
-          }
-          tmem_wait_ld();
-          if (ci + 2 >= C::NCHUNK && sub == C::CH / 8 - 1) {
-            // last TMEM read of this tile by this thread: release the accumulator
-            tc_fence_before();
-            mbar_arrive(&acc_empty[ab]);
-          }
-          const int o = o0 + oc;
           float bo8[8];
-          if (p.bias && o + 8 <= p.O) {
-            const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + o));
-            const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + o) + 1);
+          {
+            const float4 b0 = *reinterpret_cast<const float4*>(s_bias + half * C::BO + oc);
+            const float4 b1 = *reinterpret_cast<const float4*>(s_bias + half * C::BO + oc + 4);
             bo8[0] = b0.x; bo8[1] = b0.y; bo8[2] = b0.z; bo8[3] = b0.w;
             bo8[4] = b1.x; bo8[5] = b1.y; bo8[6] = b1.z; bo8[7] = b1.w;
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) bo8[c] = (p.bias && o + c < p.O) ? __ldg(p.bias + o + c) : 0.f;
           }
           // 8 channels x T outputs = T 16-byte chunks of this row's 128 bytes;
           // chunk v holds the outputs of channels v*8/T .. (v+1)*8/T - 1
@@ -463,11 +547,10 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
 #pragma unroll
             for (int cc = 0; cc < 8 / T; ++cc) {
               const int c = v * (8 / T) + cc;
-              const float bo = bo8[c];
               float Pc[T];
 #pragma unroll
-              for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][c]);
-              G::idft_scaled(Pc, bo, vals + cc * T);
+              for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][sub * 8 + c]);
+              G::idft_scaled(Pc, bo8[c], vals + cc * T);
             }
             const int j = sub * T + v;
             *reinterpret_cast<uint4*>(my_row + ((j ^ (r & 7)) << 4)) = pack8<E>(vals);
@@ -508,10 +591,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int T, typename E>
+template <int T, int BO, typename E>
 static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, int64_t N,
                             cudaStream_t st) {
-  using C = Cfg<T>;
+  using C = Cfg<T, BO>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int K = (int)(backward ? h.Dp : h.Cp);
@@ -555,14 +638,14 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
 
   static bool attr_set = false;   // per template instance
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_apply_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_apply_kernel<T, BO, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  tc_apply_kernel<T, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_out, p);
+  tc_apply_kernel<T, BO, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_out, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -570,11 +653,19 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
 template <typename E>
 static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out, int64_t N,
                             cudaStream_t st) {
+  const int bo = bwd ? h.bo_bwd : h.bo_fwd;
   switch (h.T) {
-    case 1: return launch_t<1, E>(h, bwd, in, out, N, st);
-    case 2: return launch_t<2, E>(h, bwd, in, out, N, st);
-    case 4: return launch_t<4, E>(h, bwd, in, out, N, st);
-    case 8: return launch_t<8, E>(h, bwd, in, out, N, st);
+    case 1: return bo == 256 ? launch_t<1, 256, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
+    case 2: return bo == 128 ? launch_t<2, 128, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
+    case 4:
+      switch (bo) {
+        case 128: return launch_t<4, 128, E>(h, bwd, in, out, N, st);
+        case 96: return launch_t<4, 96, E>(h, bwd, in, out, N, st);
+        case 64: return launch_t<4, 64, E>(h, bwd, in, out, N, st);
+        case 32: return launch_t<4, 32, E>(h, bwd, in, out, N, st);
+      }
+      return cudaErrorInvalidValue;
+    case 8: return bo == 32 ? launch_t<8, 32, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }

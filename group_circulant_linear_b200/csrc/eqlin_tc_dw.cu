@@ -7,27 +7,37 @@
 //   dW_hat_k[d, c] = sum_n G_k[n, d] * conj(X_k[n, c]),   G = DFT_t(gy), X = DFT_t(x)
 //   dW[d, c, tau]  = IDFT_k(dW_hat)[tau]   (with the 1/T),   db[d] = sum_n G_0[n, d]
 //
-// For a complex frequency the two real outputs come from two block products
-// of N = 2*BC columns:  [Re | Im] = Re G [Re X ; -Im X] + Im G [Im X ; Re X],
-// so p4 again needs six real GEMMs.
+// The MMA's M side (128 rows of TMEM) takes d or c, whichever pads less to a
+// multiple of 128; the other side is the N side, BC <= 128 channels.  For a
+// complex frequency the two real outputs come from two block products of
+// N = 2*BC columns, so p4 again needs six real GEMMs:
+//   M = d:  [Re | Im] = Re G [Re X ; -Im X] + Im G [Im X ; Re X]
+//           (B planes per complex frequency: Im X, Re X, -Im X)
+//   M = c:  [Re | Im] = Re X [Re G ; Im G] + Im X [Im G ; -Re G]
+//           (the transposed product conj(X)^T G; B planes: Re G, Im G, -Re G)
 //
-// Work unit of one CTA: 128 output channels d x BC input channels c x one
-// contiguous chunk of tokens, in stages of 16 tokens.  Roles:
-//   warp 8     (producer)  TMA: the stage's gy rows of the 128 d channels and
-//              x rows of the BC c channels into shared memory, and L2
-//              prefetches of later stages
-//   warps 0-3  (one thread per d)  read the channel's T group values of the 16
-//              tokens, take the group DFT (packed token pairs for T <= 4, FP32
-//              for T = 8), keep sum_n G_0 in FP32 for db and write the K-major
-//              (token-contiguous) A planes; after the main loop they read the
-//              accumulators out of TMEM
-//   warps 4-7  (one thread per c)  the same for x, writing the B planes
-//              (real frequencies, then Im X, Re X, -Im X per complex one)
-//   warp 9     allocates TMEM; one thread issues the MMAs
+// Work unit of one CTA: 128 M channels x BC N channels x one contiguous chunk
+// of tokens, in stages of 16 tokens.  Roles:
+//   warp 16    (producer)  TMA: the stage's rows of the M-side input (gy or x)
+//              for the 128 M channels and of the N-side input for the BC N
+//              channels into a raw ring, and L2 prefetches of later stages
+//   warps 0-15 (transform) two groups of eight warps, group g taking tokens
+//              8g .. 8g+7 of every stage.  In a group, warps 0-3 take one M
+//              channel each (A planes) and warps 4-7 one N channel each (B
+//              planes): read the channel's T group values of the 8 tokens,
+//              take the group DFT (packed token pairs for T <= 4, FP32 for
+//              T = 8), keep sum_n G_0 in FP32 for db on the side that holds gy,
+//              and write K-major (token-contiguous) operand planes.  After the
+//              main loop the A warps of both groups read the accumulators out
+//              of TMEM, each group half of the N columns
+//   warp 17    allocates TMEM; the warp runs the MMA loop and one lane issues
+// The raw ring (filled by TMA, freed once the transform has read a slot) and
+// the operand ring (filled by the transform, freed by the MMA commit) are
+// separate, so loads run ahead of the tensor core by the whole raw ring.
 // The per-chunk partial planes go to the handle's workspace as
-// [chunk][plane][c][d]; a second kernel sums the chunks in a fixed order and
-// applies the inverse DFT (deterministic, no atomics).  All waits are bounded
-// as in eqlin_tc.cu.
+// [chunk][plane][N channel][M channel]; a second kernel sums the chunks in a
+// fixed order and applies the inverse DFT (deterministic, no atomics).  All
+// waits are bounded as in eqlin_tc.cu.
 #include <cudaTypedefs.h>
 
 #include <type_traits>
@@ -44,7 +54,7 @@ using namespace ptx;
 template <int T>
 struct Cfg {
   using G = Group<T>;
-  static constexpr int BM = 128;                          // output channels d per tile (MMA M)
+  static constexpr int BM = 128;                          // M channels per tile (MMA M)
   static constexpr int BKN = 16;                          // tokens per stage (one MMA K step)
   static constexpr int ROWB = BKN * 2;                    // 32-byte K-major rows, 32B swizzle
   static constexpr int BC_MAX = (512 / T) < 128 ? (512 / T) : 128;
@@ -52,32 +62,40 @@ struct Cfg {
   static constexpr int A_PLANE_BYTES = BM * ROWB;
   static constexpr int A_BYTES = T * A_PLANE_BYTES;
   static constexpr int B_BYTES = Q * BC_MAX * ROWB;       // plane stride is BC * ROWB at run time
-  // raw tiles of a stage (TMA, row-major): gy [16 tokens][128 d x T], x [16 tokens][BC x T]
-  static constexpr int GY_ROWB = BM * T * 2;
-  static constexpr int X_ROWB_MAX = BC_MAX * T * 2;
-  static constexpr int RAW_BYTES = BKN * (GY_ROWB + X_ROWB_MAX);
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
-  static constexpr int STAGES_FIT = (220 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static_assert(STAGES >= 2, "two stages must fit");
-  static constexpr int NBAR = 4 * STAGES + 2;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int OP_BYTES = A_BYTES + B_BYTES;
+  // raw tiles of a stage (TMA, row-major): M side [16 tokens][128 x T], N side [16 tokens][BC x T]
+  static constexpr int MA_ROWB = BM * T * 2;
+  static constexpr int NB_ROWB_MAX = BC_MAX * T * 2;
+  static constexpr int RAW_BYTES = BKN * (MA_ROWB + NB_ROWB_MAX);
+  // three operand slots where three raw slots still fit (the transform writes
+  // stage k + 2 while the MMAs of k and k + 1 are in flight), else two; the
+  // rest of 220 KB for raw slots (memory latency)
+  static constexpr int OP_STAGES = (220 * 1024 - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3 : 2;
+  static constexpr int RAW_FIT = (220 * 1024 - OP_STAGES * OP_BYTES) / RAW_BYTES;
+  static constexpr int RAW_STAGES = RAW_FIT > 6 ? 6 : RAW_FIT;
+  static_assert(RAW_STAGES >= 2, "two raw stages must fit");
+  static constexpr int NBAR = 2 * RAW_STAGES + 2 * OP_STAGES + 2;
+  static constexpr int SMEM_BYTES = OP_STAGES * OP_BYTES + RAW_STAGES * RAW_BYTES + NBAR * 8 + 16 +
+                                    BM * 4 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
-  static constexpr int PRODUCER = 8, MMA_WARP = 9;
-  static constexpr int THREADS = 320;
+  static constexpr int TR_WARPS = 16;                     // two token groups x (4 A + 4 B warps)
+  static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;
+  static constexpr int THREADS = (TR_WARPS + 2) * 32;
   static constexpr int PF_STAGES = 12;                    // L2 prefetch distance (stages)
-  static constexpr int GY_BOX = BM * T <= 256 ? BM * T : 256;   // gy TMA box width (elements)
+  static constexpr int MA_BOX = BM * T <= 256 ? BM * T : 256;   // M-side TMA box width (elements)
   static constexpr int W = packed::Words<T>::n;
 };
 
 struct Params {
   int64_t N;
   int Cp, Dp;
-  int BC;                 // input channels per tile (multiple of 16)
-  int n_dt, n_ct;         // d tiles, c tiles
+  int mdim;               // M-side channels (Dp, or Cp when swapped)
+  int BC;                 // N-side channels per tile (multiple of 16)
+  int n_mt, n_nt;         // M tiles, N tiles
+  int swap;               // 0: M = d (A from gy, B from x); 1: M = c (A from x, B from gy)
   int64_t chunk;          // tokens per split (multiple of BKN)
-  int x_box;              // x TMA box width (elements), divides BC * T
-  float* part;            // [splits][T][Cp][Dp]
+  int nb_box;             // N-side TMA box width (elements), divides BC * T
+  float* part;            // [splits][T][N channels][M channels]
   float* dbpart;          // [splits][Dp]
   int* err;
   uint32_t wait_limit;
@@ -136,49 +154,53 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
 
 template <int T, typename E>
 __global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
-tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_gy, Params p) {
+tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_n, Params p) {
   using C = Cfg<T>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* a_buf = smem;
-  uint8_t* b_buf = a_buf + C::STAGES * C::A_BYTES;
-  uint8_t* raw_buf = b_buf + C::STAGES * C::B_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(raw_buf + C::STAGES * C::RAW_BYTES);
-  uint64_t* raw_full = bars;                      // TMA
-  uint64_t* raw_empty = raw_full + C::STAGES;     // 8 transform warps
-  uint64_t* op_full = raw_empty + C::STAGES;      // 8 transform warps
-  uint64_t* op_empty = op_full + C::STAGES;       // MMA commit
-  uint64_t* acc_full = op_empty + C::STAGES;
+  uint8_t* op_buf = smem;                                         // [OP_STAGES][A | B]
+  uint8_t* raw_buf = op_buf + C::OP_STAGES * C::OP_BYTES;        // [RAW_STAGES][M side | N side]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw_buf + C::RAW_STAGES * C::RAW_BYTES);
+  uint64_t* raw_full = bars;                          // TMA bytes
+  uint64_t* raw_empty = raw_full + C::RAW_STAGES;     // the transform warps have read the slot
+  uint64_t* op_full = raw_empty + C::RAW_STAGES;      // the transform warps have written the operands
+  uint64_t* op_empty = op_full + C::OP_STAGES;        // MMA commit
+  uint64_t* acc_full = op_empty + C::OP_STAGES;
   uint64_t* drain_bar = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* db_half = reinterpret_cast<float*>(tmem_slot + 4);       // [BM] token group 1's db sums
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int tiles = p.n_dt * p.n_ct;
+  const int tiles = p.n_mt * p.n_nt;
   const int tile = blockIdx.x % tiles, z = blockIdx.x / tiles;
-  const int d0 = (tile / p.n_ct) * C::BM, c0 = (tile % p.n_ct) * p.BC;
+  const int mt = tile / p.n_nt, nt = tile % p.n_nt;
+  const int m0 = mt * C::BM, n0 = nt * p.BC;
   const int64_t nbeg = (int64_t)z * p.chunk;
   const int64_t nend = (nbeg + p.chunk < p.N) ? nbeg + p.chunk : p.N;
   const int nst = (int)((nend - nbeg + C::BKN - 1) / C::BKN);
   const uint32_t limit = p.wait_limit;
   const int BC = p.BC;
   const uint32_t b_plane = (uint32_t)BC * C::ROWB;
-  const int x_rowb = BC * T * 2;                  // raw x row bytes of this tile
+  const int nb_rowb = BC * T * 2;                 // raw N-side row bytes of this tile
+  const bool swap = p.swap != 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < C::RAW_STAGES; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], 8);
-      mbar_init(&op_full[i], 8);
+      mbar_init(&raw_empty[i], C::TR_WARPS);
+    }
+    for (int i = 0; i < C::OP_STAGES; ++i) {
+      mbar_init(&op_full[i], C::TR_WARPS);
       mbar_init(&op_empty[i], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&map_x);
-    prefetch_tensormap(&map_gy);
+    prefetch_tensormap(&map_m);
+    prefetch_tensormap(&map_n);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -189,130 +211,155 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 8) {
+  if (warp < C::TR_WARPS) {
     // --------------------------------------------------- transform warps
-    const bool is_a = warp < 4;
-    const int r = (warp & 3) * 32 + lane;                 // operand row: d (A) or c (B)
+    const int grp = warp >> 3;                             // token group: tokens 8*grp .. 8*grp+7
+    const bool is_a = (warp & 7) < 4;
+    const int r = (warp & 3) * 32 + lane;                  // operand row: M channel (A) or N channel (B)
     const bool active = is_a || r < BC;
+    // the side that holds gy also sums G_0 for db: A when M = d, B when M = c
+    const bool sums_db = is_a != swap;
     // this thread's channel in the raw tile rows
-    const uint32_t raw_col = is_a ? (uint32_t)((r / (C::GY_BOX / T)) * C::BKN * C::GY_BOX * 2 +
-                                               (r % (C::GY_BOX / T)) * T * 2)
-                                  : (uint32_t)((r * T / p.x_box) * C::BKN * p.x_box * 2 +
-                                               ((r * T) % p.x_box) * 2);
-    const uint32_t raw_rowb = is_a ? (uint32_t)(C::GY_BOX * 2) : (uint32_t)(p.x_box * 2);
-    const uint32_t raw_base = is_a ? 0u : (uint32_t)(C::BKN * C::GY_ROWB);
+    const uint32_t raw_col = is_a ? (uint32_t)((r / (C::MA_BOX / T)) * C::BKN * C::MA_BOX * 2 +
+                                               (r % (C::MA_BOX / T)) * T * 2)
+                                  : (uint32_t)((r * T / p.nb_box) * C::BKN * p.nb_box * 2 +
+                                               ((r * T) % p.nb_box) * 2);
+    const uint32_t raw_rowb = is_a ? (uint32_t)(C::MA_BOX * 2) : (uint32_t)(p.nb_box * 2);
+    const uint32_t raw_base = (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + grp * 8 * raw_rowb;
+    const uint32_t off = kmajor_off(r, grp);
     float dbacc = 0.f;
-    int s = 0;
-    uint32_t ph = 0;
+    int rs = 0, os = 0;
+    uint32_t rph = 0, oph = 0;
     bool ok = true;
     for (int st = 0; st < nst; ++st) {
-      if (!wwait_all(&raw_full[s], ph, limit, abort_flag) ||
-          !wwait(&op_empty[s], ph ^ 1, limit, abort_flag, lane)) {
-        ok = false;
-        break;
-      }
+      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag)) { ok = false; break; }
+      uint32_t wv[8][C::W];
       if (active) {
-        const uint8_t* raw = raw_buf + s * C::RAW_BYTES + raw_base + raw_col;
-        uint8_t* a_st = a_buf + s * C::A_BYTES;
-        uint8_t* b_st = b_buf + s * C::B_BYTES;
+        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
 #pragma unroll
-        for (int g = 0; g < C::BKN / 8; ++g) {
-          uint32_t wv[8][C::W];
+        for (int j = 0; j < 8; ++j) {
+          const uint8_t* src = raw + j * raw_rowb;
+          if constexpr (C::W == 4) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src);
+            wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
+          } else if constexpr (C::W == 2) {
+            const uint2 u = *reinterpret_cast<const uint2*>(src);
+            wv[j][0] = u.x; wv[j][1] = u.y;
+          } else if constexpr (T == 2) {
+            wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
+          } else {
+            wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+          }
+        }
+      }
+      // the raw slot may be refilled by TMA (async proxy) once these generic
+      // reads are ordered before it
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[rs]);
+      if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
+      uint32_t Pw[T][4];
+      if (active) {
+        if constexpr (T <= 4) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint8_t* src = raw + (g * 8 + j) * raw_rowb;
-            if constexpr (C::W == 4) {
-              const uint4 u = *reinterpret_cast<const uint4*>(src);
-              wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
-            } else if constexpr (C::W == 2) {
-              const uint2 u = *reinterpret_cast<const uint2*>(src);
-              wv[j][0] = u.x; wv[j][1] = u.y;
-            } else if constexpr (T == 2) {
-              wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
-            } else {
-              wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+          for (int pr = 0; pr < 4; ++pr) {
+            uint32_t P[T];
+            packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
+#pragma unroll
+            for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
+            if (sums_db) {
+              const float2 f = packed::Pair<E>::to_f2(P[0]);
+              dbacc += f.x + f.y;
             }
           }
-          uint32_t Pw[T][4];
-          if constexpr (T <= 4) {
+        } else {
+          // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
 #pragma unroll
-            for (int pr = 0; pr < 4; ++pr) {
-              uint32_t P[T];
-              packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
+          for (int pr = 0; pr < 4; ++pr) {
+            float Pa[T], Pb[T], va[T], vb[T];
+            const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
+            const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
 #pragma unroll
-              for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
-              if (is_a) {
-                const float2 f = packed::Pair<E>::to_f2(P[0]);
-                dbacc += f.x + f.y;
-              }
-            }
-          } else {
-            // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
+            for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
+            G::dft(va, Pa);
+            G::dft(vb, Pb);
+            if (sums_db) dbacc += Pa[0] + Pb[0];
 #pragma unroll
-            for (int pr = 0; pr < 4; ++pr) {
-              float Pa[T], Pb[T], va[T], vb[T];
-              const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
-              const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
-#pragma unroll
-              for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
-              G::dft(va, Pa);
-              G::dft(vb, Pb);
-              dbacc += Pa[0] + Pb[0];
-#pragma unroll
-              for (int q = 0; q < T; ++q) {
-                E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
-                Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
-              }
-            }
-          }
-          const uint32_t off = kmajor_off(r, g);
-          if (is_a) {
-#pragma unroll
-            for (int q = 0; q < T; ++q)
-              *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
-                  make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
-          } else {
-#pragma unroll
-            for (int f = 0; f < G::nreal; ++f)
-              *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
-                  make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
-#pragma unroll
-            for (int k = 1; k <= G::ncomplex; ++k) {
-              const int pr = G::nreal + 2 * (k - 1);
-              const int q = G::nreal + 3 * (k - 1);
-              const uint32_t* re = Pw[pr];
-              const uint32_t* im = Pw[pr + 1];
-              *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(im[0], im[1], im[2], im[3]);
-              *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(re[0], re[1], re[2], re[3]);
-              *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
-                  make_uint4(packed::neg2(im[0]), packed::neg2(im[1]), packed::neg2(im[2]), packed::neg2(im[3]));
+            for (int q = 0; q < T; ++q) {
+              E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
+              Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
             }
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&raw_empty[s]);
+      // the operand slot must have been consumed by the MMAs issued from it
+      if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane)) { ok = false; break; }
+      if (active) {
+        uint8_t* a_st = op_buf + os * C::OP_BYTES;
+        uint8_t* b_st = a_st + C::A_BYTES;
+        if (is_a) {
+#pragma unroll
+          for (int q = 0; q < T; ++q)
+            *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
+                make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+        } else {
+#pragma unroll
+          for (int f = 0; f < G::nreal; ++f)
+            *reinterpret_cast<uint4*>(b_st + f * b_plane + off) = make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const int pr = G::nreal + 2 * (k - 1);
+            const int q = G::nreal + 3 * (k - 1);
+            // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G)
+            const uint32_t* u0 = swap ? Pw[pr] : Pw[pr + 1];
+            const uint32_t* u1 = swap ? Pw[pr + 1] : Pw[pr];
+            *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+            *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(u1[0], u1[1], u1[2], u1[3]);
+            *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
+                make_uint4(packed::neg2(u0[0]), packed::neg2(u0[1]), packed::neg2(u0[2]), packed::neg2(u0[3]));
+          }
+        }
+      }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&op_full[s]);
-      if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      if (lane == 0) mbar_arrive(&op_full[os]);
+      if (++os == C::OP_STAGES) { os = 0; oph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
 
+    // db: the side that sums G_0 writes its channels' sums; group 1 hands
+    // its sums to group 0 through shared memory.  Only the tiles of the other
+    // side's first tile write, so each d is written once per chunk.
+    const bool db_tile = swap ? (mt == 0) : (nt == 0);
+    if (sums_db && db_tile) {
+      const int bar_id = is_a ? 1 : 2;
+      named_bar_sync(bar_id, 256);
+      if (grp == 1) db_half[r] = dbacc;
+      named_bar_sync(bar_id, 256);
+      const int d = (swap ? n0 : m0) + r;
+      if (grp == 0 && active && d < p.Dp) p.dbpart[(int64_t)z * p.Dp + d] = dbacc + db_half[r];
+    }
+
     if (is_a) {
       // ------------------------------------------------------- epilogue
-      // partial planes [z][T][Cp][Dp]: a warp stores 32 consecutive d of one c
+      // The A warps of both token groups (same TMEM lane quarter, same M
+      // channel).  Partial planes [z][T][N channel][M channel]: a warp stores
+      // 32 consecutive M channels of one N channel; group g takes the N
+      // columns [g * BC/2, (g+1) * BC/2).
+      const bool all_ok = named_bar_and(3, 256, ok);
       const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-      bool got = ok && wwait_all(acc_full, 0, limit, abort_flag);
-      if (!got && ok) raise_abort(abort_flag, p.err);
+      bool got = all_ok && wwait_all(acc_full, 0, limit, abort_flag);
+      if (!got && all_ok) raise_abort(abort_flag, p.err);
       if (got) {
         tc_fence_after();
-        const int d = d0 + r;
-        const bool row_ok = d < p.Dp;
+        const int m = m0 + r;
+        const bool row_ok = m < p.mdim;
+        const int ndim = swap ? p.Dp : p.Cp;
         const int64_t plane = (int64_t)p.Cp * p.Dp;
-        float* base = p.part + (int64_t)z * T * plane + d;
+        float* base = p.part + (int64_t)z * T * plane + m;
+        const int cbeg = grp * (BC / 2), cend = cbeg + BC / 2;
 #pragma unroll 1
-        for (int cc = 0; cc < BC; cc += 8) {
+        for (int cc = cbeg; cc < cend; cc += 8) {
           uint32_t rg[T][8];
 #pragma unroll
           for (int f = 0; f < G::nreal; ++f) tmem_ld_32x32b_x8(tmem_base + lane_addr + f * BC + cc, rg[f]);
@@ -328,12 +375,11 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
             for (int q = 0; q < T; ++q)
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const int c = c0 + cc + i;
-                if (c < p.Cp) base[q * plane + (int64_t)c * p.Dp] = __uint_as_float(rg[q][i]);
+                const int n = n0 + cc + i;
+                if (n < ndim) base[q * plane + (int64_t)n * p.mdim] = __uint_as_float(rg[q][i]);
               }
           }
         }
-        if (c0 == 0 && row_ok) p.dbpart[(int64_t)z * p.Dp + d] = dbacc;
       }
     }
   } else if (warp == C::PRODUCER) {
@@ -343,12 +389,12 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       uint32_t ph = 0;
       int64_t n_raw = 0;
       bool ok = true;
-      const uint32_t tx = (uint32_t)(C::BKN * (C::GY_ROWB + x_rowb));
+      const uint32_t tx = (uint32_t)(C::BKN * (C::MA_ROWB + nb_rowb));
       auto prefetch = [&](int ps) {
         if (ps >= nst) return;
         const int n = (int)(nbeg + (int64_t)ps * C::BKN);
-        for (int xb = 0; xb < C::BM * T; xb += C::GY_BOX) tma_prefetch_2d(&map_gy, d0 * T + xb, n);
-        for (int xb = 0; xb < BC * T; xb += p.x_box) tma_prefetch_2d(&map_x, c0 * T + xb, n);
+        for (int xb = 0; xb < C::BM * T; xb += C::MA_BOX) tma_prefetch_2d(&map_m, m0 * T + xb, n);
+        for (int xb = 0; xb < BC * T; xb += p.nb_box) tma_prefetch_2d(&map_n, n0 * T + xb, n);
       };
       for (int i = 0; i < C::PF_STAGES; ++i) prefetch(i);
       for (int st = 0; st < nst; ++st) {
@@ -357,54 +403,65 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         mbar_arrive_expect_tx(&raw_full[s], tx);
         const int n = (int)(nbeg + (int64_t)st * C::BKN);
         uint8_t* dst = raw_buf + s * C::RAW_BYTES;
-        for (int b = 0; b < C::BM * T / C::GY_BOX; ++b)
-          tma_load_2d(dst + b * C::BKN * C::GY_BOX * 2, &map_gy, d0 * T + b * C::GY_BOX, n, &raw_full[s]);
-        dst += C::BKN * C::GY_ROWB;
-        for (int b = 0; b < BC * T / p.x_box; ++b)
-          tma_load_2d(dst + b * C::BKN * p.x_box * 2, &map_x, c0 * T + b * p.x_box, n, &raw_full[s]);
+        for (int b = 0; b < C::BM * T / C::MA_BOX; ++b)
+          tma_load_2d(dst + b * C::BKN * C::MA_BOX * 2, &map_m, m0 * T + b * C::MA_BOX, n, &raw_full[s]);
+        dst += C::BKN * C::MA_ROWB;
+        for (int b = 0; b < BC * T / p.nb_box; ++b)
+          tma_load_2d(dst + b * C::BKN * p.nb_box * 2, &map_n, n0 * T + b * p.nb_box, n, &raw_full[s]);
         ++n_raw;
-        if (++s == C::STAGES) { s = 0; ph ^= 1; }
+        if (++s == C::RAW_STAGES) { s = 0; ph ^= 1; }
       }
       if (!ok) raise_abort(abort_flag, p.err);
-      for (int i = 0; i < C::STAGES; ++i)
-        if (n_raw > i) mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::STAGES) & 1), kDefaultWaitLimit);
+      // every issued TMA copy must land before the CTA exits
+      for (int i = 0; i < C::RAW_STAGES; ++i)
+        if (n_raw > i)
+          mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::RAW_STAGES) & 1), kDefaultWaitLimit);
     }
-  } else if (lane == 0) {
+  } else {
     // -------------------------------------------------------------- MMA
+    // The whole warp runs the loop and takes the waits together; one lane
+    // issues the tcgen05 instructions.
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
     const uint32_t id_real = idesc_f16(p.ab_fmt, (uint32_t)BC);
     const uint32_t id_cplx = idesc_f16(p.ab_fmt, (uint32_t)(2 * BC));
+    // descriptors of slot 0, advanced by byte offset >> 4 (start-address field)
+    const uint64_t desc0 = smem_desc(smem_u32(op_buf), C::ROWB);
+    // window of the first complex product: M = d uses B planes q+1..q+2, M = c planes q..q+1
+    const int w1 = swap ? 0 : 1, w2 = swap ? 1 : 0;
     for (int st = 0; st < nst; ++st) {
-      if (!bwait(&op_full[s], ph, limit, abort_flag)) { ok = false; break; }
+      if (!wwait(&op_full[s], ph, limit, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t a_st = smem_u32(a_buf + s * C::A_BYTES);
-      const uint32_t b_st = smem_u32(b_buf + s * C::B_BYTES);
-      const uint32_t first = st > 0 ? 1u : 0u;
+      if (lane == 0) {
+        const uint64_t a_d = desc0 + (uint64_t)((s * C::OP_BYTES) >> 4);
+        const uint64_t b_d = a_d + (uint64_t)(C::A_BYTES >> 4);
+        const uint32_t bp = b_plane >> 4;
+        const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
-      for (int f = 0; f < G::nreal; ++f)
-        mma_f16_ss(tmem_base + f * BC, smem_desc(a_st + f * C::A_PLANE_BYTES, C::ROWB),
-                   smem_desc(b_st + f * b_plane, C::ROWB), id_real, first);
+        for (int f = 0; f < G::nreal; ++f)
+          mma_f16_ss(tmem_base + f * BC, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + f * bp, id_real, first);
 #pragma unroll
-      for (int k = 1; k <= G::ncomplex; ++k) {
-        const int pr = G::nreal + 2 * (k - 1);
-        const int q = G::nreal + 3 * (k - 1);
-        const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
-        // [Re | Im] += Re G [Re X ; -Im X]
-        mma_f16_ss(col, smem_desc(a_st + pr * C::A_PLANE_BYTES, C::ROWB),
-                   smem_desc(b_st + (q + 1) * b_plane, C::ROWB), id_cplx, first);
-        // [Re | Im] += Im G [Im X ; Re X]
-        mma_f16_ss(col, smem_desc(a_st + (pr + 1) * C::A_PLANE_BYTES, C::ROWB),
-                   smem_desc(b_st + q * b_plane, C::ROWB), id_cplx, 1u);
+        for (int k = 1; k <= G::ncomplex; ++k) {
+          const int pr = G::nreal + 2 * (k - 1);
+          const int q = G::nreal + 3 * (k - 1);
+          const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
+          // [Re | Im] += (Re plane of A) [first window] + (Im plane of A) [second window]
+          mma_f16_ss(col, a_d + ((pr * C::A_PLANE_BYTES) >> 4), b_d + (q + w1) * bp, id_cplx, first);
+          mma_f16_ss(col, a_d + (((pr + 1) * C::A_PLANE_BYTES) >> 4), b_d + (q + w2) * bp, id_cplx, 1u);
+        }
+        mma_commit(&op_empty[s]);
       }
-      mma_commit(&op_empty[s]);
-      if (++s == C::STAGES) { s = 0; ph ^= 1; }
+      __syncwarp();
+      if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
     }
-    if (ok) mma_commit(acc_full);
-    else raise_abort(abort_flag, p.err);
-    mma_commit(drain_bar);
-    mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+    if (lane == 0) {
+      if (ok) mma_commit(acc_full);
+      else raise_abort(abort_flag, p.err);
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -416,19 +473,26 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
 }
 
 struct Plan {
-  int BC, n_dt, n_ct, splits;
+  int BC, n_mt, n_nt, splits;
+  bool swap;
   int64_t chunk;
 };
 
+// M side: d, unless c pads less to a multiple of 128.  N side: tiles of BC
+// channels (a multiple of 16, at most BC_MAX) that split it evenly.
 template <int T>
 static Plan plan(int64_t Cp, int64_t Dp, int64_t N, int sm_count) {
   using C = Cfg<T>;
   Plan pl;
-  const int64_t nct = (Cp + C::BC_MAX - 1) / C::BC_MAX;
-  pl.BC = (int)(((Cp + nct - 1) / nct + 15) / 16 * 16);
-  pl.n_ct = (int)((Cp + pl.BC - 1) / pl.BC);
-  pl.n_dt = (int)((Dp + C::BM - 1) / C::BM);
-  const int tiles = pl.n_dt * pl.n_ct;
+  const int64_t pad_d = (Dp + C::BM - 1) / C::BM * C::BM - Dp;
+  const int64_t pad_c = (Cp + C::BM - 1) / C::BM * C::BM - Cp;
+  pl.swap = pad_c < pad_d;
+  const int64_t mdim = pl.swap ? Cp : Dp, ndim = pl.swap ? Dp : Cp;
+  const int64_t nnt = (ndim + C::BC_MAX - 1) / C::BC_MAX;
+  pl.BC = (int)(((ndim + nnt - 1) / nnt + 15) / 16 * 16);
+  pl.n_nt = (int)((ndim + pl.BC - 1) / pl.BC);
+  pl.n_mt = (int)((mdim + C::BM - 1) / C::BM);
+  const int tiles = pl.n_mt * pl.n_nt;
   int s = sm_count / tiles;
   if (s < 1) s = 1;
   const int64_t max_by_n = (N + C::BKN - 1) / C::BKN;
@@ -455,9 +519,11 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   p.N = N;
   p.Cp = (int)h.Cp;
   p.Dp = (int)h.Dp;
+  p.mdim = (int)(pl.swap ? h.Cp : h.Dp);
   p.BC = pl.BC;
-  p.n_dt = pl.n_dt;
-  p.n_ct = pl.n_ct;
+  p.n_mt = pl.n_mt;
+  p.n_nt = pl.n_nt;
+  p.swap = pl.swap ? 1 : 0;
   p.chunk = pl.chunk;
   p.part = h.ws;
   p.dbpart = h.ws + (int64_t)pl.splits * T * h.Cp * h.Dp;
@@ -475,14 +541,14 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   }
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  // x box: the largest power-of-two width <= 256 elements that divides BC * T
-  int x_box = 256;
-  while ((pl.BC * T) % x_box) x_box >>= 1;
-  CUtensorMap map_x, map_gy;
-  const void* srcs[2] = {x, gy};
-  const int64_t widths[2] = {h.Cp * T, h.Dp * T};
-  const int boxes[2] = {x_box, C::GY_BOX};
-  CUtensorMap* maps[2] = {&map_x, &map_gy};
+  // N-side box: the largest power-of-two width <= 256 elements that divides BC * T
+  int nb_box = 256;
+  while ((pl.BC * T) % nb_box) nb_box >>= 1;
+  CUtensorMap map_m, map_n;
+  const void* srcs[2] = {pl.swap ? x : gy, pl.swap ? gy : x};
+  const int64_t widths[2] = {(pl.swap ? h.Cp : h.Dp) * T, (pl.swap ? h.Dp : h.Cp) * T};
+  const int boxes[2] = {C::MA_BOX, nb_box};
+  CUtensorMap* maps[2] = {&map_m, &map_n};
   for (int i = 0; i < 2; ++i) {
     cuuint64_t dims[2] = {(cuuint64_t)widths[i], (cuuint64_t)N};
     cuuint64_t strides[1] = {(cuuint64_t)widths[i] * 2};
@@ -493,7 +559,7 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  p.x_box = x_box;
+  p.nb_box = nb_box;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(tc_dw_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -501,12 +567,13 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const unsigned grid = (unsigned)(pl.n_dt * pl.n_ct * pl.splits);
-  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(map_x, map_gy, p);
+  const unsigned grid = (unsigned)(pl.n_mt * pl.n_nt * pl.splits);
+  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(map_m, map_n, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);
-  return launch_dw_reduce(h, pl.splits, p.part, p.dbpart, dW, db, /*cd_layout=*/true, st);
+  // partials are [N channel][M channel]: c-major over d when M = d
+  return launch_dw_reduce(h, pl.splits, p.part, p.dbpart, dW, db, /*cd_layout=*/!pl.swap, st);
 }
 
 template <typename E>
