@@ -415,60 +415,62 @@ simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restr
 
 // Sum the splits in index order, then inverse DFT along the frequency planes.
 // Partials are [splits][T][Dp][Cp] (cd_layout false) or [splits][T][Cp][Dp]
-// (cd_layout true).  One block of 32 x 8 threads per 32 (d) x 8 (c) tile,
-// one element per thread: it sums the splits in index order (four partial
-// sums kept apart, combined in a fixed order), takes the inverse DFT and
-// stages the tile in shared memory so that dW [Dp][Cp][T] is written row by
-// row.
-template <int T>
+// (cd_layout true).  One block of 256 threads per tile of 32 (d) x 8 (c)
+// (cd_layout) or 8 (d) x 32 (c) channels, one element per thread, with the
+// warp's 32 lanes along the partials' contiguous index.  A thread sums the
+// splits in index order, eight at a time with all of a group's T x 8 loads
+// issued before any is added (the reduction is latency bound), in a fixed
+// order; takes the inverse DFT; and stages the tile in shared memory so that
+// dW [Dp][Cp][T] is written row by row.
+template <int T, bool CD>
 __global__ void __launch_bounds__(256)
 dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart, float* __restrict__ dW,
-                 float* __restrict__ db, int splits, int Cp, int Dp, bool cd_layout) {
+                 float* __restrict__ db, int splits, int Cp, int Dp) {
   using G = Group<T>;
-  __shared__ float sV[32][8 * T + 1];             // [d][c*T + t] of the tile
-  const int c0 = blockIdx.x * 8, d0 = blockIdx.y * 32;
+  constexpr int DT = CD ? 32 : 8, CT = CD ? 8 : 32;  // tile: d x c
+  constexpr int ZG = 8;                               // splits per load group
+  __shared__ float sV[DT][CT * T + 1];                // [d][c*T + t] of the tile
+  const int c0 = blockIdx.x * CT, d0 = blockIdx.y * DT;
   const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
   const int64_t plane = (int64_t)Cp * Dp;
-  // thread -> (d, c): the partials' contiguous index runs along tx
-  int d, c;
-  if (cd_layout) { d = d0 + tx; c = c0 + ty; }
-  else { d = d0 + (threadIdx.x >> 3); c = c0 + (threadIdx.x & 7); }
+  const int d = CD ? d0 + tx : d0 + ty;
+  const int c = CD ? c0 + ty : c0 + tx;
   float P[T], v[T];
+#pragma unroll
+  for (int q = 0; q < T; ++q) P[q] = 0.f;
   if (d < Dp && c < Cp) {
-    const int64_t idx = cd_layout ? (int64_t)c * Dp + d : (int64_t)d * Cp + c;
+    const float* src = part + (CD ? (int64_t)c * Dp + d : (int64_t)d * Cp + c);
+    const int64_t zs = (int64_t)T * plane;
+    for (int z0 = 0; z0 < splits; z0 += ZG) {
+      float val[ZG][T];
 #pragma unroll
-    for (int q = 0; q < T; ++q) {
-      const float* src = part + (int64_t)q * plane + idx;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-      int z = 0;
-      for (; z + 4 <= splits; z += 4) {
-        s0 += src[(int64_t)(z + 0) * T * plane];
-        s1 += src[(int64_t)(z + 1) * T * plane];
-        s2 += src[(int64_t)(z + 2) * T * plane];
-        s3 += src[(int64_t)(z + 3) * T * plane];
+      for (int i = 0; i < ZG; ++i)
+#pragma unroll
+        for (int q = 0; q < T; ++q)
+          val[i][q] = (z0 + i < splits) ? __ldg(src + (int64_t)(z0 + i) * zs + (int64_t)q * plane) : 0.f;
+#pragma unroll
+      for (int q = 0; q < T; ++q) {
+        const float g = ((val[0][q] + val[1][q]) + (val[2][q] + val[3][q])) +
+                        ((val[4][q] + val[5][q]) + (val[6][q] + val[7][q]));
+        P[q] += g;
       }
-      for (; z < splits; ++z) s0 += src[(int64_t)z * T * plane];
-      P[q] = (s0 + s1) + (s2 + s3);
     }
-  } else {
-#pragma unroll
-    for (int q = 0; q < T; ++q) P[q] = 0.f;
   }
   G::idft(P, v);
   const int dl = d - d0, cl = c - c0;
 #pragma unroll
   for (int t = 0; t < T; ++t) sV[dl][cl * T + t] = v[t];
   __syncthreads();
-  // each warp writes rows of 8*T contiguous floats
-  const int ncol = min(8, Cp - c0) * T;
-  for (int r = ty; r < 32; r += 8) {
+  // rows of CT*T contiguous floats, one warp per row at a time
+  const int ncol = min(CT, Cp - c0) * T;
+  for (int r = ty; r < DT; r += 8) {
     const int dd = d0 + r;
     if (dd >= Dp) continue;
     float* dst = dW + ((int64_t)dd * Cp + c0) * T;
     for (int j = tx; j < ncol; j += 32) dst[j] = sV[r][j];
   }
-  if (db && blockIdx.x == 0 && ty == 0) {
-    const int dd = d0 + tx;
+  if (db && blockIdx.x == 0 && threadIdx.x < DT) {
+    const int dd = d0 + threadIdx.x;
     if (dd < Dp) {
       float s = 0.f;
       for (int z = 0; z < splits; ++z) s += dbpart[(int64_t)z * Dp + dd];
@@ -480,8 +482,13 @@ dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpar
 template <int T>
 static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
                                float* dW, float* db, bool cd_layout, cudaStream_t st) {
-  dim3 grid((unsigned)((h.Cp + 7) / 8), (unsigned)((h.Dp + 31) / 32));
-  dw_reduce_kernel<T><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp, cd_layout);
+  if (cd_layout) {
+    dim3 grid((unsigned)((h.Cp + 7) / 8), (unsigned)((h.Dp + 31) / 32));
+    dw_reduce_kernel<T, true><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp);
+  } else {
+    dim3 grid((unsigned)((h.Cp + 31) / 32), (unsigned)((h.Dp + 7) / 8));
+    dw_reduce_kernel<T, false><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp);
+  }
   count_launches(1);
   return cudaGetLastError();
 }

@@ -468,6 +468,14 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       if (!ok) raise_abort(abort_flag, p.err);
       mma_commit(drain_bar);              // arrives once every issued MMA has completed
       mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+      // The last commit of each operand slot fires on the same completion as
+      // the drain's, and nothing else waits for it: an arrival that lands
+      // after the CTA has left would write into the shared memory of whatever
+      // the SM runs next.  (On an aborted run, with fewer commits, the
+      // wall-time cap ends the wait.)
+      const int64_t n_st = my_tiles * nk;
+      for (int i = 0; i < C::AB_ST; ++i)
+        if (n_st > i) mbar_wait(&ab_empty[i], (uint32_t)(((n_st - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
   } else {
     // ------------------------------------------------------ epilogue warps

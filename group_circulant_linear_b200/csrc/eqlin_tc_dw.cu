@@ -460,6 +460,13 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
       else raise_abort(abort_flag, p.err);
       mma_commit(drain_bar);
       mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+      // The last commit of each operand slot fires on the same completion as
+      // the drain's, and nothing else waits for it: an arrival that lands
+      // after the CTA has left would write into the shared memory of whatever
+      // the SM runs next.  (On an aborted run, with fewer commits, the
+      // wall-time cap ends the wait.)
+      for (int i = 0; i < C::OP_STAGES; ++i)
+        if (nst > i) mbar_wait(&op_empty[i], (uint32_t)(((nst - 1 - i) / C::OP_STAGES) & 1), kDefaultWaitLimit);
     }
     __syncwarp();
   }
