@@ -318,11 +318,21 @@ def main():
     avg_ms = statistics.mean(per[dom])
     kernel_of = {"fwd": "tc_apply", "dx": "tc_apply", "dw": "dw", "set_weights": "pretransform"}
     if dom[1] in ("fwd", "dx", "dw"):
+        # the bound is the resource the call's arithmetic intensity points at:
+        # tensor when its FLOP per algorithmic byte exceed the measured ridge
         flop = Ld.actual_flop()
-        achieved = flop / (avg_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_sustained"],
-                "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
+        byt = Ld.bytes_dw() if dom[1] == "dw" else Ld.bytes_fwd()
+        ridge = pk["bf16_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+        if flop / byt >= ridge / 2:
+            achieved = flop / (avg_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                    "frac": achieved / pk["bf16_sustained"],
+                    "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
+        else:
+            achieved = byt / (avg_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm_gbs"], "peak_kind": f"{pk['source']} HBM copy"}
+        roof["intensity_flop_per_byte"] = flop / byt
     else:
         byt = Ld.Dp * Ld.Cp * Ld.T * 2 * 2
         achieved = byt / (avg_ms * 1e-3) / 1e9
