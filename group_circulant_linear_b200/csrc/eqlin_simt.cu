@@ -111,8 +111,103 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
   (void)Q;
 }
 
+// Tensor-core weight images only, for handles that need no FP32 planes.
+// One thread makes 8 K-consecutive entries of one row of one image; those sit
+// in 16 contiguous bytes of a tile (see wtile_index), so every plane is one
+// 16-byte store.  Threads [0, nA) build the forward image (rows d, K c), the
+// rest the input-gradient image (rows c, K d), with consecutive threads on
+// consecutive c so that the W reads stay coalesced.  The values are those of
+// pretransform_kernel; K entries past the end are written as zeros.
+template <typename E>
+__device__ __forceinline__ uint16_t bits16(E v) {
+  uint16_t u;
+  __builtin_memcpy(&u, &v, 2);
+  return u;
+}
+
+template <typename E>
+__device__ __forceinline__ void store8(E* dst, const float (&v)[8]) {
+  uint4 u;
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = (uint32_t)bits16(Elem<E>::from_f(v[2 * i])) | ((uint32_t)bits16(Elem<E>::from_f(v[2 * i + 1])) << 16);
+  u.x = w[0]; u.y = w[1]; u.z = w[2]; u.w = w[3];
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+template <int T, typename E>
+__global__ void __launch_bounds__(256)
+pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __restrict__ wt_fwd,
+                       E* __restrict__ wt_bwd, float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b) {
+  using G = Group<T>;
+  static_assert(sizeof(E) == 2, "tensor-core images hold 16-bit elements");
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid < Dp) bias[tid] = b ? Elem<E>::to_f(b[tid]) : 0.f;
+  const int64_t gA = (Cp + 7) / 8, gB = (Dp + 7) / 8;
+  const int64_t nA = (int64_t)Dp * gA, nB = (int64_t)Cp * gB;
+  bool fwd;
+  int64_t row, k0;
+  if (tid < nA) {
+    fwd = true; row = tid / gA; k0 = (tid % gA) * 8;
+  } else if (tid < nA + nB) {
+    const int64_t j = tid - nA;
+    fwd = false; k0 = (j / Cp) * 8; row = j % Cp;
+  } else {
+    return;
+  }
+  const int64_t K = fwd ? Cp : Dp;
+  float P[8][T];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t k = k0 + i;
+    const int64_t base = fwd ? (row * Cp + k) * T : (k * Cp + row) * T;
+    float v[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) v[t] = k < K ? Elem<E>::to_f(W[base + t]) : 0.f;
+    G::dft(v, P[i]);
+  }
+  E* out = fwd ? wt_fwd : wt_bwd;
+  const int bo = fwd ? bo_f : bo_b;
+  const int64_t nkb = (K + TC_BK - 1) / TC_BK;
+  const float sr = 1.f / T, sc = 2.f / T;
+  float o[8];
+#pragma unroll
+  for (int f = 0; f < G::nreal; ++f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? P[i][f] * sr : 0.f;
+    store8(out + wtile_index(T, bo, nkb, row, k0, f), o);
+  }
+#pragma unroll
+  for (int k = 1; k <= G::ncomplex; ++k) {
+    const int pr = G::nreal + 2 * (k - 1), q = G::nreal + 3 * (k - 1);
+    // forward: (-Im, Re, Im); input gradient, conj(W_hat): (Im, Re, -Im)
+    const float s0 = fwd ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? s0 * (P[i][pr + 1] * sc) : 0.f;
+    store8(out + wtile_index(T, bo, nkb, row, k0, q + 0), o);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? P[i][pr] * sc : 0.f;
+    store8(out + wtile_index(T, bo, nkb, row, k0, q + 1), o);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? -s0 * (P[i][pr + 1] * sc) : 0.f;
+    store8(out + wtile_index(T, bo, nkb, row, k0, q + 2), o);
+  }
+}
+
 template <int T, typename E>
 static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b, cudaStream_t st) {
+  if constexpr (sizeof(E) == 2) {
+    if (!h.need_simt_fwd && !h.need_simt_bwd && h.wt_fwd && h.wt_bwd) {
+      const int64_t n = h.Dp * ((h.Cp + 7) / 8) + h.Cp * ((h.Dp + 7) / 8);
+      const int64_t threads = n > h.Dp ? n : h.Dp;
+      pretransform_tc_kernel<T, E><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+          (const E*)W, (const E*)b, (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd,
+          h.bo_bwd);
+      count_launches(1);
+      return cudaGetLastError();
+    }
+  }
   dim3 grid((unsigned)((h.Cp + pt::TILE - 1) / pt::TILE), (unsigned)((h.Dp + pt::TILE - 1) / pt::TILE));
   dim3 block(pt::TILE, pt::ROWS);
   pretransform_kernel<T, E><<<grid, block, 0, st>>>(
