@@ -210,6 +210,35 @@ constexpr uint32_t kDefaultWaitLimit = 0xFFFFFFFFu;
 // Count kernels enqueued by this library (reported by eqlin_launch_count).
 void count_launches(int n);
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of this library is launched with programmatic stream
+// serialization: its CTAs may start on SMs that the previous kernel in the
+// stream has already left, and run their prologue (barrier set-up, tensor
+// memory allocation) while that kernel finishes.  Each kernel therefore
+// calls grid_dep_wait() -- which returns once the previous grid has
+// completed and its memory is visible -- before its first global memory
+// access, and grid_dep_launch(), which lets the next kernel be scheduled
+// once every CTA of this one has issued it: at the start of short kernels,
+// after the main loop where a waiting dependent would slow the loop.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ------------------------------------------------------- launch wrappers
 // SIMT path (any T in {1,2,4,8}, any dtype).
 cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st);

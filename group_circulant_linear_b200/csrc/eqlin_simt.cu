@@ -37,6 +37,8 @@ pretransform_kernel(const E* __restrict__ W, const E* __restrict__ b, float* __r
                     float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b) {
   using G = Group<T>;
   using namespace pt;
+  grid_dep_launch();
+  grid_dep_wait();
   constexpr int Q = G::nreal + 3 * G::ncomplex;
   __shared__ float sP[T][TILE][TILE + 1];        // planes of the tile, [p][d][c]
   const int c0 = blockIdx.x * TILE, d0 = blockIdx.y * TILE;
@@ -142,6 +144,8 @@ pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __re
                        E* __restrict__ wt_bwd, float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b) {
   using G = Group<T>;
   static_assert(sizeof(E) == 2, "tensor-core images hold 16-bit elements");
+  grid_dep_launch();
+  grid_dep_wait();
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid < Dp) bias[tid] = b ? Elem<E>::to_f(b[tid]) : 0.f;
   const int64_t gA = (Cp + 7) / 8, gB = (Dp + 7) / 8;
@@ -201,20 +205,21 @@ static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b,
     if (!h.need_simt_fwd && !h.need_simt_bwd && h.wt_fwd && h.wt_bwd) {
       const int64_t n = h.Dp * ((h.Cp + 7) / 8) + h.Cp * ((h.Dp + 7) / 8);
       const int64_t threads = n > h.Dp ? n : h.Dp;
-      pretransform_tc_kernel<T, E><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-          (const E*)W, (const E*)b, (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd,
-          h.bo_bwd);
+      const cudaError_t e = launch_pdl(pretransform_tc_kernel<T, E>, dim3((unsigned)((threads + 255) / 256)),
+                                       dim3(256), 0, st, (const E*)W, (const E*)b, (E*)h.wt_fwd, (E*)h.wt_bwd,
+                                       h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
       count_launches(1);
-      return cudaGetLastError();
+      return e;
     }
   }
   dim3 grid((unsigned)((h.Cp + pt::TILE - 1) / pt::TILE), (unsigned)((h.Dp + pt::TILE - 1) / pt::TILE));
   dim3 block(pt::TILE, pt::ROWS);
-  pretransform_kernel<T, E><<<grid, block, 0, st>>>(
-      (const E*)W, (const E*)b, h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr,
-      (E*)h.wt_fwd, (E*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
+  const cudaError_t e = launch_pdl(
+      pretransform_kernel<T, E>, grid, block, 0, st, (const E*)W, (const E*)b,
+      h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr, (E*)h.wt_fwd, (E*)h.wt_bwd,
+      h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename E>
@@ -251,6 +256,8 @@ simt_apply_kernel(const E* __restrict__ in, const float* __restrict__ planes,
                   const float* __restrict__ bias, E* __restrict__ out, int64_t N, int K, int O) {
   using G = Group<T>;
   using namespace simt;
+  grid_dep_launch();
+  grid_dep_wait();
   __shared__ float Xs[T][BK][BM];
   __shared__ __align__(16) float Ws[T][BK][BO];
 
@@ -351,10 +358,11 @@ static cudaError_t simt_apply_t(const Handle& h, bool backward, const void* in, 
   const int64_t tiles_n = (N + simt::BM - 1) / simt::BM;
   if (tiles_n > 0x7fffffff) return cudaErrorInvalidValue;
   dim3 grid((unsigned)tiles_n, (unsigned)((O + simt::BO - 1) / simt::BO));
-  simt_apply_kernel<T, E><<<grid, simt::THREADS, 0, st>>>(
-      (const E*)in, backward ? h.wf_bwd : h.wf_fwd, backward ? nullptr : h.bias, (E*)out, N, K, O);
+  const cudaError_t e = launch_pdl(simt_apply_kernel<T, E>, grid, dim3(simt::THREADS), 0, st, (const E*)in,
+                                   (const float*)(backward ? h.wf_bwd : h.wf_fwd),
+                                   (const float*)(backward ? nullptr : h.bias), (E*)out, N, K, O);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename E>
@@ -410,6 +418,8 @@ simt_dw_kernel(const E* __restrict__ x, const E* __restrict__ gy, float* __restr
                float* __restrict__ dbpart, int64_t N, int Cp, int Dp, int64_t tok_per_split) {
   using G = Group<T>;
   using namespace simtdw;
+  grid_dep_launch();
+  grid_dep_wait();
   __shared__ float Gs[T][BK][BD];
   __shared__ __align__(16) float Xs[T][BK][BC];
   const int tid = threadIdx.x;
@@ -522,6 +532,8 @@ __global__ void __launch_bounds__(256)
 dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpart, float* __restrict__ dW,
                  float* __restrict__ db, int splits, int Cp, int Dp) {
   using G = Group<T>;
+  grid_dep_launch();
+  grid_dep_wait();
   constexpr int DT = CD ? 32 : 8, CT = CD ? 8 : 32;  // tile: d x c
   constexpr int ZG = 8;                               // splits per load group
   __shared__ float sV[DT][CT * T + 1];                // [d][c*T + t] of the tile
@@ -577,15 +589,18 @@ dw_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dbpar
 template <int T>
 static cudaError_t dw_reduce_t(const Handle& h, int splits, const float* part, const float* dbpart,
                                float* dW, float* db, bool cd_layout, cudaStream_t st) {
+  cudaError_t e;
   if (cd_layout) {
     dim3 grid((unsigned)((h.Cp + 7) / 8), (unsigned)((h.Dp + 31) / 32));
-    dw_reduce_kernel<T, true><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp);
+    e = launch_pdl(dw_reduce_kernel<T, true>, grid, dim3(256), 0, st, part, dbpart, dW, db, splits, (int)h.Cp,
+                   (int)h.Dp);
   } else {
     dim3 grid((unsigned)((h.Cp + 31) / 32), (unsigned)((h.Dp + 7) / 8));
-    dw_reduce_kernel<T, false><<<grid, 256, 0, st>>>(part, dbpart, dW, db, splits, (int)h.Cp, (int)h.Dp);
+    e = launch_pdl(dw_reduce_kernel<T, false>, grid, dim3(256), 0, st, part, dbpart, dW, db, splits, (int)h.Cp,
+                   (int)h.Dp);
   }
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, const float* dbpart,
@@ -611,9 +626,8 @@ static cudaError_t simt_dw_t(const Handle& h, const void* x, const void* gy, flo
   if ((size_t)splits * ((size_t)T * plane + h.Dp) * sizeof(float) > h.ws_bytes)
     return cudaErrorInvalidValue;
   dim3 grid((unsigned)((h.Cp + BC - 1) / BC), (unsigned)((h.Dp + BD - 1) / BD), (unsigned)splits);
-  simt_dw_kernel<T, E><<<grid, THREADS, 0, st>>>((const E*)x, (const E*)gy, part, dbpart, N,
-                                                 (int)h.Cp, (int)h.Dp, tps);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(simt_dw_kernel<T, E>, grid, dim3(THREADS), 0, st, (const E*)x, (const E*)gy, part,
+                             dbpart, N, (int)h.Cp, (int)h.Dp, tps);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return launch_dw_reduce(h, splits, part, dbpart, dW, db, /*cd_layout=*/false, st);

@@ -202,6 +202,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
                 Params p) {
   using C = Cfg<T, BO>;
   using G = Group<T>;
+  grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -256,6 +257,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();   // the previous kernel's writes are visible from here on
 
   if (warp < C::TR_WARPS) {
     // ----------------------------------------------------- transform warps
@@ -653,9 +655,10 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  tc_apply_kernel<T, BO, E><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, st>>>(map_in, map_out, p);
+  const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E>, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM_BYTES,
+                                   st, map_in, map_out, p);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 template <typename E>

@@ -210,6 +210,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();   // the previous kernel's writes are visible from here on
 
   if (warp < C::TR_WARPS) {
     // --------------------------------------------------- transform warps
@@ -326,6 +327,11 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
       if (++os == C::OP_STAGES) { os = 0; oph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
+    // The next kernel (the split reduction) may be scheduled once every role
+    // of every CTA is past its main loop.  Triggered any earlier, its CTAs
+    // would wait on these SMs through the whole loop, beside the transform
+    // warps whose issue slots bound it.
+    grid_dep_launch();
 
     // db: the side that sums G_0 writes its channels' sums; group 1 hands
     // its sums to group 0 through shared memory.  Only the tiles of the other
@@ -417,6 +423,8 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         if (n_raw > i)
           mbar_wait(&raw_full[i], (uint32_t)(((n_raw - 1 - i) / C::RAW_STAGES) & 1), kDefaultWaitLimit);
     }
+    __syncwarp();
+    grid_dep_launch();
   } else {
     // -------------------------------------------------------------- MMA
     // The whole warp runs the loop and takes the waits together; one lane
@@ -455,6 +463,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
       __syncwarp();
       if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
     }
+    grid_dep_launch();
     if (lane == 0) {
       if (ok) mma_commit(acc_full);
       else raise_abort(abort_flag, p.err);
@@ -575,8 +584,7 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
     attr_set = true;
   }
   const unsigned grid = (unsigned)(pl.n_mt * pl.n_nt * pl.splits);
-  tc_dw_kernel<T, E><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(map_m, map_n, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(tc_dw_kernel<T, E>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, map_m, map_n, p);
   if (e != cudaSuccess) return e;
   count_launches(1);
   // partials are [N channel][M channel]: c-major over d when M = d

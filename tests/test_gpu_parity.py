@@ -100,6 +100,38 @@ def test_integer_inputs_bit_exact(T, Cp, Dp, N, dt, amp):
     assert np.array_equal(out["db"], db)
 
 
+def test_back_to_back_dependencies():
+    """Kernels launched back to back may start their prologue under the
+    previous kernel's tail; each must still read its predecessor's output
+    (read after write) and must not overwrite a buffer an earlier kernel
+    reads (write after read).  Chain: x -L1-> y1 -L2-> y2 -L2dx-> g1
+    -L1dx-> x (overwriting the x that the first kernel read)."""
+    T, C1, C2, N = 4, 64, 96, 1000
+    a = inputs.make_inputs(T, C1, C2, N, "bf16", seed=7)
+    b = inputs.make_inputs(T, C2, C1, N, "bf16", seed=8)
+    ga, gb = _dev(a), _dev(b)
+    L1 = eqlin.EQLinear(ga["W"], ga["b"])
+    L2 = eqlin.EQLinear(gb["W"], gb["b"])
+    x = ga["x"].clone()
+    y1 = torch.empty((N, C2 * T), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty((N, C1 * T), dtype=torch.bfloat16, device="cuda")
+    g1 = torch.empty((N, C2 * T), dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        x_in = x.float().cpu().numpy()
+        eqlin.forward(L1.h, x, y1)
+        eqlin.forward(L2.h, y1, y2)
+        eqlin.backward_dx(L2.h, y2, g1)
+        eqlin.backward_dx(L1.h, g1, x)
+        torch.cuda.synchronize()
+        assert eqlin.get_error(L1.h) == 0 and eqlin.get_error(L2.h) == 0
+        k = {n: t.float().cpu().numpy() for n, t in (("y1", y1), ("y2", y2), ("g1", g1), ("x", x))}
+        tol = TOL["bf16"]
+        assert rel_err(k["y1"], oracle.forward(x_in, a["W"], a["b"])) <= tol
+        assert rel_err(k["y2"], oracle.forward(k["y1"], b["W"], b["b"])) <= tol
+        assert rel_err(k["g1"], oracle.backward_dx(k["y2"], b["W"])) <= tol
+        assert rel_err(k["x"], oracle.backward_dx(k["g1"], a["W"])) <= tol
+
+
 def _roll(a: torch.Tensor, ch: int, T: int, r: int) -> torch.Tensor:
     N = a.shape[0]
     return torch.roll(a.reshape(N, ch, T), r, dims=2).reshape(N, ch * T).contiguous()
