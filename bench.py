@@ -255,6 +255,12 @@ def main():
     kinds = ("set_weights", "fwd", "dx", "dw")
     ev_log = []   # (layer index, kind, start event, end event) during the timed region
 
+    # A layer's dW/db and its dx read the same inputs and write nothing the
+    # other reads, so dW/db runs on a second stream: its CTAs take the SMs
+    # that dx's last, partial wave leaves idle.  The main stream waits for it
+    # before each step ends (and before an all-reduce of dW/db).
+    side = torch.cuda.Stream(device=dev)
+
     def step(i, record=False):
         for li, s in enumerate(st):
             inp = s["sets"][i % N_SETS]
@@ -264,18 +270,26 @@ def main():
                 ("dx", lambda: eqlin.backward_dx(s["h"], inp["gy"], s["dx"])),
                 ("dw", lambda: eqlin.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"])),
             )
-            for kind, fn in calls:
-                if record:
+            if record:
+                # every call on the main stream, one after another, each
+                # between two events: the per-call times
+                for kind, fn in calls:
                     e0 = torch.cuda.Event(enable_timing=True)
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record(stream)
                     fn()
                     e1.record(stream)
                     ev_log.append((li, kind, e0, e1))
-                else:
-                    fn()
+            else:
+                calls[0][1]()
+                calls[1][1]()
+                side.wait_stream(stream)
+                calls[2][1]()
+                eqlin.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"], stream=side)
             if dist:
+                stream.wait_stream(side)
                 dp.allreduce_grads((s["dW"], s["db"]))
+        stream.wait_stream(side)
 
     def barrier():
         if dist:
@@ -371,8 +385,10 @@ def main():
                 s["b"].copy_(hb["b"], non_blocking=True)
                 eqlin.set_weights(s["h"], s["W"], s["b"])
                 eqlin.forward(s["h"], db_["x"], s["y"])
+                side.wait_stream(stream)
                 eqlin.backward_dx(s["h"], db_["gy"], s["dx"])
-                eqlin.backward_dw(s["h"], db_["x"], db_["gy"], s["dW"], s["db"])
+                eqlin.backward_dw(s["h"], db_["x"], db_["gy"], s["dW"], s["db"], stream=side)
+                stream.wait_stream(side)
                 if dist:
                     dp.allreduce_grads((s["dW"], s["db"]))
                 for k in ("y", "dx", "dW", "db"):
@@ -415,7 +431,8 @@ def main():
                 "workload": args.workload,
                 "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes))
                            for L in layers],
-                "step": "per layer: set_weights (weight DFT) + forward + dx + dW/db"
+                "step": "per layer: set_weights (weight DFT) + forward + dx + dW/db, dW/db on a second "
+                        "stream beside dx"
                         + (" + NCCL all-reduce of dW/db" if dist else ""),
                 "tokens_per_gpu": layers[0].N,
                 "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
