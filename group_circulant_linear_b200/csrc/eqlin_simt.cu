@@ -161,14 +161,47 @@ pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __re
     return;
   }
   const int64_t K = fwd ? Cp : Dp;
+  // W[d, c, 0..T): the forward image reads 8 consecutive c of one d (8T
+  // contiguous elements), the input-gradient image the same c of 8
+  // consecutive d (8 runs of T).  Whole groups with C' a multiple of 8 (as
+  // every tensor-core handle has) load in 16-byte / T-element vectors: W is
+  // 16-byte aligned and (d*C' + c) a multiple of 8 for the forward image.
+  alignas(16) E w[8][T];
+  if (k0 + 8 <= K && Cp % 8 == 0) {
+    if (fwd) {
+      const uint4* src = reinterpret_cast<const uint4*>(W + (row * Cp + k0) * T);
+#pragma unroll
+      for (int v = 0; v < T; ++v) reinterpret_cast<uint4*>(&w[0][0])[v] = __ldg(src + v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const E* src = W + ((k0 + i) * Cp + row) * T;
+        if constexpr (T == 8) {
+          *reinterpret_cast<uint4*>(w[i]) = __ldg(reinterpret_cast<const uint4*>(src));
+        } else if constexpr (T == 4) {
+          *reinterpret_cast<uint2*>(w[i]) = __ldg(reinterpret_cast<const uint2*>(src));
+        } else if constexpr (T == 2) {
+          *reinterpret_cast<uint32_t*>(w[i]) = __ldg(reinterpret_cast<const unsigned int*>(src));
+        } else {
+          w[i][0] = src[0];
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t k = k0 + i;
+      const int64_t base = fwd ? (row * Cp + k) * T : (k * Cp + row) * T;
+#pragma unroll
+      for (int t = 0; t < T; ++t) w[i][t] = k < K ? W[base + t] : Elem<E>::from_f(0.f);
+    }
+  }
   float P[8][T];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int64_t k = k0 + i;
-    const int64_t base = fwd ? (row * Cp + k) * T : (k * Cp + row) * T;
     float v[T];
 #pragma unroll
-    for (int t = 0; t < T; ++t) v[t] = k < K ? Elem<E>::to_f(W[base + t]) : 0.f;
+    for (int t = 0; t < T; ++t) v[t] = Elem<E>::to_f(w[i][t]);
     G::dft(v, P[i]);
   }
   E* out = fwd ? wt_fwd : wt_bwd;
