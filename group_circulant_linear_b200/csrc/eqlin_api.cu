@@ -27,13 +27,17 @@ size_t elem_size(eqlin_dtype_t dt) { return dt == EQLIN_F32 ? 4 : 2; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Make the handle's device current for the duration of a call.
+// Make the handle's device current for the duration of a call.  The set is
+// unconditional: besides selecting the device it makes the device's primary
+// context current in this host thread, which a thread that has only selected
+// the device (an autograd worker, say) may not have yet, and which the
+// tensor-map encoding needs.
 struct DeviceGuard {
   int prev = -1;
   bool ok = true;
   explicit DeviceGuard(int dev) {
     if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
-    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    if (cudaSetDevice(dev) != cudaSuccess) ok = false;
   }
   ~DeviceGuard() {
     int cur = -1;

@@ -59,6 +59,9 @@ extern "C" eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t D
 
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EQLIN_ERR_CUDA;
+  // makes the device's primary context current in this host thread (the
+  // tensor-map encoding needs one; a thread may have selected the device only)
+  if (cudaSetDevice(dev) != cudaSuccess) return EQLIN_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return EQLIN_ERR_CUDA;
   // The partials of the largest token split this shape can use must fit.

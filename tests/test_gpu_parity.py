@@ -132,6 +132,39 @@ def test_back_to_back_dependencies():
         assert rel_err(k["x"], oracle.backward_dx(k["g1"], a["W"])) <= tol
 
 
+def test_calls_from_another_host_thread():
+    """A host thread other than the one that created the handle (an autograd
+    worker, for one) can call every entry point."""
+    import threading
+    T, Cp, Dp, N = 4, 64, 96, 300
+    inp = inputs.make_inputs(T, Cp, Dp, N, "bf16", seed=14)
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    torch.cuda.synchronize()
+    out, errs = {}, []
+
+    def worker():
+        try:
+            out["y"] = layer.forward(g["x"])
+            out["dx"] = layer.backward_dx(g["gy"])
+            out["dW"], out["db"] = layer.backward_dw(g["x"], g["gy"])
+            eqlin.set_weights(layer.h, g["W"], g["b"])
+            torch.cuda.synchronize()
+        except Exception as e:  # reported below, in the test's own thread
+            errs.append(repr(e))
+
+    th = threading.Thread(target=worker)
+    th.start()
+    th.join()
+    assert not errs, errs
+    assert eqlin.get_error(layer.h) == 0
+    tol = TOL["bf16"]
+    assert rel_err(out["y"].float().cpu(), oracle.forward(inp["x"], inp["W"], inp["b"])) <= tol
+    assert rel_err(out["dx"].float().cpu(), oracle.backward_dx(inp["gy"], inp["W"])) <= tol
+    dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
+    assert rel_err(out["dW"].cpu(), dW) <= tol and rel_err(out["db"].cpu(), db) <= tol
+
+
 def _roll(a: torch.Tensor, ch: int, T: int, r: int) -> torch.Tensor:
     N = a.shape[0]
     return torch.roll(a.reshape(N, ch, T), r, dims=2).reshape(N, ch * T).contiguous()
