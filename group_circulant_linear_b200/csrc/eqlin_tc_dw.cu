@@ -31,9 +31,10 @@
 //              main loop the A warps of both groups read the accumulators out
 //              of TMEM, each group half of the N columns
 //   warp 17    allocates TMEM; the warp runs the MMA loop and one lane issues
-// The raw ring (filled by TMA, freed once the transform has read a slot) and
-// the operand ring (filled by the transform, freed by the MMA commit) are
-// separate, so loads run ahead of the tensor core by the whole raw ring.
+// The raw ring (filled by TMA, freed once the transform has written the
+// stage's operands from it) and the operand ring (filled by the transform,
+// freed by the MMA commit) are separate, so loads run ahead of the tensor
+// core by the whole raw ring.
 // The per-chunk partial planes go to the handle's workspace as
 // [chunk][plane][N channel][M channel]; a second kernel sums the chunks in a
 // fixed order and applies the inverse DFT (deterministic, no atomics).  All
@@ -253,12 +254,6 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
           }
         }
       }
-      // the raw slot may be refilled by TMA (async proxy) once these generic
-      // reads are ordered before it
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&raw_empty[rs]);
-      if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
       uint32_t Pw[T][4];
       if (active) {
         if constexpr (T <= 4) {
@@ -321,9 +316,15 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
           }
         }
       }
+      // one generic->async proxy fence orders both this stage's reads of the
+      // raw slot (before its TMA refill) and its operand writes (before the MMA)
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&op_full[os]);
+      if (lane == 0) {
+        mbar_arrive(&raw_empty[rs]);
+        mbar_arrive(&op_full[os]);
+      }
+      if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
       if (++os == C::OP_STAGES) { os = 0; oph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
