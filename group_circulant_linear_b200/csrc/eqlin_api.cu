@@ -91,7 +91,7 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
   *out = nullptr;
   if (dtype != EQLIN_F32 && dtype != EQLIN_F16 && dtype != EQLIN_BF16) return EQLIN_ERR_INVALID_ARG;
   if (Cp < 1 || Dp < 1) return EQLIN_ERR_INVALID_ARG;
-  if (T != 1 && T != 2 && T != 4 && T != 8) return EQLIN_ERR_UNSUPPORTED;
+  if (T != 1 && T != 2 && T != 3 && T != 4 && T != 6 && T != 8) return EQLIN_ERR_UNSUPPORTED;
   if (Cp > 65536 || Dp > 65536) return EQLIN_ERR_UNSUPPORTED;
   const size_t e = elem_size(dtype);
   if ((Cp * T * e) % 16 || (Dp * T * e) % 16) return EQLIN_ERR_MISALIGNED;
@@ -119,7 +119,8 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
             cudaMalloc(&h.bias, (size_t)Dp * 4) == cudaSuccess &&
             cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
             cudaMalloc(&h.err, sizeof(int)) == cudaSuccess;
-  if (ok && dtype != EQLIN_F32) {
+  // tensor-core weight tiles only where a tensor-core pass exists (T | 8)
+  if (ok && dtype != EQLIN_F32 && (eqlin::tc_supported(h, false) || eqlin::tc_supported(h, true))) {
     h.bo_fwd = eqlin::tc_pick_bo(T, Dp);
     h.bo_bwd = eqlin::tc_pick_bo(T, Cp);
     const size_t nf = (size_t)eqlin::wtile_elems(T, h.bo_fwd, Dp, Cp);

@@ -40,13 +40,17 @@ template <> struct Elem<__nv_bfloat16> {
 };
 
 // --------------------------------------------------- group-axis plane tables
-// cos/sin of 2*pi*j/8; T in {1,2,4,8} reads entry (j * 8/T) mod 8.  The only
-// inexact entry is sqrt(2)/2 (T = 8), rounded once to float.
+// cos/sin of 2*pi*j/8 for T in {1,2,4,8} (entry j * 8/T), and of 2*pi*j/12
+// for T in {3,6} (entry j * 12/T).  The only inexact entries are sqrt(2)/2
+// (T = 8) and sqrt(3)/2 (T = 3, 6), each rounded once to float; the others
+// are 0, +-1/2 and +-1.
 #define EQLIN_RSQRT2 0.70710678118654752440f
+#define EQLIN_SQRT3_2 0.86602540378443864676f
 
 template <int T> struct Group {
-  static constexpr int nreal = (T == 1) ? 1 : 2;        // k = 0 and k = T/2
-  static constexpr int ncomplex = (T - nreal) / 2;      // k = 1 .. T/2-1
+  static_assert(8 % T == 0 || 12 % T == 0, "T in {1, 2, 3, 4, 6, 8}");
+  static constexpr int nreal = (T % 2) ? 1 : 2;         // k = 0, and k = T/2 for even T
+  static constexpr int ncomplex = (T - nreal) / 2;      // k = 1 .. ceil(T/2)-1
   static constexpr int planes = T;                      // real planes of the half spectrum
   // Real GEMM count R(T): one per real frequency, four per complex one.
   static constexpr int gemms = nreal + 4 * ncomplex;
@@ -57,9 +61,22 @@ template <int T> struct Group {
          : j == 4 ? -1.f : j == 5 ? -EQLIN_RSQRT2 : j == 6 ? 0.f : EQLIN_RSQRT2;
   }
   static __host__ __device__ __forceinline__ float sin8(int j) { return cos8(j - 2); }
+  static __host__ __device__ __forceinline__ float cos12(int j) {
+    j = ((j % 12) + 12) % 12;
+    return j == 0 ? 1.f : j == 1 ? EQLIN_SQRT3_2 : j == 2 ? 0.5f : j == 3 ? 0.f : j == 4 ? -0.5f
+         : j == 5 ? -EQLIN_SQRT3_2 : j == 6 ? -1.f : j == 7 ? -EQLIN_SQRT3_2 : j == 8 ? -0.5f
+         : j == 9 ? 0.f : j == 10 ? 0.5f : EQLIN_SQRT3_2;
+  }
+  static __host__ __device__ __forceinline__ float sin12(int j) { return cos12(j - 3); }
   // cos / sin of 2*pi*k*t/T
-  static __host__ __device__ __forceinline__ float c(int k, int t) { return cos8(k * t * (8 / T)); }
-  static __host__ __device__ __forceinline__ float s(int k, int t) { return sin8(k * t * (8 / T)); }
+  static __host__ __device__ __forceinline__ float c(int k, int t) {
+    if constexpr (8 % T == 0) return cos8(k * t * (8 / T));
+    else return cos12(k * t * (12 / T));
+  }
+  static __host__ __device__ __forceinline__ float s(int k, int t) {
+    if constexpr (8 % T == 0) return sin8(k * t * (8 / T));
+    else return sin12(k * t * (12 / T));
+  }
 
   // Forward real DFT of v[0..T) into planes P[0..T).
   static __host__ __device__ __forceinline__ void dft(const float* v, float* P) {
@@ -67,7 +84,7 @@ template <int T> struct Group {
 #pragma unroll
     for (int t = 0; t < T; ++t) a += v[t];
     P[0] = a;
-    if (T >= 2) {
+    if constexpr (T % 2 == 0) {
       float h = 0.f;
 #pragma unroll
       for (int t = 0; t < T; ++t) h += (t & 1) ? -v[t] : v[t];
@@ -93,7 +110,8 @@ template <int T> struct Group {
   static __host__ __device__ __forceinline__ void idft_scaled(const float* P, float add, float* v) {
     const float a = P[0] + add;
     if (T == 1) { v[0] = a; return; }
-    const float ep = a + P[1], em = a - P[1];      // even / odd s
+    // even T: + (-1)^s P1 (the k = T/2 plane); odd T has none
+    const float ep = (T % 2 == 0) ? a + P[1] : a, em = (T % 2 == 0) ? a - P[1] : a;
 #pragma unroll
     for (int s_ = 0; s_ < T; ++s_) {
       float acc = (s_ & 1) ? em : ep;
@@ -113,7 +131,7 @@ template <int T> struct Group {
 #pragma unroll
     for (int s_ = 0; s_ < T; ++s_) {
       float a = P[0];
-      if (T >= 2) a += (s_ & 1) ? -P[1] : P[1];
+      if constexpr (T % 2 == 0) a += (s_ & 1) ? -P[1] : P[1];
       float acc2 = 0.f;
 #pragma unroll
       for (int k = 1; k <= ncomplex; ++k) {
@@ -143,7 +161,7 @@ template <int T> struct Group {
 // input transform).  Other T use one width.
 constexpr int TC_BK = 16;
 __host__ __device__ constexpr int tc_planes(int T) {
-  return (T == 1 ? 1 : 2) + 3 * ((T - (T == 1 ? 1 : 2)) / 2);
+  return (T % 2 ? 1 : 2) + 3 * ((T - (T % 2 ? 1 : 2)) / 2);
 }
 inline int tc_pick_bo(int T, int64_t O) {
   if (T == 1) return 256;

@@ -183,7 +183,8 @@ pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __re
         } else if constexpr (T == 2) {
           *reinterpret_cast<uint32_t*>(w[i]) = __ldg(reinterpret_cast<const unsigned int*>(src));
         } else {
-          w[i][0] = src[0];
+#pragma unroll
+          for (int t = 0; t < T; ++t) w[i][t] = src[t];
         }
       }
     }
@@ -260,6 +261,8 @@ static cudaError_t pretransform_e(const Handle& h, const void* W, const void* b,
   switch (h.T) {
     case 1: return pretransform_t<1, E>(h, W, b, st);
     case 2: return pretransform_t<2, E>(h, W, b, st);
+    case 3: return pretransform_t<3, E>(h, W, b, st);
+    case 6: return pretransform_t<6, E>(h, W, b, st);
     case 4: return pretransform_t<4, E>(h, W, b, st);
     case 8: return pretransform_t<8, E>(h, W, b, st);
   }
@@ -404,6 +407,8 @@ static cudaError_t simt_apply_e(const Handle& h, bool bwd, const void* in, void*
   switch (h.T) {
     case 1: return simt_apply_t<1, E>(h, bwd, in, out, N, st);
     case 2: return simt_apply_t<2, E>(h, bwd, in, out, N, st);
+    case 3: return simt_apply_t<3, E>(h, bwd, in, out, N, st);
+    case 6: return simt_apply_t<6, E>(h, bwd, in, out, N, st);
     case 4: return simt_apply_t<4, E>(h, bwd, in, out, N, st);
     case 8: return simt_apply_t<8, E>(h, bwd, in, out, N, st);
   }
@@ -641,6 +646,8 @@ cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, con
   switch (h.T) {
     case 1: return dw_reduce_t<1>(h, splits, part, dbpart, dW, db, cd_layout, st);
     case 2: return dw_reduce_t<2>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 3: return dw_reduce_t<3>(h, splits, part, dbpart, dW, db, cd_layout, st);
+    case 6: return dw_reduce_t<6>(h, splits, part, dbpart, dW, db, cd_layout, st);
     case 4: return dw_reduce_t<4>(h, splits, part, dbpart, dW, db, cd_layout, st);
     case 8: return dw_reduce_t<8>(h, splits, part, dbpart, dW, db, cd_layout, st);
   }
@@ -672,6 +679,8 @@ static cudaError_t simt_dw_e(const Handle& h, const void* x, const void* gy, flo
   switch (h.T) {
     case 1: return simt_dw_t<1, E>(h, x, gy, dW, db, N, st);
     case 2: return simt_dw_t<2, E>(h, x, gy, dW, db, N, st);
+    case 3: return simt_dw_t<3, E>(h, x, gy, dW, db, N, st);
+    case 6: return simt_dw_t<6, E>(h, x, gy, dW, db, N, st);
     case 4: return simt_dw_t<4, E>(h, x, gy, dW, db, N, st);
     case 8: return simt_dw_t<8, E>(h, x, gy, dW, db, N, st);
   }

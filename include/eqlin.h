@@ -35,7 +35,10 @@
  *   that ran out) are recorded in the handle and read with eqlin_get_error()
  *   after the caller has synchronised the stream.
  * - N = 0 is a no-op that returns EQLIN_OK (dW and db are then zeroed).
- * - Supported T: 1, 2, 4, 8.  Other values give EQLIN_ERR_UNSUPPORTED.
+ * - Supported T: 1, 2, 3, 4, 6, 8.  Other values give EQLIN_ERR_UNSUPPORTED.
+ *   T = 3 and 6 (twiddles with sqrt(3)/2) run the FP32 SIMT kernels in every
+ *   dtype; the tensor-core kernels serve f16/bf16 for T = 1, 2, 4, 8.
+ *   eqlin_backward_dw_noalloc takes T = 1, 2, 4, 8 only.
  * - Nothing is thrown across the ABI; every call returns a status.
  * - A handle may be used from one host thread at a time.
  */

@@ -48,7 +48,8 @@ def test_status_strings():
 def test_create_rejects_bad_arguments_before_touching_cuda():
     L = eqlin.lib()
     out = ctypes.c_void_p()
-    assert L.eqlin_create(3, 16, 16, eqlin.F32, ctypes.byref(out)) == -2   # T = 3
+    assert L.eqlin_create(5, 16, 16, eqlin.F32, ctypes.byref(out)) == -2   # T = 5
+    assert L.eqlin_create(12, 16, 16, eqlin.F32, ctypes.byref(out)) == -2  # T = 12
     assert L.eqlin_create(16, 16, 16, eqlin.F32, ctypes.byref(out)) == -2  # T = 16
     assert L.eqlin_create(4, 0, 16, eqlin.F32, ctypes.byref(out)) == -1
     assert L.eqlin_create(4, 16, -1, eqlin.F32, ctypes.byref(out)) == -1

@@ -63,6 +63,8 @@ SMALL = [  # (T, C', D', N, dtype)
     (1, 64, 48, 200, "f32"), (1, 64, 48, 200, "bf16"),
     (8, 64, 16, 130, "bf16"), (2, 40, 72, 129, "bf16"),
     (4, 8, 8, 1, "f16"), (4, 200, 40, 131, "f16"),
+    # T = 3 and 6: sqrt(3)/2 twiddles, one real frequency for odd T (SIMT kernels)
+    (3, 64, 48, 257, "f32"), (6, 32, 40, 130, "f32"), (3, 40, 64, 300, "bf16"), (6, 48, 24, 200, "f16"),
 ]
 
 
@@ -130,6 +132,23 @@ def test_back_to_back_dependencies():
         assert rel_err(k["y2"], oracle.forward(k["y1"], b["W"], b["b"])) <= tol
         assert rel_err(k["g1"], oracle.backward_dx(k["y2"], b["W"])) <= tol
         assert rel_err(k["x"], oracle.backward_dx(k["g1"], a["W"])) <= tol
+
+
+@pytest.mark.parametrize("T,dt", [(3, "f32"), (6, "f32"), (3, "bf16"), (6, "f16")], ids=str)
+def test_odd_and_sixfold_groups_are_equivariant(T, dt):
+    """T = 3 and 6 run the SIMT kernels; a cyclic shift of the input's group
+    axis shifts the output's, and the backend says so."""
+    Cp, Dp, N = 16, 24, 150
+    inp = _dev(inputs.make_inputs(T, Cp, Dp, N, dt, seed=15))
+    layer = eqlin.EQLinear(inp["W"], inp["b"])
+    assert layer.h.backend() == "simt"
+    y = layer.forward(inp["x"])
+    tol = 1e-5 if dt == "f32" else TOL[dt]
+    for r in range(1, T):
+        yr = layer.forward(_roll(inp["x"], Cp, T, r))
+        assert rel_err(yr.float().cpu(), _roll(y, Dp, T, r).float().cpu()) <= tol
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
 
 
 def test_calls_from_another_host_thread():

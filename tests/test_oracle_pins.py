@@ -142,7 +142,7 @@ def pin_fft(impl):
 
 def pin_integer_exact(impl):
     rng = np.random.default_rng(5)
-    for T, Cp, Dp, N in [(4, 3, 2, 4), (2, 4, 3, 5), (8, 2, 2, 3), (3, 2, 3, 2)]:
+    for T, Cp, Dp, N in [(4, 3, 2, 4), (2, 4, 3, 5), (8, 2, 2, 3), (3, 2, 3, 2), (6, 2, 2, 3)]:
         x = rng.integers(-4, 5, (N, Cp * T))
         W = rng.integers(-4, 5, (Dp, Cp, T))
         b = rng.integers(-1, 2, Dp)
