@@ -16,7 +16,8 @@ HEADER = os.path.join(ROOT, "include", "eqlin.h")
 
 
 def declared_symbols():
-    src = open(HEADER).read()
+    with open(HEADER) as f:
+        src = f.read()
     return sorted(set(re.findall(r"EQLIN_API\s+[^;(]*?\b(eqlin_\w+)\s*\(", src)))
 
 

@@ -57,8 +57,13 @@ def test_two_rank_gradients_match_whole_batch():
     T, Cp, Dp, N = 4, 3, 2, 37
     world = 2
     port = _free_port()
-    out = mp.Manager().dict()
-    mp.spawn(_worker, args=(world, port, T, Cp, Dp, N, out), nprocs=world, join=True)
+    manager = mp.get_context("spawn").Manager()
+    try:
+        out = manager.dict()
+        mp.spawn(_worker, args=(world, port, T, Cp, Dp, N, out), nprocs=world, join=True)
+        out = dict(out)
+    finally:
+        manager.shutdown()
     inp = inputs.make_inputs(T, Cp, Dp, N, "f32", seed=5)
     y = oracle.forward(inp["x"], inp["W"], inp["b"])
     dx = oracle.backward_dx(inp["gy"], inp["W"])
