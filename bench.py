@@ -125,6 +125,31 @@ def oracle_data(layers, seed: int = 0):
     return data
 
 
+_RATES = {}
+
+
+def _oracle_rates(layers, data):
+    """The oracle's rates (dense-equivalent FLOP/s) for token rows and for
+    weight pairs, measured once per process on a probe that gives each of its
+    threads a few rows / pairs, as the samples will."""
+    import numpy as np
+
+    import oracle
+    L0, d0 = layers[0], data[0]
+    key = (L0.T, L0.Cp, L0.Dp, L0.N)
+    if key not in _RATES:
+        per_thread = 4 * oracle.threads()
+        probe = min(per_thread, L0.N)
+        t = time.perf_counter()
+        oracle.forward(d0["x"], d0["W"], d0["b"], rows=np.arange(probe))
+        row_rate = probe * 2 * L0.C * L0.D / max(time.perf_counter() - t, 1e-6)
+        t = time.perf_counter()
+        oracle.backward_dw(d0["x"], d0["gy"], L0.T, L0.Cp, L0.Dp, pairs=[[0, 0]] * per_thread, want_db=False)
+        dw_rate = per_thread * L0.T * 2 * L0.N * L0.T / max(time.perf_counter() - t, 1e-6)
+        _RATES[key] = (row_rate, dw_rate)
+    return _RATES[key]
+
+
 def oracle_sample(layers, data, budget_s: float, seed: int = 0):
     """Time the oracle on a bounded sample of every layer's fwd, dx and dW work.
 
@@ -133,17 +158,7 @@ def oracle_sample(layers, data, budget_s: float, seed: int = 0):
 
     import oracle
     oracle.build()
-    # calibrate the oracle's rates (dense-equivalent FLOP/s) on a probe that
-    # gives each of its threads a few rows / weight pairs, as the sample will
-    L0, d0 = layers[0], data[0]
-    per_thread = 4 * oracle.threads()
-    probe = min(per_thread, L0.N)
-    t = time.perf_counter()
-    oracle.forward(d0["x"], d0["W"], d0["b"], rows=np.arange(probe))
-    row_rate = probe * 2 * L0.C * L0.D / max(time.perf_counter() - t, 1e-6)
-    t = time.perf_counter()
-    oracle.backward_dw(d0["x"], d0["gy"], L0.T, L0.Cp, L0.Dp, pairs=[[0, 0]] * per_thread, want_db=False)
-    dw_rate = per_thread * L0.T * 2 * L0.N * L0.T / max(time.perf_counter() - t, 1e-6)
+    row_rate, dw_rate = _oracle_rates(layers, data)
     done, desc, t_total = 0, [], 0.0
     for L, d in zip(layers, data):
         share_s = budget_s / (len(layers) * len(L.passes))     # seconds per pass
