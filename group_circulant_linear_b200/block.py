@@ -102,7 +102,9 @@ class EQLinear(nn.Module):
 
     def sync_weights(self, W: torch.Tensor, b: torch.Tensor | None):
         """Run the weight transform if W or b changed since it last ran."""
-        key = (W.data_ptr(), W._version, None if b is None else (b.data_ptr(), b._version))
+        # the handle's identity too: a deep copy of the module gets a new,
+        # empty handle and must load its weights again
+        key = (id(self.h), W.data_ptr(), W._version, None if b is None else (b.data_ptr(), b._version))
         if key != self._seen:
             eqlin.set_weights(self.h, W.detach().to(self.dtype).contiguous(),
                               None if b is None else b.detach().to(self.dtype).contiguous())

@@ -122,6 +122,13 @@ class Handle:
     def backend(self) -> str:
         return lib().eqlin_backend_name(self._h).decode()
 
+    def __copy__(self):
+        raise TypeError("a Handle owns device buffers; use copy.deepcopy for a new handle of the same shape")
+
+    def __deepcopy__(self, memo):
+        # a new handle of the same shape; it holds no weights until set_weights
+        return Handle(self.T, self.Cp, self.Dp, self.dtype)
+
 
 # ------------------------------------------------------------------ the ABI
 

@@ -103,6 +103,23 @@ def test_eqlinear_rereads_weights_after_update():
 
 
 @pytest.mark.gpu
+def test_eqlinear_deepcopy_gets_its_own_handle():
+    import copy
+
+    from group_circulant_linear_b200.block import EQLinear
+    T, Cp, Dp, N = 4, 32, 32, 64
+    layer = EQLinear(Cp, Dp, T, dtype=torch.bfloat16, generator=torch.Generator().manual_seed(6))
+    x = inputs.make_inputs(T, Cp, Dp, N, "bf16", seed=16)["x"].cuda()
+    y = layer(x)
+    twin = copy.deepcopy(layer)
+    assert twin.h.ptr.value != layer.h.ptr.value
+    del layer                     # destroys only the original's handle
+    y2 = twin(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+
+
+@pytest.mark.gpu
 def test_block_against_fp32_dense_block_and_equivariance():
     from group_circulant_linear_b200.block import DenseEQViTBlock, EQViTBlock
     T, Cp, heads, B, L = 4, 32, 4, 2, 50
