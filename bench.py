@@ -8,9 +8,22 @@ shapes in bf16: fc1 768->3072 and fc2 3072->768 over 64 images x 197 tokens.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (launched by torch.distributed.run) every rank processes its own
-batch (weak scaling) and the dW/db gradients are summed over ranks with NCCL,
-the data-parallel exchange of the backward pass.  Rank 0 prints one JSON line.
+With N > 1 every rank processes its own batch (weak scaling) and the dW/db
+gradients are summed over ranks with NCCL, the data-parallel exchange of the
+backward pass.  Launched by torch.distributed.run, each rank reads its
+RANK / LOCAL_RANK / WORLD_SIZE from the environment; launched directly with
+--gpus N > 1, the script starts the N local ranks itself.  Rank 0 prints one
+JSON line.
+
+Regions timed with CUDA events on the launching streams:
+  * the headline: exactly K whole steps, nothing else in between;
+  * per kernel: each (layer, pass) call launched back to back on its own, for
+    the roofline of the dominant kernel and the per-call breakdown;
+  * sub-measurements on other workloads of the same path (the p4 FP16 forward
+    at EQ-ViT-B shapes, the EQ-Swin-T stage-1 step, the T=8 FP16 layer), each
+    with its own roofline fractions;
+  * end to end: the same step through the public API with the inputs copied
+    from pinned host memory and the results copied back every step.
 
 `--impl reference` times the CPU oracle (plain loops over the layer's
 definition, double precision) on a bounded sample of the same workload.
@@ -21,9 +34,12 @@ import argparse
 import hashlib
 import json
 import os
+import platform
+import socket
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -35,11 +51,11 @@ from group_circulant_linear_b200 import dp, inputs, workloads  # noqa: E402
 
 METRIC = "EQ-Linear p4 fwd+bwd TFLOP/s (dense-equiv) & fraction of tensor-pipe roofline"
 UNIT = "TFLOP/s"
-N_SETS = 3   # rotating input sets, together larger than the 126 MB L2
-REC_EVERY = 8   # timed steps per step with per-call events (kernel_ms, roofline)
+N_SETS = 3        # rotating input sets, together larger than the 126 MB L2
+KERNEL_REPS = 50  # back-to-back launches per (layer, pass) in the per-kernel region
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -48,7 +64,8 @@ def parse():
     ap.add_argument("--workload", default=workloads.DEFAULT_BENCH, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--no-sub", action="store_true", help="skip the sub-measurements")
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -67,50 +84,80 @@ def dense_flop_step(layers):
     return sum(L.dense_flop() * len(L.passes) for L in layers)
 
 
+def cpu_info() -> dict:
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """nvidia-smi samples of one GPU, read line by line on a background thread.
+
+    Samples are kept only while `active` is set (the timed regions); the
+    summary takes the samples drawn under load (power at least half of the
+    maximum seen) for the median SM clock and the throttle reasons."""
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device: int):
-        self.proc = None
+    def __init__(self, device: int, period_ms: int = 100):
+        self.rows, self.active, self.error = [], False, None
+        self.proc = self.thread = None
         try:
-            props = torch.cuda.get_device_properties(device)
-            gid = "GPU-" + str(props.uuid)
+            gid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
             gid = str(device)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", gid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+                 "-lms", str(period_ms), "-i", gid], stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                text=True, bufsize=1)
+        except Exception as e:  # reported in the summary
+            self.error = f"nvidia-smi did not start: {e}"
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
 
-    def stop(self) -> dict | None:
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except Exception:
-            self.proc.kill()
-            return None
-        rows = []
-        for line in out.strip().splitlines():
+    def _read(self):
+        for line in self.proc.stdout:
+            if not self.active:
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != len(self.FIELDS):
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+                self.rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:]))
             except ValueError:
                 continue
+
+    def stop(self) -> dict:
+        self.active = False
+        if self.proc is None:
+            return {"sm_mhz": None, "samples": 0, "note": self.error}
+        self.proc.terminate()
+        try:
+            _, err = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            err = ""
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        rows = list(self.rows)
         if not rows:
-            return None
+            return {"sm_mhz": None, "samples": 0,
+                    "note": "no nvidia-smi samples during the timed regions" + (f": {err.strip()[:200]}" if err else "")}
         pmax = max(r[2] for r in rows)
         loaded = [r for r in rows if r[2] >= 0.5 * pmax] or rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
+        reasons = sorted({self.REASONS[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
                 "reasons": reasons, "samples": len(loaded), "power_w_max": pmax}
 
@@ -206,13 +253,13 @@ def run_reference(args, layers, rank):
         "config": {"workload": args.workload,
                    "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N) for L in layers]},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": "per step: " + desc},
+                         "sample": "per step: " + desc, **cpu_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-# ----------------------------------------------------------------- our arm
+# ------------------------------------------------------------- roofline
 def kernel_src_sha(name: str) -> str:
     path = os.path.join(ROOT, "group_circulant_linear_b200", "csrc", name)
     with open(path, "rb") as f:
@@ -234,9 +281,134 @@ def profiled_traffic(kernel_key: str):
     return None
 
 
-def main():
-    args = parse()
+def pass_work(L, kind):
+    """(actual FLOP, algorithmic bytes) of one call of a pass."""
+    if kind == "set_weights":
+        return 0, L.Dp * L.Cp * L.T * 2 * 2
+    return L.actual_flop(), (L.bytes_dw() if kind == "dw" else L.bytes_fwd())
+
+
+def roofline_of(L, kind, us, pk):
+    """Roofline of one call of `kind` on layer L that took `us` microseconds.
+
+    The bound is the resource the call's arithmetic intensity points at:
+    tensor when its FLOP per algorithmic byte reach half the measured ridge
+    (dense bf16 peak / copy bandwidth), else HBM.  Calls timed in sub-second
+    regions use the burst tensor peak (FP16 and BF16 have the same nominal
+    rate).  `frac_roofline` = max(FLOP / tensor peak, bytes / HBM) / time."""
+    flop, byt = pass_work(L, kind)
+    t = us * 1e-6
+    tens = pk["bf16"] * 1e12
+    hbm = pk["hbm_gbs"] * 1e9
+    r = {"us": round(us, 2), "tflops": flop / t / 1e12 if flop else 0.0, "gbs": byt / t / 1e9,
+         "frac_tensor": flop / t / tens if flop else 0.0, "frac_hbm": byt / t / hbm,
+         "frac_roofline": max(flop / tens, byt / hbm) / t}
+    ridge = tens / hbm
+    if flop and flop / byt >= ridge / 2:
+        r.update(bound="tensor", achieved=r["tflops"], peak=pk["bf16"], unit="TFLOP/s", frac=r["frac_tensor"])
+    else:
+        r.update(bound="hbm", achieved=r["gbs"], peak=pk["hbm_gbs"], unit="GB/s", frac=r["frac_hbm"])
+    r["intensity_flop_per_byte"] = flop / byt
+    return r
+
+
+# ----------------------------------------------------------------- our arm
+class Layers:
+    """Device state of a workload's layers: handles, weights, rotating input sets, outputs."""
+
+    def __init__(self, layers, dev, rank, seed_base=0):
+        from group_circulant_linear_b200 import eqlin
+        self.eqlin = eqlin
+        self.layers = layers
+        self.st = []
+        for li, L in enumerate(layers):
+            dt = inputs.DTYPES[L.dtype]
+            w = inputs.make_inputs(L.T, L.Cp, L.Dp, 1, L.dtype, seed=seed_base + 1000 + li, with_gy=False,
+                                   device=dev)
+            sets = [inputs.make_inputs(L.T, L.Cp, L.Dp, L.N, L.dtype, seed=seed_base + 17 * rank + 100 * li + s,
+                                       with_gy=("dx" in L.passes or "dw" in L.passes), device=dev)
+                    for s in range(N_SETS)]
+            h = eqlin.create(L.T, L.Cp, L.Dp, dt)
+            self.st.append(dict(L=L, h=h, W=w["W"], b=w["b"], sets=sets,
+                                y=torch.empty((L.N, L.D), dtype=dt, device=dev),
+                                dx=torch.empty((L.N, L.C), dtype=dt, device=dev),
+                                dW=torch.empty((L.Dp, L.Cp, L.T), dtype=torch.float32, device=dev),
+                                db=torch.empty((L.Dp,), dtype=torch.float32, device=dev)))
+
+    def set_bytes(self):
+        return sum(sum(t.numel() * t.element_size() for t in s["sets"][0].values()) for s in self.st)
+
+    def call(self, s, kind, i, stream=None):
+        e, inp = self.eqlin, s["sets"][i % N_SETS]
+        if kind == "set_weights":
+            e.set_weights(s["h"], s["W"], s["b"], stream)
+        elif kind == "fwd":
+            e.forward(s["h"], inp["x"], s["y"], stream)
+        elif kind == "dx":
+            e.backward_dx(s["h"], inp["gy"], s["dx"], stream)
+        else:
+            e.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"], stream)
+
+    def errors(self):
+        return [self.eqlin.get_error(s["h"]) for s in self.st]
+
+    def close(self):
+        for s in self.st:
+            s["h"].close()
+
+
+def time_calls(state, li, kind, reps, stream):
+    """Average microseconds of one (layer, pass) call, `reps` launches back to
+    back between two events on the launching stream (inputs rotate)."""
+    s = state.st[li]
+    for i in range(3):
+        state.call(s, kind, i, stream)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(reps):
+        state.call(s, kind, i, stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps * 1e3
+
+
+def sub_measurements(dev, pk, reps):
+    """The same path on other workload shapes, each call timed on its own."""
+    out = {}
+    vit_b_f16 = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd",))
+                 for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
+    t8 = [L for L in workloads.WORKLOADS["cyclic-sweep-fwdbwd"] if L.T == 8 and L.dtype == "f16"]
+    subs = {
+        "p4 FP16 forward, EQ-ViT-B MLP shapes": vit_b_f16,
+        "EQ-Swin-T stage-1 step (f16)": workloads.WORKLOADS["eq-swin-t-s1-f16-fwdbwd"],
+        "cyclic T=8 f16 layer": t8,
+    }
+    stream = torch.cuda.current_stream()
+    for name, layers in subs.items():
+        state = Layers(layers, dev, 0, seed_base=5000)
+        rows, tot_us, dense = [], 0.0, 0
+        for li, L in enumerate(layers):
+            for kind in L.passes:
+                us = time_calls(state, li, kind, reps, stream)
+                rows.append({"layer": L.name, "pass": kind, **roofline_of(L, kind, us, pk)})
+                tot_us += us
+                dense += L.dense_flop()
+        assert all(e == 0 for e in state.errors()), f"device-side timeout in {name}"
+        state.close()
+        del state
+        torch.cuda.empty_cache()
+        out[name] = {"calls": rows, "dense_tflops": dense / (tot_us * 1e-6) / 1e12,
+                     "us_sum": round(tot_us, 2)}
+    return out
+
+
+def main(argv=None):
+    args = parse(argv)
     layers = workloads.WORKLOADS[args.workload]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "ours":
+        launch_local(args.gpus, argv if argv is not None else sys.argv[1:])
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -248,27 +420,12 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    from group_circulant_linear_b200 import eqlin
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-
-    # ------------------------------------------------------------ state
-    st = []
-    for li, L in enumerate(layers):
-        dt = inputs.DTYPES[L.dtype]
-        w = inputs.make_inputs(L.T, L.Cp, L.Dp, 1, L.dtype, seed=1000 + li, with_gy=False, device=dev)
-        sets = [inputs.make_inputs(L.T, L.Cp, L.Dp, L.N, L.dtype, seed=17 * rank + 100 * li + s,
-                                   device=dev) for s in range(N_SETS)]
-        h = eqlin.create(L.T, L.Cp, L.Dp, dt)
-        st.append(dict(L=L, h=h, W=w["W"], b=w["b"], sets=sets,
-                       y=torch.empty((L.N, L.D), dtype=dt, device=dev),
-                       dx=torch.empty((L.N, L.C), dtype=dt, device=dev),
-                       dW=torch.empty((L.Dp, L.Cp, L.T), dtype=torch.float32, device=dev),
-                       db=torch.empty((L.Dp,), dtype=torch.float32, device=dev)))
-
-    kinds = ("set_weights", "fwd", "dx", "dw")
-    ev_log = []   # (layer index, kind, start event, end event) during the timed region
+    state = Layers(layers, dev, rank)
+    eqlin = state.eqlin
+    st = state.st
 
     # A layer's dW/db and its dx read the same inputs and write nothing the
     # other reads, so dW/db runs on a second stream: its CTAs take the SMs
@@ -276,31 +433,13 @@ def main():
     # before each step ends (and before an all-reduce of dW/db).
     side = torch.cuda.Stream(device=dev)
 
-    def step(i, record=False):
-        for li, s in enumerate(st):
-            inp = s["sets"][i % N_SETS]
-            calls = (
-                ("set_weights", lambda: eqlin.set_weights(s["h"], s["W"], s["b"])),
-                ("fwd", lambda: eqlin.forward(s["h"], inp["x"], s["y"])),
-                ("dx", lambda: eqlin.backward_dx(s["h"], inp["gy"], s["dx"])),
-                ("dw", lambda: eqlin.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"])),
-            )
-            if record:
-                # every call on the main stream, one after another, each
-                # between two events: the per-call times
-                for kind, fn in calls:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    fn()
-                    e1.record(stream)
-                    ev_log.append((li, kind, e0, e1))
-            else:
-                calls[0][1]()
-                calls[1][1]()
-                side.wait_stream(stream)
-                calls[2][1]()
-                eqlin.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"], stream=side)
+    def step(i):
+        for s in st:
+            state.call(s, "set_weights", i)
+            state.call(s, "fwd", i)
+            side.wait_stream(stream)
+            state.call(s, "dx", i)
+            state.call(s, "dw", i, stream=side)
             if dist:
                 stream.wait_stream(side)
                 dp.allreduce_grads((s["dW"], s["db"]))
@@ -311,6 +450,7 @@ def main():
             torch.distributed.barrier()
 
     clocks = ClockSampler(local)
+    clocks.active = True
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -320,62 +460,41 @@ def main():
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    # per-call events on every REC_EVERY-th step only: an event between two
-    # kernels keeps the second from starting its prologue under the first's tail
     for i in range(args.steps):
-        step(i, record=(i % REC_EVERY == 0))
+        step(i)
     t1.record(stream)
     torch.cuda.synchronize()
     launches = eqlin.launch_count() - n0
     barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     if dist:
         tt = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
         ms = float(tt.item())
-    for s in st:
-        assert eqlin.get_error(s["h"]) == 0, "device-side timeout in the timed region"
+    assert all(e == 0 for e in state.errors()), "device-side timeout in the timed region"
     ms_per_step = ms / args.steps
     flop_step = dense_flop_step(layers)
     value = flop_step * world / (ms_per_step * 1e-3) / 1e12
 
     # ---------------------------------------------- per-kernel roofline
-    per = {}
-    for li, kind, e0, e1 in ev_log:
-        per.setdefault((li, kind), []).append(e0.elapsed_time(e1))
-    tot = {k: sum(v) for k, v in per.items()}
     pk = peaks()
-    dom = max(tot, key=tot.get)
+    per = {}
+    for li, L in enumerate(layers):
+        for kind in ("set_weights",) + tuple(L.passes):
+            per[(li, kind)] = time_calls(state, li, kind, KERNEL_REPS, stream)
+    clk = clocks.stop()
+    assert all(e == 0 for e in state.errors()), "device-side timeout in the per-kernel region"
+    dom = max(per, key=per.get)
     Ld = layers[dom[0]]
-    avg_ms = statistics.mean(per[dom])
+    roof = roofline_of(Ld, dom[1], per[dom], pk)
     kernel_of = {"fwd": "tc_apply", "dx": "tc_apply", "dw": "dw", "set_weights": "pretransform"}
-    if dom[1] in ("fwd", "dx", "dw"):
-        # the bound is the resource the call's arithmetic intensity points at:
-        # tensor when its FLOP per algorithmic byte exceed the measured ridge
-        flop = Ld.actual_flop()
-        byt = Ld.bytes_dw() if dom[1] == "dw" else Ld.bytes_fwd()
-        ridge = pk["bf16_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-        if flop / byt >= ridge / 2:
-            achieved = flop / (avg_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                    "frac": achieved / pk["bf16_sustained"],
-                    "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
-        else:
-            achieved = byt / (avg_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / pk["hbm_gbs"], "peak_kind": f"{pk['source']} HBM copy"}
-        roof["intensity_flop_per_byte"] = flop / byt
-    else:
-        byt = Ld.Dp * Ld.Cp * Ld.T * 2 * 2
-        achieved = byt / (avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "peak_kind": f"{pk['source']} HBM copy"}
     key = f"{kernel_of[dom[1]]}:{Ld.name}:{dom[1]}"
     roof["kernel"] = key
+    roof["peak_kind"] = (f"{pk['source']} " + ("bf16 dense, burst (call timed in a sub-second region)"
+                                               if roof["bound"] == "tensor" else "HBM copy"))
     roof["traffic"] = profiled_traffic(key)
-    breakdown = {f"{layers[li].name}/{kind}": round(statistics.mean(v) * 1e3, 2) for (li, kind), v in per.items()}
+    breakdown = {f"{layers[li].name}/{kind}": round(us, 2) for (li, kind), us in per.items()}
 
     # ---------------------------------------------------------- e2e
     e2e = None
@@ -390,6 +509,12 @@ def main():
         dbuf = [{k: torch.empty_like(s["sets"][0][k]) for k in ("x", "gy")} for s in st]
         h2d = sum(host[i][k].numel() * host[i][k].element_size() for i in range(len(st)) for k in ("x", "gy", "W", "b"))
         d2h = sum(host[i][k].numel() * host[i][k].element_size() for i in range(len(st)) for k in ("y", "dx", "dW", "db"))
+        # host->device copies and kernels on the main streams, device->host
+        # copies of each layer's results on a third stream, so that they overlap
+        # the next layer's uploads and kernels; a layer's outputs are
+        # overwritten (next step) only after its copies have run
+        d2h_stream = torch.cuda.Stream(device=dev)
+        copied = [None] * len(st)
 
         def e2e_step():
             for i, s in enumerate(st):
@@ -398,6 +523,8 @@ def main():
                 db_["gy"].copy_(hb["gy"], non_blocking=True)
                 s["W"].copy_(hb["W"], non_blocking=True)
                 s["b"].copy_(hb["b"], non_blocking=True)
+                if copied[i] is not None:
+                    stream.wait_event(copied[i])
                 eqlin.set_weights(s["h"], s["W"], s["b"])
                 eqlin.forward(s["h"], db_["x"], s["y"])
                 side.wait_stream(stream)
@@ -406,8 +533,12 @@ def main():
                 stream.wait_stream(side)
                 if dist:
                     dp.allreduce_grads((s["dW"], s["db"]))
-                for k in ("y", "dx", "dW", "db"):
-                    hb[k].copy_(s[k], non_blocking=True)
+                d2h_stream.wait_stream(stream)
+                with torch.cuda.stream(d2h_stream):
+                    for k in ("y", "dx", "dW", "db"):
+                        hb[k].copy_(s[k], non_blocking=True)
+                    copied[i] = torch.cuda.Event()
+                    copied[i].record(d2h_stream)
 
         ke = max(3, min(args.steps, 30))
         for _ in range(3):
@@ -419,6 +550,7 @@ def main():
         a.record(stream)
         for _ in range(ke):
             e2e_step()
+        stream.wait_stream(d2h_stream)      # the last results are on the host
         b.record(stream)
         torch.cuda.synchronize()
         ems = a.elapsed_time(b) / ke
@@ -429,45 +561,79 @@ def main():
         e2e = {"value": flop_step * world / (ems * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
+    set_bytes = state.set_bytes()
+    config = {
+        "workload": args.workload,
+        "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes)) for L in layers],
+        "step": "per layer: set_weights (weight DFT) + forward + dx + dW/db, dW/db on a second stream "
+                "beside dx" + (" + NCCL all-reduce of dW/db" if dist else ""),
+        "tokens_per_gpu": layers[0].N,
+        "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
+              f"({N_SETS * set_bytes / 1e6:.0f} MB > 126 MB L2)",
+        "actual_tflops": sum(L.actual_flop() * len(L.passes) for L in layers) * world
+                         / (ms_per_step * 1e-3) / 1e12,
+        "kernel_us": breakdown,
+        "kernel_us_sampling": f"CUDA events around {KERNEL_REPS} back-to-back launches of each call, "
+                              "after the headline region",
+    }
+    state.close()
+    del state, st
+    torch.cuda.empty_cache()
+
+    sub = None
+    if rank == 0 and not args.no_sub:
+        sub = sub_measurements(dev, pk, KERNEL_REPS)
+
     # ---------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, secs, threads, desc = oracle_sample(layers, oracle_data(layers), budget_s=12.0)
         cpu = {"value": f / secs / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc, "seconds": secs}
+               "sample": desc, "seconds": secs, **cpu_info()}
 
     if rank == 0:
-        set_bytes = sum(sum(t.numel() * t.element_size() for t in s["sets"][0].values()) for s in st)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": layers[0].dtype, "data": "synthetic",
-            "config": {
-                "workload": args.workload,
-                "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes))
-                           for L in layers],
-                "step": "per layer: set_weights (weight DFT) + forward + dx + dW/db, dW/db on a second "
-                        "stream beside dx"
-                        + (" + NCCL all-reduce of dW/db" if dist else ""),
-                "tokens_per_gpu": layers[0].N,
-                "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
-                      f"({N_SETS * set_bytes / 1e6:.0f} MB > 126 MB L2)",
-                "actual_tflops": sum(L.actual_flop() * len(L.passes) for L in layers) * world
-                                 / (ms_per_step * 1e-3) / 1e12,
-                "kernel_ms": breakdown,
-                "kernel_ms_sampling": f"CUDA events around each call on every {REC_EVERY}th timed step",
-            },
+            "config": config,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
+            "sub": sub,
         }
         print(json.dumps(line), flush=True)
-    for s in st:
-        s["h"].close()
     if dist:
         torch.distributed.destroy_process_group()
+
+
+# ----------------------------------------------------- local multi-rank launch
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def rank_env(rank: int, world: int, port: int) -> dict:
+    """Environment of local rank `rank` of `world` on this node (torchrun's variables)."""
+    return {"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+            "LOCAL_WORLD_SIZE": str(world), "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)}
+
+
+def _rank_entry(rank, world, port, target, argv):
+    os.environ.update(rank_env(rank, world, port))
+    target(argv)
+
+
+def launch_local(world: int, argv, target=None):
+    """Start `world` local ranks (one process per GPU) and wait for them; a
+    rank that fails makes this raise."""
+    import torch.multiprocessing as mp
+    port = free_port()
+    mp.start_processes(_rank_entry, args=(world, port, target or main, list(argv)), nprocs=world,
+                       join=True, start_method="spawn")
 
 
 if __name__ == "__main__":

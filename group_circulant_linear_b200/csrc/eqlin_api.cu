@@ -5,8 +5,12 @@
 // eqlin_get_error (which reads the device error word) and eqlin_destroy.
 #include <stdlib.h>
 #include <string.h>
+#include <stdio.h>
 #include <atomic>
+#include <mutex>
 #include <new>
+#include <set>
+#include <utility>
 
 #include "eqlin_internal.cuh"
 
@@ -15,6 +19,32 @@ using eqlin::Handle;
 namespace eqlin {
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({kernel, dev});
+  return e;
+}
+
+void* tensor_map_encoder() {
+  // function-local static: initialised once, thread-safe
+  static void* const fn = []() -> void* {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return ptr;
+    return nullptr;
+  }();
+  return fn;
+}
 }  // namespace eqlin
 
 struct eqlin_handle {
@@ -136,9 +166,10 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
     delete hh;
     return EQLIN_ERR_OOM;
   }
-  h.backend = (dtype == EQLIN_F32) ? "simt" : (eqlin::tc_supported(h, false) ? "tcgen05" : "simt");
   h.need_simt_fwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, false);
   h.need_simt_bwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, true);
+  snprintf(h.backend, sizeof(h.backend), "fwd=%s dx=%s dw=%s", h.need_simt_fwd ? "simt" : "tcgen05",
+           h.need_simt_bwd ? "simt" : "tcgen05", eqlin::tc_dw_supported(h) ? "tcgen05" : "simt");
   *out = hh;
   return EQLIN_OK;
 }

@@ -216,7 +216,8 @@ struct Handle {
   size_t ws_bytes = 0;
   int* err = nullptr;             // device error word
   uint32_t wait_limit = 0;        // 0 = default
-  const char* backend = "simt";
+  // kernel family of each pass, "fwd=<k> dx=<k> dw=<k>" (<k>: tcgen05 or simt)
+  char backend[48] = "fwd=simt dx=simt dw=simt";
 };
 
 // Device error codes written into Handle::err (first writer wins).
@@ -227,6 +228,14 @@ constexpr uint32_t kDefaultWaitLimit = 0xFFFFFFFFu;
 
 // Count kernels enqueued by this library (reported by eqlin_launch_count).
 void count_launches(int n);
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to the device's context, so it is set once
+// per (kernel, device) pair in this process; safe to call from any host thread.
+cudaError_t set_smem_limit(const void* kernel, int bytes);
+
+// cuTensorMapEncodeTiled from the driver, looked up once (nullptr if absent).
+void* tensor_map_encoder();
 
 // ------------------------------------------- programmatic dependent launch
 // Every kernel of this library is launched with programmatic stream

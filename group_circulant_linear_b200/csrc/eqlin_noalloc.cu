@@ -10,10 +10,13 @@
 // sums in the fixed-size device array below instead of an allocated workspace.
 //
 // The array is a file-scope __device__ object: the CUDA runtime reserves it on
-// a device when this module is first loaded there and holds it until the
-// process exits.  Host code may not use its name as a device address, so the
-// address is looked up with cudaGetSymbolAddress, once per device, with that
-// device current, the first time the entry point runs on it.
+// a device when this module's device code is loaded there and holds it until
+// the process exits.  Module loading is lazy, so that happens at the first
+// call on each device -- inside cudaGetSymbolAddress, which this file calls
+// once per device, with that device current, to turn the host-side stand-in
+// `g_dw_scratch` into the array's device address.  A device without room for
+// the array makes that lookup fail with cudaErrorMemoryAllocation, reported
+// as EQLIN_ERR_OOM.
 #include <mutex>
 
 #include "eqlin_internal.cuh"
@@ -75,7 +78,13 @@ extern "C" eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t D
   }
 
   unsigned char* scratch = nullptr;
-  if (scratch_address(dev, &scratch) != cudaSuccess) return EQLIN_ERR_CUDA;
+  {
+    const cudaError_t e = scratch_address(dev, &scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();   // a failed lazy load leaves no sticky error behind
+      return e == cudaErrorMemoryAllocation ? EQLIN_ERR_OOM : EQLIN_ERR_CUDA;
+    }
+  }
 
   eqlin::Handle h;                       // a description of the call; owns nothing
   h.T = T;

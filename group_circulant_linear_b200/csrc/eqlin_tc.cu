@@ -590,15 +590,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
 
 // ------------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
 template <int T, int BO, typename E>
@@ -646,12 +638,9 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
 
-  static bool attr_set = false;   // per template instance
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_apply_kernel<T, BO, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+  {
+    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;

@@ -547,15 +547,8 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
-  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  if (!enc) {
-    cudaDriverEntryPointQueryResult q;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return cudaErrorNotSupported;
-    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+  const auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   // N-side box: the largest power-of-two width <= 256 elements that divides BC * T
@@ -577,12 +570,9 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
       return cudaErrorInvalidValue;
   }
   p.nb_box = nb_box;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_dw_kernel<T, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+  {
+    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(tc_dw_kernel<T, E>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const unsigned grid = (unsigned)(pl.n_mt * pl.n_nt * pl.splits);
   cudaError_t e = launch_pdl(tc_dw_kernel<T, E>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, map_m, map_n, p);

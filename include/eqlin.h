@@ -66,7 +66,7 @@ typedef enum {
 typedef enum {
     EQLIN_OK = 0,
     EQLIN_ERR_INVALID_ARG = -1,  /* NULL handle/pointer, negative size, bad dtype */
-    EQLIN_ERR_UNSUPPORTED = -2,  /* T not in {1,2,4,8}, or a size beyond the limits */
+    EQLIN_ERR_UNSUPPORTED = -2,  /* T not in {1,2,3,4,6,8}, or a size beyond the limits */
     EQLIN_ERR_MISALIGNED = -3,   /* pointer or row not 16-byte aligned */
     EQLIN_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed */
     EQLIN_ERR_NO_WEIGHTS = -5,   /* forward/backward before eqlin_set_weights */
@@ -132,20 +132,24 @@ EQLIN_API eqlin_status_t eqlin_backward_dw(eqlin_t h, const void *x, const void 
  * NULL), computed by the same tensor-core kernels.  f16 and bf16 only
  * (EQLIN_ERR_UNSUPPORTED for f32).
  *
- * Scratch: a fixed 64 MiB device array inside the library, reserved on a
- * device when the library's code first loads there and held until the
- * process exits.  A shape whose per-chunk partial sums would not fit returns
- * EQLIN_ERR_UNSUPPORTED (the need is splits * (T*C'*D' + D') * 4 bytes, with
- * up to one token split per SM for a single 128 x 128 channel tile; e.g. p4
- * with C' = D' = 1024 fits, C' = D' = 2048 does not).
- * - The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Scratch: a fixed 64 MiB device array inside the library, held on a device
+ * until the process exits.  A shape whose per-chunk partial sums would not fit
+ * returns EQLIN_ERR_UNSUPPORTED (the need is splits * (T*C'*D' + D') * 4
+ * bytes, with up to one token split per SM for a single 128 x 128 channel
+ * tile; e.g. p4 with C' = D' = 1024 fits, C' = D' = 2048 does not).
+ * - The CUDA runtime loads the library's device code on a device lazily, so
+ *   the array is reserved by the FIRST call on each device (which also looks
+ *   up its device address with cudaGetSymbolAddress).  Make that first call
+ *   at start-up -- before the caller's own allocator takes the device's
+ *   memory, and before any stream capture.  If the device has no room for the
+ *   array then, that call returns EQLIN_ERR_OOM and computes nothing; a later
+ *   call tries again.
  * - Every call on a device shares the array, so calls that may overlap on
  *   the GPU (different streams, or concurrent host threads) race and give
  *   wrong results: order them on one stream.
  * - A device-side wait that runs out (only if the GPU stalls for seconds)
  *   leaves dW and db undefined; there is no handle to report it through.
- * The call itself allocates nothing and frees nothing.
+ * After that first call, the call allocates nothing and frees nothing.
  */
 EQLIN_API eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t Dp,
                                                    eqlin_dtype_t dtype, const void *x,
@@ -168,8 +172,13 @@ EQLIN_API eqlin_status_t eqlin_get_error(eqlin_t h);
 EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
 
 /*
- * Which kernel family serves each call of this handle, as a short string
- * (e.g. "tcgen05" or "simt"); for logging and tests.
+ * Which kernel family serves each pass of this handle, as
+ * "fwd=<k> dx=<k> dw=<k>", where <k> is "tcgen05" (the tensor-core kernels)
+ * or "simt" (the FP32 CUDA-core kernels).  f32 handles run simt for every
+ * pass.  f16/bf16 handles run tcgen05 except where the shape rules it out:
+ * T = 3 or 6 (all passes), or a forward (dx) whose K = C' (D') is not a
+ * multiple of 8 -- the row pitch of that pass's weight tiles would not be a
+ * TMA stride.  For logging and tests; the string lives as long as the handle.
  */
 EQLIN_API const char *eqlin_backend_name(eqlin_t h);
 

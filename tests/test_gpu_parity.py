@@ -4,11 +4,18 @@ Tolerances (relative Frobenius norm of the difference, i.e. RMS(err)/RMS(ref)):
 FP32 1e-5; FP16/BF16 with FP32 accumulation 2e-2.  Integer-valued inputs
 whose every intermediate is exactly representable must match bit for bit
 (T in {1, 2, 4}: the p4 and T=2 transforms use only +-1 and +-1/2, +-1/4).
+Every comparison records the error it achieved (tests/_parity.py).
 
-Small cases span several 128-token tiles with a ragged tail; full-size cases
-use the benchmark's shapes and launch path and compare sampled rows (forward,
-dx) and sampled (d, c) weight pairs (dW) against the oracle, plus the
-equivariance property on the whole output.
+Coverage:
+* small cases that span several 128-token tiles with a ragged tail;
+* bit-exact integer cases, including ones whose persistent grid runs three
+  or more output tiles per CTA (accumulator double-buffer phase flips, ring
+  wrap-around) and dW splits of many token stages;
+* every full-size workload in the benchmark's launch path: the EQ-ViT-S,
+  EQ-ViT-B and EQ-Swin-T layers compared on every output element (y, dx, dW,
+  db); the cyclic sweep on one token row of every 128-token tile and on
+  sampled (d, c) pairs of every 128 x 128 weight block; plus the
+  equivariance property on the whole output.
 """
 from __future__ import annotations
 
@@ -17,18 +24,10 @@ import pytest
 import torch
 
 import oracle
+from _parity import TOL, Accum, check, check_exact, finish
 from group_circulant_linear_b200 import eqlin, inputs, workloads
 
 pytestmark = pytest.mark.gpu
-
-TOL = {"f32": 1e-5, "f16": 2e-2, "bf16": 2e-2}
-
-
-def rel_err(out, ref) -> float:
-    out = np.asarray(out, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    den = np.linalg.norm(ref)
-    return float(np.linalg.norm(out - ref) / (den if den > 0 else 1.0))
 
 
 def _dev(d):
@@ -76,16 +75,31 @@ def test_small_parity(T, Cp, Dp, N, dt):
     dx = oracle.backward_dx(inp["gy"], inp["W"])
     dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
     tol = TOL[dt]
-    assert rel_err(out["y"], y) <= tol
-    assert rel_err(out["dx"], dx) <= tol
-    assert rel_err(out["dW"], dW) <= tol
-    assert rel_err(out["db"], db) <= tol
+    tag = f"small T={T} C'={Cp} D'={Dp} N={N} {dt}"
+    check(f"{tag} y", out["y"], y, tol)
+    check(f"{tag} dx", out["dx"], dx, tol)
+    check(f"{tag} dW", out["dW"], dW, tol)
+    check(f"{tag} db", out["db"], db, tol)
 
 
-EXACT = [  # (T, C', D', N, dtype, amp): every intermediate exactly representable
+# (T, C', D', N, dtype, amp): integer inputs in [-amp, amp] whose every
+# intermediate is exactly representable, so the result must equal the
+# oracle's exactly.  Bounds: y and dx are at most K*T*amp^2 + 1 in magnitude
+# (K = C' or D'), below 2^11 for f16 and 2^8 for bf16; the transformed
+# operands at most T*amp; every dW partial sum at most N*(T*amp)^2 <= 2^24,
+# exact in the FP32 accumulator.
+EXACT = [
     (4, 64, 64, 1024, "f32", 4), (2, 64, 48, 515, "f32", 4), (1, 32, 64, 300, "f32", 4),
     (4, 16, 16, 700, "f16", 4), (2, 16, 16, 300, "f16", 4), (4, 16, 8, 129, "f16", 4),
     (4, 8, 8, 400, "bf16", 2), (2, 8, 8, 200, "bf16", 2),
+    # 512 token tiles: 3-4 output tiles per persistent CTA of the forward and
+    # dx kernels, the dW token split over 147 chunks of 28 stages each
+    (4, 16, 16, 65536, "f16", 2),        # BO = 32 both ways (double-buffered accumulator)
+    (4, 16, 128, 65536, "f16", 2),       # forward BO = 128 (single accumulator), dx BO = 32
+    (4, 16, 96, 65536, "f16", 2),        # forward BO = 96
+    (4, 128, 16, 65536, "f16", 1),       # dx BO = 128, dW with c on the MMA's M side
+    (2, 16, 16, 65536, "f16", 2), (1, 16, 32, 65536, "f16", 2),
+    (4, 8, 8, 65536, "bf16", 2),
 ]
 
 
@@ -96,10 +110,11 @@ def test_integer_inputs_bit_exact(T, Cp, Dp, N, dt, amp):
     y = oracle.forward(inp["x"], inp["W"], inp["b"])
     dx = oracle.backward_dx(inp["gy"], inp["W"])
     dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
-    assert np.array_equal(out["y"], y)
-    assert np.array_equal(out["dx"], dx)
-    assert np.array_equal(out["dW"], dW)
-    assert np.array_equal(out["db"], db)
+    tag = f"integer T={T} C'={Cp} D'={Dp} N={N} {dt}"
+    check_exact(f"{tag} y", out["y"], y)
+    check_exact(f"{tag} dx", out["dx"], dx)
+    check_exact(f"{tag} dW", out["dW"], dW)
+    check_exact(f"{tag} db", out["db"], db)
 
 
 def test_back_to_back_dependencies():
@@ -128,10 +143,10 @@ def test_back_to_back_dependencies():
         assert eqlin.get_error(L1.h) == 0 and eqlin.get_error(L2.h) == 0
         k = {n: t.float().cpu().numpy() for n, t in (("y1", y1), ("y2", y2), ("g1", g1), ("x", x))}
         tol = TOL["bf16"]
-        assert rel_err(k["y1"], oracle.forward(x_in, a["W"], a["b"])) <= tol
-        assert rel_err(k["y2"], oracle.forward(k["y1"], b["W"], b["b"])) <= tol
-        assert rel_err(k["g1"], oracle.backward_dx(k["y2"], b["W"])) <= tol
-        assert rel_err(k["x"], oracle.backward_dx(k["g1"], a["W"])) <= tol
+        check("chain y1", k["y1"], oracle.forward(x_in, a["W"], a["b"]), tol)
+        check("chain y2", k["y2"], oracle.forward(k["y1"], b["W"], b["b"]), tol)
+        check("chain g1", k["g1"], oracle.backward_dx(k["y2"], b["W"]), tol)
+        check("chain x", k["x"], oracle.backward_dx(k["g1"], a["W"]), tol)
 
 
 @pytest.mark.parametrize("T,dt", [(3, "f32"), (6, "f32"), (3, "bf16"), (6, "f16")], ids=str)
@@ -141,12 +156,12 @@ def test_odd_and_sixfold_groups_are_equivariant(T, dt):
     Cp, Dp, N = 16, 24, 150
     inp = _dev(inputs.make_inputs(T, Cp, Dp, N, dt, seed=15))
     layer = eqlin.EQLinear(inp["W"], inp["b"])
-    assert layer.h.backend() == "simt"
+    assert layer.h.backend() == "fwd=simt dx=simt dw=simt"
     y = layer.forward(inp["x"])
     tol = 1e-5 if dt == "f32" else TOL[dt]
     for r in range(1, T):
         yr = layer.forward(_roll(inp["x"], Cp, T, r))
-        assert rel_err(yr.float().cpu(), _roll(y, Dp, T, r).float().cpu()) <= tol
+        check(f"T={T} {dt} equivariance shift {r}", yr, _roll(y, Dp, T, r), tol)
     torch.cuda.synchronize()
     assert eqlin.get_error(layer.h) == 0
 
@@ -178,10 +193,11 @@ def test_calls_from_another_host_thread():
     assert not errs, errs
     assert eqlin.get_error(layer.h) == 0
     tol = TOL["bf16"]
-    assert rel_err(out["y"].float().cpu(), oracle.forward(inp["x"], inp["W"], inp["b"])) <= tol
-    assert rel_err(out["dx"].float().cpu(), oracle.backward_dx(inp["gy"], inp["W"])) <= tol
+    check("other thread y", out["y"], oracle.forward(inp["x"], inp["W"], inp["b"]), tol)
+    check("other thread dx", out["dx"], oracle.backward_dx(inp["gy"], inp["W"]), tol)
     dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
-    assert rel_err(out["dW"].cpu(), dW) <= tol and rel_err(out["db"].cpu(), db) <= tol
+    check("other thread dW", out["dW"], dW, tol)
+    check("other thread db", out["db"], db, tol)
 
 
 def _roll(a: torch.Tensor, ch: int, T: int, r: int) -> torch.Tensor:
@@ -190,39 +206,79 @@ def _roll(a: torch.Tensor, ch: int, T: int, r: int) -> torch.Tensor:
 
 
 FULL = [(name, i) for name, layers in workloads.WORKLOADS.items() for i in range(len(layers))]
+# workloads compared on every output element; the others on stratified samples
+WHOLE = {"p4-tiny-f32-fwd", "eq-vit-s-f16-fwd", "eq-vit-b-mlp-bf16-fwdbwd", "eq-swin-t-s1-f16-fwdbwd"}
+ROW_BLOCK = 16384          # tokens per oracle call when the whole output is compared
+
+
+def _rows_one_per_tile(N: int, rng) -> np.ndarray:
+    """One random token of every 128-token tile, plus the first and the last."""
+    starts = np.arange(0, N, 128)
+    ends = np.minimum(starts + 128, N)
+    pick = starts + (rng.random(len(starts)) * (ends - starts)).astype(np.int64)
+    return np.unique(np.concatenate([[0, N - 1], pick]))
+
+
+def _pairs_every_block(Dp: int, Cp: int, rng, per_block: int = 8) -> np.ndarray:
+    """`per_block` random (d, c) pairs in every 128 x 128 block of the weight."""
+    out = []
+    for d0 in range(0, Dp, 128):
+        for c0 in range(0, Cp, 128):
+            d1, c1 = min(Dp, d0 + 128), min(Cp, c0 + 128)
+            out.append(np.stack([rng.integers(d0, d1, per_block), rng.integers(c0, c1, per_block)], 1))
+    return np.concatenate(out)
+
+
+def _compare_rows(label, got, ref_fn, N, tol, rows=None):
+    """Compare a [N, width] device output with the oracle, in row blocks."""
+    acc = Accum()
+    if rows is None:
+        for a in range(0, N, ROW_BLOCK):
+            r = np.arange(a, min(N, a + ROW_BLOCK))
+            acc.add(got[a:a + len(r)], ref_fn(r))
+    else:
+        acc.add(got[torch.as_tensor(rows, device=got.device)], ref_fn(rows))
+    finish(label, acc, tol)
 
 
 @pytest.mark.parametrize("name,idx", FULL, ids=lambda v: str(v))
-def test_full_size_sampled(name, idx):
+def test_full_size(name, idx):
+    """Every workload at full size, through the same entry points bench.py times."""
     L = workloads.WORKLOADS[name][idx]
     T, Cp, Dp, N, dt = L.T, L.Cp, L.Dp, L.N, L.dtype
+    whole = name in WHOLE
     inp = inputs.make_inputs(T, Cp, Dp, N, dt, seed=0, with_gy=("dx" in L.passes or "dw" in L.passes))
     g = _dev(inp)
+    f64 = {k: v.double().numpy() for k, v in inp.items()}
     layer = eqlin.EQLinear(g["W"], g["b"])
     rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, 62)]))
+    rows = None if whole else _rows_one_per_tile(N, rng)
     tol = TOL[dt]
+    tag = f"full {L.name} N={N} {dt}" + ("" if whole else " (sampled)")
     y = layer.forward(g["x"])
     torch.cuda.synchronize()
     assert eqlin.get_error(layer.h) == 0
-    assert rel_err(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
-                   oracle.forward(inp["x"], inp["W"], inp["b"], rows=rows)) <= tol
+    _compare_rows(f"{tag} y", y, lambda r: oracle.forward(f64["x"], f64["W"], f64["b"], rows=r), N, tol, rows)
     # equivariance on the whole output: rotate the group axis of x by one step
     yr = layer.forward(_roll(g["x"], Cp, T, 1))
-    assert rel_err(yr.float().cpu().numpy(), _roll(y, Dp, T, 1).float().cpu().numpy()) <= tol
+    check(f"{tag} y equivariance", yr, _roll(y, Dp, T, 1), tol)
+    del yr
     if "dx" in L.passes:
         dx = layer.backward_dx(g["gy"])
         torch.cuda.synchronize()
-        assert rel_err(dx[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
-                       oracle.backward_dx(inp["gy"], inp["W"], rows=rows)) <= tol
+        _compare_rows(f"{tag} dx", dx, lambda r: oracle.backward_dx(f64["gy"], f64["W"], rows=r), N, tol, rows)
+        del dx
     if "dw" in L.passes:
         dW, db = layer.backward_dw(g["x"], g["gy"])
         torch.cuda.synchronize()
-        pairs = np.stack([rng.integers(0, Dp, 48), rng.integers(0, Cp, 48)], 1)
-        want, want_db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp, pairs=pairs)
-        got = dW.cpu().numpy()[pairs[:, 0], pairs[:, 1]]
-        assert rel_err(got, want) <= tol
-        assert rel_err(db.cpu().numpy(), want_db) <= tol
+        if whole:
+            want, want_db = oracle.backward_dw(f64["x"], f64["gy"], T, Cp, Dp)
+            check(f"{tag} dW", dW, want, tol)
+        else:
+            pairs = _pairs_every_block(Dp, Cp, rng)
+            want, want_db = oracle.backward_dw(f64["x"], f64["gy"], T, Cp, Dp, pairs=pairs)
+            check(f"{tag} dW", dW.cpu().numpy()[pairs[:, 0], pairs[:, 1]], want, tol)
+        check(f"{tag} db", db, want_db, tol)
     assert eqlin.get_error(layer.h) == 0
 
 
@@ -278,14 +334,18 @@ def test_outputs_have_no_stray_writes():
     assert not (buf[32:32 + N] == 123).all()
 
 
-def test_tensor_core_backend_is_used():
-    """f16/bf16 handles with 8-aligned channel counts run the tcgen05 kernels."""
+def test_backend_is_reported_per_pass():
+    """f16/bf16 handles with 8-aligned channel counts run the tcgen05 kernels in
+    every pass; a pass whose K is not a multiple of 8 runs the SIMT kernels, and
+    the handle says which pass."""
     for dt in ("f16", "bf16"):
         for T in (1, 2, 4, 8):
             h = eqlin.create(T, 64, 64, dt)
-            assert h.backend() == "tcgen05", (T, dt, h.backend())
+            assert h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", (T, dt, h.backend())
             h.close()
-    assert eqlin.create(4, 16, 16, "f32").backend() == "simt"
+    assert eqlin.create(4, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt"
+    assert eqlin.create(4, 6, 16, "f16").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
+    assert eqlin.create(4, 16, 6, "bf16").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
@@ -295,7 +355,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     inp = inputs.make_inputs(T, Cp, Dp, N, "bf16", seed=4)
     g = _dev(inp)
     layer = eqlin.EQLinear(g["W"], g["b"])
-    assert layer.h.backend() == "tcgen05"
+    assert layer.h.backend().startswith("fwd=tcgen05")
     eqlin.set_wait_limit(layer.h, 1)
     layer.forward(g["x"])
     torch.cuda.synchronize()
@@ -306,5 +366,5 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert eqlin.get_error(layer.h) == 0
     rows = np.arange(0, N, 97)
-    assert rel_err(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
-                   oracle.forward(inp["x"], inp["W"], inp["b"], rows=rows)) <= TOL["bf16"]
+    check("after timeout y (sampled rows)", y[torch.as_tensor(rows, device="cuda")],
+          oracle.forward(inp["x"], inp["W"], inp["b"], rows=rows), TOL["bf16"])
