@@ -65,6 +65,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the sub-measurements")
+    ap.add_argument("--path", choices=("fused", "plain"), default="fused",
+                    help="fused: forward and dx stash the spectra, dW from the spectra; "
+                         "plain: dW transforms x and gy itself")
     return ap.parse_args(argv)
 
 
@@ -281,14 +284,21 @@ def profiled_traffic(kernel_key: str):
     return None
 
 
-def pass_work(L, kind):
-    """(actual FLOP, algorithmic bytes) of one call of a pass."""
+def pass_work(L, kind, fused=False):
+    """(actual FLOP, algorithmic bytes) of one call of a pass.  The stash forms
+    (fused path) also write the input's spectrum, as many elements as the input."""
     if kind == "set_weights":
         return 0, L.Dp * L.Cp * L.T * 2 * 2
-    return L.actual_flop(), (L.bytes_dw() if kind == "dw" else L.bytes_fwd())
+    e = workloads.BYTES[L.dtype]
+    extra = 0
+    if fused and kind == "fwd":
+        extra = L.N * L.C * e
+    elif fused and kind == "dx":
+        extra = L.N * L.D * e
+    return L.actual_flop(), (L.bytes_dw() if kind == "dw" else L.bytes_fwd()) + extra
 
 
-def roofline_of(L, kind, us, pk):
+def roofline_of(L, kind, us, pk, fused=False):
     """Roofline of one call of `kind` on layer L that took `us` microseconds.
 
     The bound is the resource the call's arithmetic intensity points at:
@@ -296,7 +306,7 @@ def roofline_of(L, kind, us, pk):
     (dense bf16 peak / copy bandwidth), else HBM.  Calls timed in sub-second
     regions use the burst tensor peak (FP16 and BF16 have the same nominal
     rate).  `frac_roofline` = max(FLOP / tensor peak, bytes / HBM) / time."""
-    flop, byt = pass_work(L, kind)
+    flop, byt = pass_work(L, kind, fused)
     t = us * 1e-6
     tens = pk["bf16"] * 1e12
     hbm = pk["hbm_gbs"] * 1e9
@@ -314,12 +324,17 @@ def roofline_of(L, kind, us, pk):
 
 # ----------------------------------------------------------------- our arm
 class Layers:
-    """Device state of a workload's layers: handles, weights, rotating input sets, outputs."""
+    """Device state of a workload's layers: handles, weights, rotating input sets, outputs.
 
-    def __init__(self, layers, dev, rank, seed_base=0):
+    fused: forward and dx are the stash forms (they also write the spectra
+    X = DFT(x) and G = DFT(gy)) and dW/db come from the spectra; otherwise
+    dW/db transform x and gy themselves."""
+
+    def __init__(self, layers, dev, rank, seed_base=0, fused=True):
         from group_circulant_linear_b200 import eqlin
         self.eqlin = eqlin
         self.layers = layers
+        self.fused = fused
         self.st = []
         for li, L in enumerate(layers):
             dt = inputs.DTYPES[L.dtype]
@@ -329,23 +344,40 @@ class Layers:
                                        with_gy=("dx" in L.passes or "dw" in L.passes), device=dev)
                     for s in range(N_SETS)]
             h = eqlin.create(L.T, L.Cp, L.Dp, dt)
-            self.st.append(dict(L=L, h=h, W=w["W"], b=w["b"], sets=sets,
-                                y=torch.empty((L.N, L.D), dtype=dt, device=dev),
-                                dx=torch.empty((L.N, L.C), dtype=dt, device=dev),
-                                dW=torch.empty((L.Dp, L.Cp, L.T), dtype=torch.float32, device=dev),
-                                db=torch.empty((L.Dp,), dtype=torch.float32, device=dev)))
+            entry = dict(L=L, h=h, W=w["W"], b=w["b"], sets=sets,
+                         y=torch.empty((L.N, L.D), dtype=dt, device=dev),
+                         dx=torch.empty((L.N, L.C), dtype=dt, device=dev),
+                         dW=torch.empty((L.Dp, L.Cp, L.T), dtype=torch.float32, device=dev),
+                         db=torch.empty((L.Dp,), dtype=torch.float32, device=dev))
+            if fused:
+                # one spectra pair per input set: dW of set i reads what the
+                # stash forms wrote for set i
+                entry["xs"] = [eqlin.empty_spectra(h, "x", L.N, device=dev) for _ in range(N_SETS)]
+                entry["gs"] = [eqlin.empty_spectra(h, "gy", L.N, device=dev) for _ in range(N_SETS)]
+            # weights loaded once here; a step also reloads them (set_weights is part of the step)
+            eqlin.set_weights(h, entry["W"], entry["b"])
+            self.st.append(entry)
 
     def set_bytes(self):
         return sum(sum(t.numel() * t.element_size() for t in s["sets"][0].values()) for s in self.st)
 
     def call(self, s, kind, i, stream=None):
-        e, inp = self.eqlin, s["sets"][i % N_SETS]
+        e, j = self.eqlin, i % N_SETS
+        inp = s["sets"][j]
         if kind == "set_weights":
             e.set_weights(s["h"], s["W"], s["b"], stream)
         elif kind == "fwd":
-            e.forward(s["h"], inp["x"], s["y"], stream)
+            if self.fused:
+                e.forward_stash(s["h"], inp["x"], s["y"], s["xs"][j], stream)
+            else:
+                e.forward(s["h"], inp["x"], s["y"], stream)
         elif kind == "dx":
-            e.backward_dx(s["h"], inp["gy"], s["dx"], stream)
+            if self.fused:
+                e.backward_dx_stash(s["h"], inp["gy"], s["dx"], s["gs"][j], stream)
+            else:
+                e.backward_dx(s["h"], inp["gy"], s["dx"], stream)
+        elif self.fused:
+            e.backward_dw_spectra(s["h"], s["xs"][j], s["gs"][j], s["L"].N, s["dW"], s["db"], stream)
         else:
             e.backward_dw(s["h"], inp["x"], inp["gy"], s["dW"], s["db"], stream)
 
@@ -373,7 +405,7 @@ def time_calls(state, li, kind, reps, stream):
     return a.elapsed_time(b) / reps * 1e3
 
 
-def sub_measurements(dev, pk, reps):
+def sub_measurements(dev, pk, reps, fused):
     """The same path on other workload shapes, each call timed on its own."""
     out = {}
     vit_b_f16 = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd",))
@@ -386,12 +418,13 @@ def sub_measurements(dev, pk, reps):
     }
     stream = torch.cuda.current_stream()
     for name, layers in subs.items():
-        state = Layers(layers, dev, 0, seed_base=5000)
+        f = fused and "dw" in layers[0].passes
+        state = Layers(layers, dev, 0, seed_base=5000, fused=f)
         rows, tot_us, dense = [], 0.0, 0
         for li, L in enumerate(layers):
             for kind in L.passes:
                 us = time_calls(state, li, kind, reps, stream)
-                rows.append({"layer": L.name, "pass": kind, **roofline_of(L, kind, us, pk)})
+                rows.append({"layer": L.name, "pass": kind, **roofline_of(L, kind, us, pk, f)})
                 tot_us += us
                 dense += L.dense_flop()
         assert all(e == 0 for e in state.errors()), f"device-side timeout in {name}"
@@ -399,7 +432,7 @@ def sub_measurements(dev, pk, reps):
         del state
         torch.cuda.empty_cache()
         out[name] = {"calls": rows, "dense_tflops": dense / (tot_us * 1e-6) / 1e12,
-                     "us_sum": round(tot_us, 2)}
+                     "us_sum": round(tot_us, 2), "path": "fused" if f else "plain"}
     return out
 
 
@@ -423,13 +456,16 @@ def main(argv=None):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    state = Layers(layers, dev, rank)
+    fused = args.path == "fused"
+    state = Layers(layers, dev, rank, fused=fused)
     eqlin = state.eqlin
     st = state.st
 
-    # A layer's dW/db and its dx read the same inputs and write nothing the
-    # other reads, so dW/db runs on a second stream: its CTAs take the SMs
-    # that dx's last, partial wave leaves idle.  The main stream waits for it
+    # dW/db of a layer runs on a second stream.  Plain path: it reads the same
+    # inputs as dx and writes nothing dx reads, so it starts beside dx and its
+    # CTAs take the SMs of dx's last, partial wave.  Fused path: it reads the
+    # spectrum dx writes, so it starts after dx and runs beside the next
+    # layer's weight transform and forward.  The main stream waits for it
     # before each step ends (and before an all-reduce of dW/db).
     side = torch.cuda.Stream(device=dev)
 
@@ -437,8 +473,11 @@ def main(argv=None):
         for s in st:
             state.call(s, "set_weights", i)
             state.call(s, "fwd", i)
-            side.wait_stream(stream)
+            if not fused:
+                side.wait_stream(stream)
             state.call(s, "dx", i)
+            if fused:
+                side.wait_stream(stream)
             state.call(s, "dw", i, stream=side)
             if dist:
                 stream.wait_stream(side)
@@ -487,14 +526,16 @@ def main(argv=None):
     assert all(e == 0 for e in state.errors()), "device-side timeout in the per-kernel region"
     dom = max(per, key=per.get)
     Ld = layers[dom[0]]
-    roof = roofline_of(Ld, dom[1], per[dom], pk)
-    kernel_of = {"fwd": "tc_apply", "dx": "tc_apply", "dw": "dw", "set_weights": "pretransform"}
+    roof = roofline_of(Ld, dom[1], per[dom], pk, fused)
+    kernel_of = {"fwd": "tc_apply", "dx": "tc_apply", "dw": "dws" if fused else "dw", "set_weights": "pretransform"}
     key = f"{kernel_of[dom[1]]}:{Ld.name}:{dom[1]}"
     roof["kernel"] = key
     roof["peak_kind"] = (f"{pk['source']} " + ("bf16 dense, burst (call timed in a sub-second region)"
                                                if roof["bound"] == "tensor" else "HBM copy"))
     roof["traffic"] = profiled_traffic(key)
     breakdown = {f"{layers[li].name}/{kind}": round(us, 2) for (li, kind), us in per.items()}
+    per_call = {f"{layers[li].name}/{kind}": roofline_of(layers[li], kind, us, pk, fused)
+                for (li, kind), us in per.items() if kind != "set_weights"}
 
     # ---------------------------------------------------------- e2e
     e2e = None
@@ -526,11 +567,15 @@ def main(argv=None):
                 if copied[i] is not None:
                     stream.wait_event(copied[i])
                 eqlin.set_weights(s["h"], s["W"], s["b"])
-                eqlin.forward(s["h"], db_["x"], s["y"])
-                side.wait_stream(stream)
-                eqlin.backward_dx(s["h"], db_["gy"], s["dx"])
-                eqlin.backward_dw(s["h"], db_["x"], db_["gy"], s["dW"], s["db"], stream=side)
-                stream.wait_stream(side)
+                if fused:
+                    eqlin.forward_stash(s["h"], db_["x"], s["y"], s["xs"][0])
+                    eqlin.backward(s["h"], db_["gy"], s["xs"][0], s["dx"], s["gs"][0], s["dW"], s["db"])
+                else:
+                    eqlin.forward(s["h"], db_["x"], s["y"])
+                    side.wait_stream(stream)
+                    eqlin.backward_dx(s["h"], db_["gy"], s["dx"])
+                    eqlin.backward_dw(s["h"], db_["x"], db_["gy"], s["dW"], s["db"], stream=side)
+                    stream.wait_stream(side)
                 if dist:
                     dp.allreduce_grads((s["dW"], s["db"]))
                 d2h_stream.wait_stream(stream)
@@ -565,14 +610,19 @@ def main(argv=None):
     config = {
         "workload": args.workload,
         "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes)) for L in layers],
-        "step": "per layer: set_weights (weight DFT) + forward + dx + dW/db, dW/db on a second stream "
-                "beside dx" + (" + NCCL all-reduce of dW/db" if dist else ""),
+        "path": args.path,
+        "step": ("per layer: set_weights (weight DFT) + forward writing X = DFT(x) + dx writing G = DFT(gy) "
+                 "+ dW/db from the spectra on a second stream beside the next layer"
+                 if fused else
+                 "per layer: set_weights (weight DFT) + forward + dx + dW/db (transforming x and gy), "
+                 "dW/db on a second stream beside dx") + (" + NCCL all-reduce of dW/db" if dist else ""),
         "tokens_per_gpu": layers[0].N,
         "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
               f"({N_SETS * set_bytes / 1e6:.0f} MB > 126 MB L2)",
         "actual_tflops": sum(L.actual_flop() * len(L.passes) for L in layers) * world
                          / (ms_per_step * 1e-3) / 1e12,
         "kernel_us": breakdown,
+        "per_call_roofline": per_call,
         "kernel_us_sampling": f"CUDA events around {KERNEL_REPS} back-to-back launches of each call, "
                               "after the headline region",
     }
@@ -582,7 +632,7 @@ def main(argv=None):
 
     sub = None
     if rank == 0 and not args.no_sub:
-        sub = sub_measurements(dev, pk, KERNEL_REPS)
+        sub = sub_measurements(dev, pk, KERNEL_REPS, fused)
 
     # ---------------------------------------------------- CPU baseline
     cpu = None

@@ -5,9 +5,13 @@ equivariant linear layer, with no retraining, and time it inside EQ-ViT
 blocks ("Flash EQ-Linear", technical summary, sections "Implementacao" and
 "Resultados Experimentais").  This module is that drop-in:
 
-* ``EQLinearFunction`` -- forward runs ``eqlin_forward``; backward runs
-  ``eqlin_backward_dx`` for the input gradient and ``eqlin_backward_dw`` for
-  the weight and bias gradients, all through the C ABI binding.
+* ``EQLinearFunction`` -- when gradients are needed and every pass runs on
+  the tensor cores, forward runs ``eqlin_forward_stash`` and keeps the input's
+  spectrum X = DFT(x) (instead of x) for the backward, which is one
+  ``eqlin_backward`` call: dx with G = DFT(gy) stashed, then dW and db from
+  the two spectra.  Otherwise forward runs ``eqlin_forward`` and backward
+  ``eqlin_backward_dx`` and ``eqlin_backward_dw``.  All through the C ABI
+  binding.
 * ``EQLinear`` -- an ``nn.Module`` holding W [D', C', T] and b [D'] as
   parameters and one library handle; it re-runs the weight transform
   (``eqlin_set_weights``) only when the parameters have changed.
@@ -46,9 +50,18 @@ class EQLinearFunction(torch.autograd.Function):
         lead = x.shape[:-1]
         x2 = x.reshape(-1, layer.Cp * layer.T).to(layer.dtype).contiguous()
         layer.sync_weights(W, b)
-        y = torch.empty((x2.shape[0], layer.Dp * layer.T), dtype=layer.dtype, device=x.device)
-        eqlin.forward(layer.h, x2, y)
-        ctx.save_for_backward(x2)
+        N = x2.shape[0]
+        y = torch.empty((N, layer.Dp * layer.T), dtype=layer.dtype, device=x.device)
+        fused = layer.fused and any(ctx.needs_input_grad[:3]) and N > 0
+        if fused:
+            xs = eqlin.empty_spectra(layer.h, "x", N, device=x.device)
+            eqlin.forward_stash(layer.h, x2, y, xs)
+            ctx.save_for_backward(xs)
+        else:
+            eqlin.forward(layer.h, x2, y)
+            ctx.save_for_backward(x2)
+        ctx.fused = fused
+        ctx.N = N
         ctx.layer = layer
         ctx.lead = lead
         ctx.x_dtype = x.dtype
@@ -58,22 +71,31 @@ class EQLinearFunction(torch.autograd.Function):
 
     @staticmethod
     def backward(ctx, gy):
-        (x2,) = ctx.saved_tensors
+        (saved,) = ctx.saved_tensors
         L = ctx.layer
         gy2 = gy.reshape(-1, L.Dp * L.T).to(L.dtype).contiguous()
         dx = dW = db = None
-        if ctx.needs_input_grad[0]:
-            dx2 = torch.empty_like(x2)
-            eqlin.backward_dx(L.h, gy2, dx2)
-            dx = dx2.reshape(*ctx.lead, L.Cp * L.T).to(ctx.x_dtype)
-        if ctx.needs_input_grad[1] or ctx.needs_input_grad[2]:
+        want_w = ctx.needs_input_grad[1] or ctx.needs_input_grad[2]
+        dx2 = torch.empty((ctx.N, L.Cp * L.T), dtype=L.dtype, device=gy.device) \
+            if (ctx.needs_input_grad[0] or (ctx.fused and want_w)) else None
+        if want_w:
             dWf = torch.empty((L.Dp, L.Cp, L.T), dtype=torch.float32, device=gy.device)
             dbf = torch.empty((L.Dp,), dtype=torch.float32, device=gy.device)
-            eqlin.backward_dw(L.h, x2, gy2, dWf, dbf)
-            if ctx.needs_input_grad[1]:
-                dW = dWf.to(ctx.w_dtype)
-            if ctx.needs_input_grad[2]:
-                db = dbf.to(ctx.b_dtype)
+        if ctx.fused and want_w:
+            # one pass over gy: dx and G = DFT(gy), then dW, db from the spectra
+            gs = eqlin.empty_spectra(L.h, "gy", ctx.N, device=gy.device)
+            eqlin.backward(L.h, gy2, saved, dx2, gs, dWf, dbf)
+        else:
+            if dx2 is not None:
+                eqlin.backward_dx(L.h, gy2, dx2)
+            if want_w:
+                eqlin.backward_dw(L.h, saved, gy2, dWf, dbf)
+        if ctx.needs_input_grad[0]:
+            dx = dx2.reshape(*ctx.lead, L.Cp * L.T).to(ctx.x_dtype)
+        if ctx.needs_input_grad[1]:
+            dW = dWf.to(ctx.w_dtype)
+        if ctx.needs_input_grad[2]:
+            db = dbf.to(ctx.b_dtype)
         return dx, dW, db, None
 
 
@@ -98,6 +120,8 @@ class EQLinear(nn.Module):
         else:
             self.register_parameter("bias", None)
         self.h = eqlin.create(T, Cp, Dp, dtype)
+        # the stash forms serve handles whose every pass runs on the tensor cores
+        self.fused = self.h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
         self._seen = None
 
     def sync_weights(self, W: torch.Tensor, b: torch.Tensor | None):

@@ -140,9 +140,11 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
   }
   const size_t planes = (size_t)T * Cp * Dp;
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
-  if (dtype != EQLIN_F32) {
+  if (dtype != EQLIN_F32 && T != 3 && T != 6) {
     const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
     if (tcb > h.ws_bytes) h.ws_bytes = tcb;
+    const size_t tcs = eqlin::tc_dws_workspace_bytes(T, Cp, Dp, h.sm_count);
+    if (tcs > h.ws_bytes) h.ws_bytes = tcs;
   }
   bool ok = cudaMalloc(&h.wf_fwd, planes * 4) == cudaSuccess &&
             cudaMalloc(&h.wf_bwd, planes * 4) == cudaSuccess &&
@@ -203,7 +205,7 @@ eqlin_status_t eqlin_forward(eqlin_t hh, const void* x, void* y, int64_t N, void
   if (!g.ok) return EQLIN_ERR_CUDA;
   cudaError_t e;
   if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, false))
-    e = eqlin::launch_tc_apply(h, false, x, y, N, (cudaStream_t)stream);
+    e = eqlin::launch_tc_apply(h, false, x, y, nullptr, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, false, x, y, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
@@ -218,7 +220,7 @@ eqlin_status_t eqlin_backward_dx(eqlin_t hh, const void* gy, void* dx, int64_t N
   if (!g.ok) return EQLIN_ERR_CUDA;
   cudaError_t e;
   if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, true))
-    e = eqlin::launch_tc_apply(h, true, gy, dx, N, (cudaStream_t)stream);
+    e = eqlin::launch_tc_apply(h, true, gy, dx, nullptr, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, true, gy, dx, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
@@ -243,6 +245,63 @@ eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, floa
                       ? eqlin::launch_tc_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
                       : eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+int64_t eqlin_spectra_ld(int64_t N) { return N < 0 ? -1 : eqlin::spectra_ld(N); }
+
+eqlin_status_t eqlin_forward_stash(eqlin_t hh, const void* x, void* y, void* xs, int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  eqlin_status_t s = check_io(h, x, y, N);
+  if (s != EQLIN_OK || N == 0) return s;
+  if (!xs) return EQLIN_ERR_INVALID_ARG;
+  if (!aligned16(xs)) return EQLIN_ERR_MISALIGNED;
+  if (h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, false)) return EQLIN_ERR_UNSUPPORTED;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  const cudaError_t e = eqlin::launch_tc_apply(h, false, x, y, xs, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_backward_dx_stash(eqlin_t hh, const void* gy, void* dx, void* gs, int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  eqlin_status_t s = check_io(h, gy, dx, N);
+  if (s != EQLIN_OK || N == 0) return s;
+  if (!gs) return EQLIN_ERR_INVALID_ARG;
+  if (!aligned16(gs)) return EQLIN_ERR_MISALIGNED;
+  if (h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, true)) return EQLIN_ERR_UNSUPPORTED;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  const cudaError_t e = eqlin::launch_tc_apply(h, true, gy, dx, gs, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_backward_dw_spectra(eqlin_t hh, const void* xs, const void* gs, float* dW, float* db,
+                                         int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  if (!dW || N < 0) return EQLIN_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (db && !aligned16(db))) return EQLIN_ERR_MISALIGNED;
+  if (h.dtype == EQLIN_F32 || !eqlin::tc_dw_supported(h)) return EQLIN_ERR_UNSUPPORTED;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  if (N == 0) {
+    cudaError_t e = cudaMemsetAsync(dW, 0, (size_t)h.Dp * h.Cp * h.T * 4, (cudaStream_t)stream);
+    if (e == cudaSuccess && db) e = cudaMemsetAsync(db, 0, (size_t)h.Dp * 4, (cudaStream_t)stream);
+    return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+  }
+  eqlin_status_t s = check_io(h, xs, gs, N);
+  if (s != EQLIN_OK) return s;
+  const cudaError_t e = eqlin::launch_tc_dw_spectra(h, xs, gs, dW, db, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_backward(eqlin_t hh, const void* gy, const void* xs, void* dx, void* gs, float* dW,
+                              float* db, int64_t N, void* stream) {
+  eqlin_status_t s = eqlin_backward_dx_stash(hh, gy, dx, gs, N, stream);
+  if (s != EQLIN_OK) return s;
+  return eqlin_backward_dw_spectra(hh, xs, gs, dW, db, N, stream);
 }
 
 eqlin_status_t eqlin_get_error(eqlin_t hh) {

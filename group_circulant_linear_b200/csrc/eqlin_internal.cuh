@@ -190,6 +190,14 @@ __host__ __device__ inline int64_t wtile_elems(int T, int bo, int64_t rows, int6
   return ((rows + bo - 1) / bo) * ((kdim + TC_BK - 1) / TC_BK) * tc_planes(T) * bo * TC_BK;
 }
 
+// ------------------------------------------------------------ spectra
+// The stash forms of the forward and the input gradient also write the group
+// DFT of their input -- X = DFT(x) [T][C'][ld], G = DFT(gy) [T][D'][ld] --
+// which the weight gradient then reads instead of x and gy.  Planes in the
+// order above, unscaled, in the handle's dtype, tokens contiguous; the row
+// pitch ld is N rounded up to a multiple of 64 tokens (128-byte rows).
+inline int64_t spectra_ld(int64_t N) { return (N + 63) / 64 * 64; }
+
 // ------------------------------------------------------------------ handle
 struct Handle {
   int T = 0;
@@ -283,9 +291,15 @@ cudaError_t launch_dw_reduce(const Handle& h, int splits, const float* part, con
 // tcgen05 path (f16/bf16).  Returns cudaErrorNotSupported when the shape is
 // outside what the kernel handles, so the caller can fall back to SIMT.
 bool tc_supported(const Handle& h, bool backward);
-cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out,
+// Forward (backward = false) or input gradient; with `stash` non-null, also
+// writes the input's spectrum there (see spectra_ld).
+cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out, void* stash,
                             int64_t N, cudaStream_t st);
 bool tc_dw_supported(const Handle& h);
+// dW, db from the spectra written by the stash forms (eqlin_tc_dws.cu).
+size_t tc_dws_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);
+cudaError_t launch_tc_dw_spectra(const Handle& h, const void* xs, const void* gs, float* dW, float* db, int64_t N,
+                                 cudaStream_t st);
 size_t tc_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);
 cudaError_t launch_tc_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
                          int64_t N, cudaStream_t st);

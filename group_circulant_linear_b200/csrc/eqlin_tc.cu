@@ -27,6 +27,14 @@
 //                    (the weight planes carry its 1/T and 2/T scales, so this
 //                    is additions only), bias, cast into a 128B-swizzled
 //                    staging tile, TMA store of 64 output elements x 128 rows
+//   stash warp       (19, stash forms only) TMA stores of the stage's
+//                    transformed A planes -- the input's spectrum, X = DFT(x)
+//                    for the forward, G = DFT(gy) for the input gradient -- to
+//                    a caller-owned buffer [T planes][channels][tokens], for the
+//                    tiles of each token block's first output tile; the weight
+//                    gradient then reads the spectra instead of transforming
+//                    x and gy again.  An operand slot is free once both the
+//                    MMAs and these stores have read it.
 //
 // The two rings are independent: a raw slot is refilled as soon as the
 // transform warps have read it, and an operand slot (the stage's A planes and
@@ -55,7 +63,7 @@ namespace tc {
 
 using namespace ptx;
 
-template <int T, int BO_>
+template <int T, int BO_, bool STASH_ = false>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
@@ -108,7 +116,8 @@ struct Cfg {
   static constexpr int RAW_PRODUCER = TR_WARPS, B_PRODUCER = TR_WARPS + 1;
   static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = TR_WARPS + 3;
   static constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter
-  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+  static constexpr int STASH_WARP = EPI0 + EPI_WARPS;  // present in the stash forms only
+  static constexpr int THREADS = (EPI0 + EPI_WARPS + (STASH_ ? 1 : 0)) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
   static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
 };
@@ -196,11 +205,11 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
   return d;
 }
 
-template <int T, int BO, typename E>
-__global__ void __launch_bounds__(Cfg<T, BO>::THREADS, 1)
+template <int T, int BO, typename E, bool STASH>
+__global__ void __launch_bounds__(Cfg<T, BO, STASH>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
-                Params p) {
-  using C = Cfg<T, BO>;
+                const __grid_constant__ CUtensorMap map_stash, Params p) {
+  using C = Cfg<T, BO, STASH>;
   using G = Group<T>;
   grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -237,7 +246,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     }
     for (int i = 0; i < C::AB_ST; ++i) {
       mbar_init(&ab_full[i], C::GRP_WARPS + 1);
-      mbar_init(&ab_empty[i], 1);
+      mbar_init(&ab_empty[i], STASH ? 2 : 1);     // MMA commit (+ the stash warp)
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -248,6 +257,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     fence_barrier_init();
     prefetch_tensormap(&map_in);
     prefetch_tensormap(&map_out);
+    if (STASH) prefetch_tensormap(&map_stash);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -479,6 +489,52 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       for (int i = 0; i < C::AB_ST; ++i)
         if (n_st > i) mbar_wait(&ab_empty[i], (uint32_t)(((n_st - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
+  } else if (STASH && warp == C::STASH_WARP) {
+    // --------------------------------------------------------- stash warp
+    // Per stage: once the operand slot is full, the tiles of output tile 0
+    // store the slot's T A planes (each two TMA boxes of 64 tokens x 16
+    // channels, the 128B-swizzled image they already have) to the spectra
+    // buffer; the slot is released (second arrival on its empty barrier) once
+    // the stores have read it.  Other tiles release at once.
+    if (lane == 0) {
+      int s = 0, pend = -1;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
+        const int tile = (int)(blockIdx.x + ti * gridDim.x);
+        const bool store = (tile % p.n_otiles) == 0;
+        const int m0 = (tile / p.n_otiles) * C::BM;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!bwait(&ab_full[s], ph, limit, abort_flag)) { ok = false; break; }
+          if (store) {
+            const uint8_t* a_st = a_buf + s * C::A_BYTES;
+#pragma unroll
+            for (int q = 0; q < T; ++q)
+#pragma unroll
+              for (int b = 0; b < 2; ++b)
+                tma_store_3d(&map_stash, a_st + q * C::A_PLANE_BYTES + b * C::A_LBO, m0 + 64 * b, kb * C::BK, q);
+            bulk_commit();
+            bulk_wait_read<1>();          // the previous stage's stores have read their slot
+            if (pend >= 0) mbar_arrive(&ab_empty[pend]);
+            pend = s;
+          } else {
+            if (pend >= 0) {
+              bulk_wait_read<0>();
+              mbar_arrive(&ab_empty[pend]);
+              pend = -1;
+            }
+            mbar_arrive(&ab_empty[s]);
+          }
+          if (++s == C::AB_ST) { s = 0; ph ^= 1; }
+        }
+      }
+      if (pend >= 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(&ab_empty[pend]);
+      }
+      if (!ok) raise_abort(abort_flag, p.err);
+      bulk_wait<0>();                     // the stores have completed before the CTA exits
+    }
   } else {
     // ------------------------------------------------------ epilogue warps
     // Two halves of four warps (one per TMEM lane quarter); half h takes the
@@ -593,10 +649,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
-template <int T, int BO, typename E>
-static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, int64_t N,
+template <int T, int BO, typename E, bool STASH>
+static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, void* stash, int64_t N,
                             cudaStream_t st) {
-  using C = Cfg<T, BO>;
+  using C = Cfg<T, BO, STASH>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int K = (int)(backward ? h.Dp : h.Cp);
@@ -625,6 +681,21 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // spectra of the stash forms: [T planes][K channels][ld tokens], TMA stores of
+  // 64 tokens x 16 channels x 1 plane, 128B swizzle (the A planes' own image);
+  // the token extent N clips the last tile's rows
+  CUtensorMap map_stash = map_out;
+  if (STASH) {
+    const int64_t ld = spectra_ld(N);
+    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)K * ld * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)C::BK, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&map_stash, dt, 3, stash, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   Params p;
   p.N = N;
   p.K = K;
@@ -639,33 +710,41 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
 
   {
-    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E>), C::SMEM_BYTES);
+    const cudaError_t e =
+        set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E, STASH>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E>, dim3((unsigned)grid), dim3(C::THREADS), C::SMEM_BYTES,
-                                   st, map_in, map_out, p);
+  const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH>, dim3((unsigned)grid), dim3(C::THREADS),
+                                   C::SMEM_BYTES, st, map_in, map_out, map_stash, p);
   count_launches(1);
   return e;
 }
 
+template <int T, int BO, typename E>
+static cudaError_t launch_s(const Handle& h, bool bwd, const void* in, void* out, void* stash, int64_t N,
+                            cudaStream_t st) {
+  return stash ? launch_t<T, BO, E, true>(h, bwd, in, out, stash, N, st)
+               : launch_t<T, BO, E, false>(h, bwd, in, out, nullptr, N, st);
+}
+
 template <typename E>
-static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out, int64_t N,
+static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out, void* stash, int64_t N,
                             cudaStream_t st) {
   const int bo = bwd ? h.bo_bwd : h.bo_fwd;
   switch (h.T) {
-    case 1: return bo == 256 ? launch_t<1, 256, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
-    case 2: return bo == 128 ? launch_t<2, 128, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
+    case 1: return bo == 256 ? launch_s<1, 256, E>(h, bwd, in, out, stash, N, st) : cudaErrorInvalidValue;
+    case 2: return bo == 128 ? launch_s<2, 128, E>(h, bwd, in, out, stash, N, st) : cudaErrorInvalidValue;
     case 4:
       switch (bo) {
-        case 128: return launch_t<4, 128, E>(h, bwd, in, out, N, st);
-        case 96: return launch_t<4, 96, E>(h, bwd, in, out, N, st);
-        case 64: return launch_t<4, 64, E>(h, bwd, in, out, N, st);
-        case 32: return launch_t<4, 32, E>(h, bwd, in, out, N, st);
+        case 128: return launch_s<4, 128, E>(h, bwd, in, out, stash, N, st);
+        case 96: return launch_s<4, 96, E>(h, bwd, in, out, stash, N, st);
+        case 64: return launch_s<4, 64, E>(h, bwd, in, out, stash, N, st);
+        case 32: return launch_s<4, 32, E>(h, bwd, in, out, stash, N, st);
       }
       return cudaErrorInvalidValue;
-    case 8: return bo == 32 ? launch_t<8, 32, E>(h, bwd, in, out, N, st) : cudaErrorInvalidValue;
+    case 8: return bo == 32 ? launch_s<8, 32, E>(h, bwd, in, out, stash, N, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }
@@ -682,10 +761,10 @@ bool tc_supported(const Handle& h, bool backward) {
   return true;
 }
 
-cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out, int64_t N,
-                            cudaStream_t st) {
-  if (h.dtype == EQLIN_F16) return tc::launch_e<__half>(h, backward, in, out, N, st);
-  if (h.dtype == EQLIN_BF16) return tc::launch_e<__nv_bfloat16>(h, backward, in, out, N, st);
+cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out, void* stash,
+                            int64_t N, cudaStream_t st) {
+  if (h.dtype == EQLIN_F16) return tc::launch_e<__half>(h, backward, in, out, stash, N, st);
+  if (h.dtype == EQLIN_BF16) return tc::launch_e<__nv_bfloat16>(h, backward, in, out, stash, N, st);
   return cudaErrorNotSupported;
 }
 

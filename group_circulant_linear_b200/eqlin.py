@@ -40,6 +40,11 @@ SIGNATURES = {
     "eqlin_status_string": ([_int], ctypes.c_char_p),
     "eqlin_launch_count": ([], ctypes.c_uint64),
     "eqlin_backward_dw_noalloc": ([_int, _i64, _i64, _int, _vp, _vp, _vp, _vp, _i64, _vp], _int),
+    "eqlin_spectra_ld": ([_i64], _i64),
+    "eqlin_forward_stash": ([_vp, _vp, _vp, _vp, _i64, _vp], _int),
+    "eqlin_backward_dx_stash": ([_vp, _vp, _vp, _vp, _i64, _vp], _int),
+    "eqlin_backward_dw_spectra": ([_vp, _vp, _vp, _vp, _vp, _i64, _vp], _int),
+    "eqlin_backward": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_destroy": ([_vp], None),
 }
 
@@ -164,6 +169,64 @@ def backward_dw(h: Handle, x: torch.Tensor, gy: torch.Tensor, dW: torch.Tensor,
     pw = _dev_ptr(dW, torch.float32, (h.Dp, h.Cp, h.T), "dW")
     pb = None if db is None else _dev_ptr(db, torch.float32, (h.Dp,), "db")
     _check(lib().eqlin_backward_dw(h.ptr, px, pg, pw, pb, N, _stream(stream)), "eqlin_backward_dw")
+
+
+def spectra_ld(N: int) -> int:
+    """Row pitch (tokens) of a spectra buffer for N tokens."""
+    return int(lib().eqlin_spectra_ld(int(N)))
+
+
+def spectra_shape(h: Handle, which: str, N: int) -> tuple:
+    """Shape of the spectra buffer of the input ("x": [T, C', ld]) or of the
+    output gradient ("gy": [T, D', ld]) for N tokens."""
+    ch = {"x": h.Cp, "gy": h.Dp}[which]
+    return (h.T, ch, spectra_ld(N))
+
+
+def empty_spectra(h: Handle, which: str, N: int, device=None) -> torch.Tensor:
+    return torch.empty(spectra_shape(h, which, N), dtype=h.dtype, device=device or "cuda")
+
+
+def forward_stash(h: Handle, x: torch.Tensor, y: torch.Tensor, xs: torch.Tensor, stream=None):
+    """Forward that also writes X = DFT(x) into xs [T, C', ld]."""
+    N = x.shape[0]
+    px = _dev_ptr(x, h.dtype, (N, h.Cp * h.T), "x")
+    py = _dev_ptr(y, h.dtype, (N, h.Dp * h.T), "y")
+    ps = _dev_ptr(xs, h.dtype, spectra_shape(h, "x", N), "xs")
+    _check(lib().eqlin_forward_stash(h.ptr, px, py, ps, N, _stream(stream)), "eqlin_forward_stash")
+
+
+def backward_dx_stash(h: Handle, gy: torch.Tensor, dx: torch.Tensor, gs: torch.Tensor, stream=None):
+    """Input gradient that also writes G = DFT(gy) into gs [T, D', ld]."""
+    N = gy.shape[0]
+    pg = _dev_ptr(gy, h.dtype, (N, h.Dp * h.T), "gy")
+    pd = _dev_ptr(dx, h.dtype, (N, h.Cp * h.T), "dx")
+    ps = _dev_ptr(gs, h.dtype, spectra_shape(h, "gy", N), "gs")
+    _check(lib().eqlin_backward_dx_stash(h.ptr, pg, pd, ps, N, _stream(stream)), "eqlin_backward_dx_stash")
+
+
+def backward_dw_spectra(h: Handle, xs: torch.Tensor, gs: torch.Tensor, N: int, dW: torch.Tensor,
+                        db: torch.Tensor | None = None, stream=None):
+    """dW, db from the spectra of the same N tokens."""
+    pxs = _dev_ptr(xs, h.dtype, spectra_shape(h, "x", N), "xs")
+    pgs = _dev_ptr(gs, h.dtype, spectra_shape(h, "gy", N), "gs")
+    pw = _dev_ptr(dW, torch.float32, (h.Dp, h.Cp, h.T), "dW")
+    pb = None if db is None else _dev_ptr(db, torch.float32, (h.Dp,), "db")
+    _check(lib().eqlin_backward_dw_spectra(h.ptr, pxs, pgs, pw, pb, int(N), _stream(stream)),
+           "eqlin_backward_dw_spectra")
+
+
+def backward(h: Handle, gy: torch.Tensor, xs: torch.Tensor, dx: torch.Tensor, gs: torch.Tensor,
+             dW: torch.Tensor, db: torch.Tensor | None = None, stream=None):
+    """The whole backward (dx, dW, db) given the forward's stash xs; writes gs."""
+    N = gy.shape[0]
+    pg = _dev_ptr(gy, h.dtype, (N, h.Dp * h.T), "gy")
+    pxs = _dev_ptr(xs, h.dtype, spectra_shape(h, "x", N), "xs")
+    pd = _dev_ptr(dx, h.dtype, (N, h.Cp * h.T), "dx")
+    pgs = _dev_ptr(gs, h.dtype, spectra_shape(h, "gy", N), "gs")
+    pw = _dev_ptr(dW, torch.float32, (h.Dp, h.Cp, h.T), "dW")
+    pb = None if db is None else _dev_ptr(db, torch.float32, (h.Dp,), "db")
+    _check(lib().eqlin_backward(h.ptr, pg, pxs, pd, pgs, pw, pb, N, _stream(stream)), "eqlin_backward")
 
 
 def backward_dw_noalloc(T: int, x: torch.Tensor, gy: torch.Tensor, dW: torch.Tensor,

@@ -117,6 +117,60 @@ EQLIN_API eqlin_status_t eqlin_backward_dw(eqlin_t h, const void *x, const void 
                                  float *db, int64_t N, void *stream);
 
 /*
+ * The fused backward: spectra formed once, by the kernels that already form them
+ * --------------------------------------------------------------------------------
+ * The paper fuses the data flow so that the Fourier fragments are formed on
+ * chip and no intermediate goes through global memory where it can be avoided
+ * (technical summary, section "Implementacao"), and attributes the backward
+ * pass's smaller speed-up to the gradient's extra memory traffic (section
+ * "Resultados Experimentais", operator level).  In this library the forward
+ * and the input gradient already form the group DFT of their inputs, X =
+ * DFT(x) and G = DFT(gy), in shared memory as their GEMMs' operands.  Their
+ * stash forms also write those spectra out, and the weight gradient is then
+ * a plain per-frequency GEMM over them (no second DFT of x and gy):
+ *
+ *   dW_hat_k[d, c] = sum_n G_k[n, d] conj(X_k[n, c]),   db[d] = sum_n G_0[n, d]
+ *
+ * Spectra layout: T planes x channels x ld tokens of the handle's dtype,
+ * tokens contiguous, ld = eqlin_spectra_ld(N) (N rounded up to a multiple of
+ * 64); planes in the order Re V_0, Re V_{T/2} (even T), then Re V_k, Im V_k
+ * for k = 1 .. ceil(T/2)-1 (p4: V_0, V_2, Re V_1, Im V_1), the unscaled DFT
+ * V_k = sum_t v_t e^{-2 pi i k t / T}, rounded to the dtype.  X is
+ * [T][C'][ld], G is [T][D'][ld]; columns past N are not written.  The caller
+ * owns these buffers (16-byte aligned device memory).
+ *
+ * The stash forms take f16/bf16 handles whose pass runs on the tensor cores
+ * (eqlin_backend_name shows "tcgen05" for it), else EQLIN_ERR_UNSUPPORTED.
+ */
+
+/* Row pitch, in elements, of a spectra buffer for N tokens (-1 if N < 0). */
+EQLIN_API int64_t eqlin_spectra_ld(int64_t N);
+
+/* eqlin_forward that also writes X = DFT(x) into xs [T][C'][ld]. */
+EQLIN_API eqlin_status_t eqlin_forward_stash(eqlin_t h, const void *x, void *y, void *xs, int64_t N,
+                                             void *stream);
+
+/* eqlin_backward_dx that also writes G = DFT(gy) into gs [T][D'][ld]. */
+EQLIN_API eqlin_status_t eqlin_backward_dx_stash(eqlin_t h, const void *gy, void *dx, void *gs,
+                                                 int64_t N, void *stream);
+
+/*
+ * dW [D', C', T] and db [D'] (float32, overwritten; db may be NULL) from the
+ * spectra xs and gs of the same N tokens, as eqlin_backward_dw computes them
+ * from x and gy.  Uses the handle's workspace; deterministic.
+ */
+EQLIN_API eqlin_status_t eqlin_backward_dw_spectra(eqlin_t h, const void *xs, const void *gs, float *dW,
+                                                   float *db, int64_t N, void *stream);
+
+/*
+ * The whole backward pass in one call, given the forward's stash xs:
+ * dx from gy (writing G into gs), then dW and db from xs and gs.  gy is read
+ * from memory once and transformed once.
+ */
+EQLIN_API eqlin_status_t eqlin_backward(eqlin_t h, const void *gy, const void *xs, void *dx, void *gs,
+                                        float *dW, float *db, int64_t N, void *stream);
+
+/*
  * dW and db without a handle and without any device allocation.
  *
  * For callers that cannot call cudaMalloc -- code that runs while another

@@ -68,7 +68,18 @@ def test_null_handle_calls():
     assert L.eqlin_set_weights(None, None, None, None) == -1
     assert L.eqlin_get_error(None) == -1
     assert L.eqlin_backend_name(None) == b"none"
+    assert L.eqlin_forward_stash(None, None, None, None, 0, None) == -1
+    assert L.eqlin_backward_dx_stash(None, None, None, None, 0, None) == -1
+    assert L.eqlin_backward_dw_spectra(None, None, None, None, None, 0, None) == -1
+    assert L.eqlin_backward(None, None, None, None, None, None, None, 0, None) == -1
     L.eqlin_destroy(None)
+
+
+def test_spectra_row_pitch():
+    L = eqlin.lib()
+    assert [L.eqlin_spectra_ld(n) for n in (0, 1, 63, 64, 65, 12608, 401408)] == \
+        [0, 64, 64, 64, 128, 12608, 401408]
+    assert L.eqlin_spectra_ld(-1) == -1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -34,6 +34,39 @@ def _dev(d):
     return {k: v.cuda() for k, v in d.items()}
 
 
+def _fused_capable(T, Cp, Dp, dt) -> bool:
+    """The stash forms serve f16/bf16 layers whose passes all run on tensor cores."""
+    return dt != "f32" and T in (1, 2, 4, 8) and Cp % 8 == 0 and Dp % 8 == 0
+
+
+def _run_fused(layer, g):
+    """Forward with the input's spectrum stashed, then the one-call backward
+    (dx with G stashed, dW/db from the two spectra)."""
+    h = layer.h
+    N = g["x"].shape[0]
+    xs = eqlin.empty_spectra(h, "x", N)
+    gs = eqlin.empty_spectra(h, "gy", N)
+    y = torch.empty((N, h.Dp * h.T), dtype=h.dtype, device="cuda")
+    dx = torch.empty((N, h.Cp * h.T), dtype=h.dtype, device="cuda")
+    dW = torch.full((h.Dp, h.Cp, h.T), float("nan"), device="cuda")
+    db = torch.full((h.Dp,), float("nan"), device="cuda")
+    eqlin.forward_stash(h, g["x"], y, xs)
+    eqlin.backward(h, g["gy"], xs, dx, gs, dW, db)
+    torch.cuda.synchronize()
+    assert eqlin.get_error(h) == 0
+    return {"y": y, "dx": dx, "dW": dW, "db": db, "xs": xs, "gs": gs}
+
+
+def _spectrum(v: np.ndarray, ch: int, T: int) -> np.ndarray:
+    """[T planes, ch, N] real planes of the DFT along the group axis of v [N, ch*T],
+    from numpy's real FFT: Re V_0, Re V_{T/2} (even T), then Re V_k, Im V_k."""
+    F = np.fft.rfft(np.asarray(v, dtype=np.float64).reshape(-1, ch, T), axis=-1)
+    planes = [F[..., 0].real] + ([F[..., T // 2].real] if T % 2 == 0 else [])
+    for k in range(1, (T + 1) // 2):
+        planes += [F[..., k].real, F[..., k].imag]
+    return np.stack(planes).transpose(0, 2, 1)
+
+
 def _run_all(T, Cp, Dp, dt, inp, passes=("fwd", "dx", "dw")):
     g = _dev(inp)
     layer = eqlin.EQLinear(g["W"], g["b"])
@@ -115,6 +148,72 @@ def test_integer_inputs_bit_exact(T, Cp, Dp, N, dt, amp):
     check_exact(f"{tag} dx", out["dx"], dx)
     check_exact(f"{tag} dW", out["dW"], dW)
     check_exact(f"{tag} db", out["db"], db)
+    if _fused_capable(T, Cp, Dp, dt):
+        layer = eqlin.EQLinear(*(t.cuda() for t in (inp["W"], inp["b"])))
+        f = _run_fused(layer, _dev(inp))
+        check_exact(f"{tag} fused y", f["y"], y)
+        check_exact(f"{tag} fused dx", f["dx"], dx)
+        check_exact(f"{tag} fused dW", f["dW"], dW)
+        check_exact(f"{tag} fused db", f["db"], db)
+        # integer inputs have integer spectra for T in {1, 2, 4} (twiddles 0, +-1):
+        # exact in the operand type; the FFT's rounding noise is removed by rint
+        check_exact(f"{tag} stashed X", f["xs"][..., :N], np.rint(_spectrum(inp["x"].double().numpy(), Cp, T)))
+        check_exact(f"{tag} stashed G", f["gs"][..., :N], np.rint(_spectrum(inp["gy"].double().numpy(), Dp, T)))
+
+
+FUSED = [  # (T, C', D', N, dtype): the stash forms and the one-call backward
+    (4, 192, 768, 1000, "bf16"), (4, 768, 192, 777, "bf16"), (4, 24, 96, 3000, "f16"),
+    (4, 96, 24, 3000, "f16"), (4, 96, 288, 333, "f16"), (2, 64, 48, 515, "bf16"),
+    (8, 64, 16, 257, "f16"), (1, 64, 48, 200, "bf16"), (4, 8, 8, 1, "f16"), (4, 200, 40, 131, "f16"),
+]
+
+
+@pytest.mark.parametrize("T,Cp,Dp,N,dt", FUSED, ids=lambda v: str(v))
+def test_fused_backward(T, Cp, Dp, N, dt):
+    inp = inputs.make_inputs(T, Cp, Dp, N, dt, seed=9)
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    f = _run_fused(layer, g)
+    plain_y, plain_dx = layer.forward(g["x"]), layer.backward_dx(g["gy"])
+    torch.cuda.synchronize()
+    tag = f"fused T={T} C'={Cp} D'={Dp} N={N} {dt}"
+    # the stash forms run the same kernels: identical outputs
+    check_exact(f"{tag} y vs eqlin_forward", f["y"], plain_y)
+    check_exact(f"{tag} dx vs eqlin_backward_dx", f["dx"], plain_dx)
+    tol = TOL[dt]
+    check(f"{tag} y", f["y"], oracle.forward(inp["x"], inp["W"], inp["b"]), tol)
+    check(f"{tag} dx", f["dx"], oracle.backward_dx(inp["gy"], inp["W"]), tol)
+    dW, db = oracle.backward_dw(inp["x"], inp["gy"], T, Cp, Dp)
+    check(f"{tag} dW", f["dW"], dW, tol)
+    check(f"{tag} db", f["db"], db, tol)
+    # the spectra themselves, against numpy's FFT of the same inputs
+    check(f"{tag} stashed X", f["xs"][..., :N], _spectrum(inp["x"].double().numpy(), Cp, T), tol)
+    check(f"{tag} stashed G", f["gs"][..., :N], _spectrum(inp["gy"].double().numpy(), Dp, T), tol)
+    # dW from the spectra alone equals the one-call backward's
+    dW2 = torch.empty_like(f["dW"])
+    db2 = torch.empty_like(f["db"])
+    eqlin.backward_dw_spectra(layer.h, f["xs"], f["gs"], N, dW2, db2)
+    torch.cuda.synchronize()
+    check_exact(f"{tag} dW_spectra vs eqlin_backward", dW2, f["dW"])
+    check_exact(f"{tag} db_spectra vs eqlin_backward", db2, f["db"])
+    assert eqlin.get_error(layer.h) == 0
+
+
+def test_stash_forms_reject_what_they_cannot_serve():
+    h32 = eqlin.create(4, 16, 16, "f32")
+    W = torch.zeros((16, 16, 4), device="cuda")
+    eqlin.set_weights(h32, W, None)
+    x = torch.zeros((10, 64), device="cuda")
+    with pytest.raises(eqlin.EqlinError):
+        eqlin.forward_stash(h32, x, torch.empty_like(x), eqlin.empty_spectra(h32, "x", 10))
+    h3 = eqlin.create(3, 16, 16, "bf16")
+    eqlin.set_weights(h3, torch.zeros((16, 16, 3), device="cuda", dtype=torch.bfloat16), None)
+    xb = torch.zeros((10, 48), device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(eqlin.EqlinError):
+        eqlin.forward_stash(h3, xb, torch.empty_like(xb), eqlin.empty_spectra(h3, "x", 10))
+    assert eqlin.spectra_ld(0) == 0 and eqlin.spectra_ld(1) == 64 and eqlin.spectra_ld(129) == 192
+    h32.close()
+    h3.close()
 
 
 def test_back_to_back_dependencies():
@@ -263,10 +362,18 @@ def test_full_size(name, idx):
     yr = layer.forward(_roll(g["x"], Cp, T, 1))
     check(f"{tag} y equivariance", yr, _roll(y, Dp, T, 1), tol)
     del yr
+    fused = None
+    if "dx" in L.passes and "dw" in L.passes and _fused_capable(T, Cp, Dp, dt):
+        fused = _run_fused(layer, g)
+        check_exact(f"{tag} fused y vs eqlin_forward", fused["y"], y)
+        del fused["xs"], fused["gs"]
+    del y
     if "dx" in L.passes:
         dx = layer.backward_dx(g["gy"])
         torch.cuda.synchronize()
         _compare_rows(f"{tag} dx", dx, lambda r: oracle.backward_dx(f64["gy"], f64["W"], rows=r), N, tol, rows)
+        if fused is not None:
+            check_exact(f"{tag} fused dx vs eqlin_backward_dx", fused["dx"], dx)
         del dx
     if "dw" in L.passes:
         dW, db = layer.backward_dw(g["x"], g["gy"])
@@ -274,11 +381,17 @@ def test_full_size(name, idx):
         if whole:
             want, want_db = oracle.backward_dw(f64["x"], f64["gy"], T, Cp, Dp)
             check(f"{tag} dW", dW, want, tol)
+            if fused is not None:
+                check(f"{tag} fused dW", fused["dW"], want, tol)
         else:
             pairs = _pairs_every_block(Dp, Cp, rng)
             want, want_db = oracle.backward_dw(f64["x"], f64["gy"], T, Cp, Dp, pairs=pairs)
             check(f"{tag} dW", dW.cpu().numpy()[pairs[:, 0], pairs[:, 1]], want, tol)
+            if fused is not None:
+                check(f"{tag} fused dW", fused["dW"].cpu().numpy()[pairs[:, 0], pairs[:, 1]], want, tol)
         check(f"{tag} db", db, want_db, tol)
+        if fused is not None:
+            check(f"{tag} fused db", fused["db"], want_db, tol)
     assert eqlin.get_error(layer.h) == 0
 
 
