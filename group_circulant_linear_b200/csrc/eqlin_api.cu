@@ -150,7 +150,7 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
             cudaMalloc(&h.wf_bwd, planes * 4) == cudaSuccess &&
             cudaMalloc(&h.bias, (size_t)Dp * 4) == cudaSuccess &&
             cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
-            cudaMalloc(&h.err, sizeof(int)) == cudaSuccess;
+            cudaMalloc(&h.err, 4 * sizeof(int)) == cudaSuccess;
   // tensor-core weight tiles only where a tensor-core pass exists (T | 8)
   if (ok && dtype != EQLIN_F32 && (eqlin::tc_supported(h, false) || eqlin::tc_supported(h, true))) {
     h.bo_fwd = eqlin::tc_pick_bo(T, Dp);
@@ -161,7 +161,7 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
     // padding rows and K columns of the tiles stay zero
     if (ok) ok = cudaMemset(h.wt_fwd, 0, nf * e) == cudaSuccess && cudaMemset(h.wt_bwd, 0, nb * e) == cudaSuccess;
   }
-  if (ok) ok = cudaMemset(h.err, 0, sizeof(int)) == cudaSuccess;
+  if (ok) ok = cudaMemset(h.err, 0, 4 * sizeof(int)) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_all(h);
@@ -308,14 +308,22 @@ eqlin_status_t eqlin_get_error(eqlin_t hh) {
   if (!hh) return EQLIN_ERR_INVALID_ARG;
   Handle& h = hh->h;
   DeviceGuard g(h.device);
-  int v = 0;
-  if (cudaMemcpy(&v, h.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return EQLIN_ERR_CUDA;
+  int rec[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(rec, h.err, sizeof(rec), cudaMemcpyDeviceToHost) != cudaSuccess) return EQLIN_ERR_CUDA;
+  const int v = rec[0];
   if (v != eqlin::DEV_OK) {
-    const int zero = 0;
-    if (cudaMemcpy(h.err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    for (int i = 0; i < 4; ++i) h.last_error[i] = (uint32_t)rec[i];
+    const int zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(h.err, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
       return EQLIN_ERR_CUDA;
   }
   return v == eqlin::DEV_OK ? EQLIN_OK : v == eqlin::DEV_TIMEOUT ? EQLIN_ERR_TIMEOUT : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_error_detail(eqlin_t hh, uint32_t detail[4]) {
+  if (!hh || !detail) return EQLIN_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i) detail[i] = hh->h.last_error[i];
+  return EQLIN_OK;
 }
 
 eqlin_status_t eqlin_set_wait_limit(eqlin_t hh, uint32_t iterations) {

@@ -222,7 +222,8 @@ struct Handle {
   float* bias = nullptr;          // [Dp] float32 (zeros when no bias)
   float* ws = nullptr;            // dW split partials
   size_t ws_bytes = 0;
-  int* err = nullptr;             // device error word
+  int* err = nullptr;             // device error record, 4 words (eqlin_wait.cuh)
+  uint32_t last_error[4] = {0, 0, 0, 0};   // the record eqlin_get_error last read, when not OK
   uint32_t wait_limit = 0;        // 0 = default
   // kernel family of each pass, "fwd=<k> dx=<k> dw=<k>" (<k>: tcgen05 or simt)
   char backend[48] = "fwd=simt dx=simt dw=simt";

@@ -24,7 +24,7 @@
 namespace {
 
 constexpr size_t kPartialBytes = size_t(64) << 20;       // per-chunk partial planes
-constexpr size_t kScratchBytes = kPartialBytes + 256;     // + the kernels' error word
+constexpr size_t kScratchBytes = kPartialBytes + 256;     // + the kernels' error record
 
 static __device__ __align__(256) unsigned char g_dw_scratch[kScratchBytes];
 
@@ -97,7 +97,7 @@ extern "C" eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t D
   h.ws_bytes = kPartialBytes;
   h.err = reinterpret_cast<int*>(scratch + kPartialBytes);
   // The error word keeps the previous call's value; it must start at zero.
-  if (cudaMemsetAsync(h.err, 0, sizeof(int), st) != cudaSuccess) return EQLIN_ERR_CUDA;
+  if (cudaMemsetAsync(h.err, 0, 4 * sizeof(int), st) != cudaSuccess) return EQLIN_ERR_CUDA;
   const cudaError_t e = eqlin::launch_tc_dw(h, x, gy, dW, db, N, st);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }

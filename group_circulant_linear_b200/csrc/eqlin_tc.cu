@@ -57,11 +57,13 @@
 #include "eqlin_internal.cuh"
 #include "eqlin_packed.cuh"
 #include "eqlin_ptx.cuh"
+#include "eqlin_wait.cuh"
 
 namespace eqlin {
 namespace tc {
 
 using namespace ptx;
+using namespace waits;
 
 template <int T, int BO_, bool STASH_ = false>
 struct Cfg {
@@ -135,46 +137,6 @@ struct Params {
   uint32_t wait_limit;
   uint32_t ab_fmt;     // 0 f16, 1 bf16
 };
-
-// Bounded wait that also gives up as soon as another role raised the abort flag.
-__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag) {
-  if (mbar_test_wait(bar, parity)) return true;     // already complete: no suspension
-  uint64_t t0 = 0;
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 15u) {
-      if (*abort_flag) return false;
-      const uint64_t t = globaltimer_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > kWaitTimeNs) return false;
-    }
-  }
-  return false;
-}
-
-// Lane 0 waits; the warp then agrees on the outcome (and is ordered after the
-// wait), so no lane leaves a loop that holds warp-synchronous operations.
-__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag, int lane) {
-  int ok = 0;
-  if (lane == 0) ok = bwait(bar, parity, limit, abort_flag) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
-// Every lane waits (each acquires the phase, as a reader of TMA-written data
-// must); the warp agrees on the outcome.
-__device__ __forceinline__ bool wwait_all(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                          volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, bwait(bar, parity, limit, abort_flag));
-}
-
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) {
-  *abort_flag = 1;
-  atomicCAS(err, DEV_OK, DEV_TIMEOUT);
-}
 
 // Eight floats to eight 16-bit values (round to nearest even), two per conversion.
 template <typename E>
@@ -291,7 +253,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     uint32_t rph = 0, aph = 0;
     bool ok = true;
     for (int64_t it = grp; it < my_tiles * nk; it += 2) {
-      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag)) { ok = false; break; }
+      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_APPLY, 1, 1), (uint32_t)it)) { ok = false; break; }
       const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_off;
       uint32_t Pw[2][T][4];
       if constexpr (T <= 4) {
@@ -354,7 +316,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       rs += 2;
       if (rs >= C::RAW_ST) { rs -= C::RAW_ST; rph ^= 1; }
       // the operand slot must have been consumed by the MMAs issued from it
-      if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane)) { ok = false; break; }
+      if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane, p.err, site(K_APPLY, 1, 4), (uint32_t)it)) { ok = false; break; }
       uint8_t* a_st = a_buf + as * C::A_BYTES;
 #pragma unroll
       for (int b = 0; b < 2; ++b)
@@ -391,7 +353,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         const int m0 = (tile / p.n_otiles) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
-          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+          if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 2, 2), (uint32_t)n_raw)) { ok = false; break; }
           mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
           tma_load_2d(raw_buf + s * C::RAW_BYTES, &map_in, kb * C::BK * T, m0, &raw_full[s]);
           ++n_raw;
@@ -415,7 +377,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
         const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)(tile % p.n_otiles) * nk * C::B_BYTES;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+          if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 3, 4), (uint32_t)n_b)) { ok = false; break; }
           // the stage's Q weight planes are one contiguous, pre-swizzled tile
           mbar_arrive_expect_tx(&ab_full[s], C::B_BYTES);
           bulk_load(b_buf + s * C::B_BYTES, wt + (int64_t)kb * C::B_BYTES, C::B_BYTES, &ab_full[s]);
@@ -445,11 +407,11 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       const uint64_t a_desc0 = smem_desc_mn(smem_u32(a_buf), C::A_LBO, C::A_SBO);
       const uint64_t b_desc0 = smem_desc(smem_u32(b_buf), C::B_ROWB);
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag)) { ok = false; break; }
+        if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 4, 6), (uint32_t)ti)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&ab_full[s], ph, limit, abort_flag)) { ok = false; break; }
+          if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 4, 3), (uint32_t)(ti * nk + kb))) { ok = false; break; }
           tc_fence_after();
           const uint64_t a_d = a_desc0 + (uint64_t)((s * C::A_BYTES) >> 4);
           const uint64_t b_d = b_desc0 + (uint64_t)((s * C::B_BYTES) >> 4);
@@ -505,7 +467,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         const bool store = (tile % p.n_otiles) == 0;
         const int m0 = (tile / p.n_otiles) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&ab_full[s], ph, limit, abort_flag)) { ok = false; break; }
+          if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 3), (uint32_t)(ti * nk + kb))) { ok = false; break; }
           if (store) {
             const uint8_t* a_st = a_buf + s * C::A_BYTES;
 #pragma unroll
@@ -561,7 +523,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           s_bias[half * C::BO + i] = (p.bias && ob + i < p.O) ? __ldg(p.bias + ob + i) : 0.f;
       }
       // the four warps of a half share named barriers, so they decide together
-      const bool got = named_bar_and(1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane));
+      const bool got = named_bar_and(
+          1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane, p.err, site(K_APPLY, 5, 5), (uint32_t)ti));
       if (!got) { ok = false; break; }
       tc_fence_after();
       const int m0 = (tile / p.n_otiles) * C::BM;

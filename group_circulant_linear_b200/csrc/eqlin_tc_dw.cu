@@ -46,11 +46,13 @@
 #include "eqlin_internal.cuh"
 #include "eqlin_packed.cuh"
 #include "eqlin_ptx.cuh"
+#include "eqlin_wait.cuh"
 
 namespace eqlin {
 namespace tcdw {
 
 using namespace ptx;
+using namespace waits;
 
 template <int T>
 struct Cfg {
@@ -102,42 +104,6 @@ struct Params {
   uint32_t wait_limit;
   uint32_t ab_fmt;
 };
-
-__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag) {
-  uint64_t t0 = 0;
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 15u) {
-      if (*abort_flag) return false;
-      const uint64_t t = globaltimer_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > kWaitTimeNs) return false;
-    }
-  }
-  return false;
-}
-
-// every lane waits (readers of TMA-written data); the warp agrees on the outcome
-__device__ __forceinline__ bool wwait_all(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                          volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, bwait(bar, parity, limit, abort_flag));
-}
-
-// lane 0 waits, the warp follows (slot reuse)
-__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag, int lane) {
-  int ok = 0;
-  if (lane == 0) ok = bwait(bar, parity, limit, abort_flag) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) {
-  *abort_flag = 1;
-  atomicCAS(err, DEV_OK, DEV_TIMEOUT);
-}
 
 template <typename E>
 __device__ __forceinline__ uint4 pack8(const float* f) {
@@ -234,7 +200,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
     uint32_t rph = 0, oph = 0;
     bool ok = true;
     for (int st = 0; st < nst; ++st) {
-      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag)) { ok = false; break; }
+      if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_DW, 1, 1), (uint32_t)st)) { ok = false; break; }
       uint32_t wv[8][C::W];
       if (active) {
         const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
@@ -289,7 +255,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         }
       }
       // the operand slot must have been consumed by the MMAs issued from it
-      if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane)) { ok = false; break; }
+      if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
       if (active) {
         uint8_t* a_st = op_buf + os * C::OP_BYTES;
         uint8_t* b_st = a_st + C::A_BYTES;
@@ -355,7 +321,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
       // columns [g * BC/2, (g+1) * BC/2).
       const bool all_ok = named_bar_and(3, 256, ok);
       const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-      bool got = all_ok && wwait_all(acc_full, 0, limit, abort_flag);
+      bool got = all_ok && wwait_all(acc_full, 0, limit, abort_flag, p.err, site(K_DW, 4, 5), 0u);
       if (!got && all_ok) raise_abort(abort_flag, p.err);
       if (got) {
         tc_fence_after();
@@ -406,7 +372,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
       for (int i = 0; i < C::PF_STAGES; ++i) prefetch(i);
       for (int st = 0; st < nst; ++st) {
         prefetch(st + C::PF_STAGES);
-        if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+        if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_DW, 2, 2), (uint32_t)st)) { ok = false; break; }
         mbar_arrive_expect_tx(&raw_full[s], tx);
         const int n = (int)(nbeg + (int64_t)st * C::BKN);
         uint8_t* dst = raw_buf + s * C::RAW_BYTES;
@@ -440,7 +406,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
     // window of the first complex product: M = d uses B planes q+1..q+2, M = c planes q..q+1
     const int w1 = swap ? 0 : 1, w2 = swap ? 1 : 0;
     for (int st = 0; st < nst; ++st) {
-      if (!wwait(&op_full[s], ph, limit, abort_flag, lane)) { ok = false; break; }
+      if (!wwait(&op_full[s], ph, limit, abort_flag, lane, p.err, site(K_DW, 3, 3), (uint32_t)st)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint64_t a_d = desc0 + (uint64_t)((s * C::OP_BYTES) >> 4);

@@ -40,11 +40,13 @@
 
 #include "eqlin_internal.cuh"
 #include "eqlin_ptx.cuh"
+#include "eqlin_wait.cuh"
 
 namespace eqlin {
 namespace tcdws {
 
 using namespace ptx;
+using namespace waits;
 
 template <int T>
 struct Cfg {
@@ -80,33 +82,6 @@ struct Params {
   uint32_t wait_limit;
   uint32_t ab_fmt;
 };
-
-__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                      volatile int* abort_flag) {
-  if (mbar_test_wait(bar, parity)) return true;
-  uint64_t t0 = 0;
-  for (uint32_t i = 0; i < limit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 15u) {
-      if (*abort_flag) return false;
-      const uint64_t t = globaltimer_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > kWaitTimeNs) return false;
-    }
-  }
-  return false;
-}
-
-// every lane waits (readers of TMA-written data); the warp agrees on the outcome
-__device__ __forceinline__ bool wwait_all(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                          volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, bwait(bar, parity, limit, abort_flag));
-}
-
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* err) {
-  *abort_flag = 1;
-  atomicCAS(err, DEV_OK, DEV_TIMEOUT);
-}
 
 // Sum of the eight 16-bit values of a 16-byte chunk, in FP32.
 template <typename E>
@@ -178,7 +153,7 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       bool ok = true;
       const uint32_t tx = (uint32_t)C::A_BYTES + (uint32_t)T * b_plane;
       for (int st = 0; st < nst; ++st) {
-        if (!bwait(&empty[s], ph ^ 1, limit, abort_flag)) { ok = false; break; }
+        if (!bwait(&empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_DWS, 1, 2), (uint32_t)st)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[s], tx);
         const int n = (int)(nbeg + (int64_t)st * C::BKN);
         uint8_t* a = smem + s * C::STAGE_BYTES;
@@ -209,7 +184,7 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       const uint64_t desc0 = smem_desc(smem_u32(smem), C::ROWB);
       const uint32_t ap = C::A_PLANE >> 4, bp = b_plane >> 4;
       for (int st = 0; st < nst; ++st) {
-        if (!bwait(&full[s], ph, limit, abort_flag)) { ok = false; break; }
+        if (!bwait(&full[s], ph, limit, abort_flag, p.err, site(K_DWS, 2, 1), (uint32_t)st)) { ok = false; break; }
         tc_fence_after();
         const uint64_t a_d = desc0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
         const uint64_t b_d = a_d + (uint64_t)(C::A_BYTES >> 4);
@@ -263,7 +238,7 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       int s = 0;
       uint32_t ph = 0;
       for (int st = 0; st < nst; ++st) {
-        if (!wwait_all(&full[s], ph, limit, abort_flag)) { ok = false; break; }
+        if (!wwait_all(&full[s], ph, limit, abort_flag, p.err, site(K_DWS, 3, 1), (uint32_t)st)) { ok = false; break; }
         if (r < db_rows) {
           // row r of plane 0 of G: 32 tokens in four 16-byte chunks (the
           // 64B swizzle permutes the chunks within the row; the sum is over all)
@@ -285,7 +260,7 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     // of every CTA is past its main loop; earlier, its waiting CTAs would sit
     // on these SMs through the loop.
     grid_dep_launch();
-    const bool got = ok && wwait_all(acc_full, 0, limit, abort_flag);
+    const bool got = ok && wwait_all(acc_full, 0, limit, abort_flag, p.err, site(K_DWS, 3, 3), 0u);
     if (ok && !got) raise_abort(abort_flag, p.err);
     if (got) {
       tc_fence_after();

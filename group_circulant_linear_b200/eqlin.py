@@ -35,6 +35,7 @@ SIGNATURES = {
     "eqlin_backward_dx": ([_vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_backward_dw": ([_vp, _vp, _vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_get_error": ([_vp], _int),
+    "eqlin_error_detail": ([_vp, ctypes.POINTER(ctypes.c_uint32)], _int),
     "eqlin_set_wait_limit": ([_vp, _u32], _int),
     "eqlin_backend_name": ([_vp], ctypes.c_char_p),
     "eqlin_status_string": ([_int], ctypes.c_char_p),
@@ -245,6 +246,14 @@ def backward_dw_noalloc(T: int, x: torch.Tensor, gy: torch.Tensor, dW: torch.Ten
 def get_error(h: Handle) -> int:
     """Device-side status (0, or -6 for a wait that timed out); clears it."""
     return int(lib().eqlin_get_error(h.ptr))
+
+
+def error_detail(h: Handle) -> dict:
+    """Where the last non-OK eqlin_get_error came from (see eqlin_error_detail)."""
+    d = (ctypes.c_uint32 * 4)()
+    _check(lib().eqlin_error_detail(h.ptr, d), "eqlin_error_detail")
+    return {"status": d[0], "kernel": d[1] >> 8, "role": (d[1] >> 4) & 15, "barrier": d[1] & 15,
+            "cta": d[2] & 0xFFF, "iteration": d[2] >> 12, "polls": d[3] & 0xFFFFF, "ms": d[3] >> 20}
 
 
 def set_wait_limit(h: Handle, iterations: int):

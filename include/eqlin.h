@@ -219,6 +219,17 @@ EQLIN_API eqlin_status_t eqlin_backward_dw_noalloc(int T, int64_t Cp, int64_t Dp
 EQLIN_API eqlin_status_t eqlin_get_error(eqlin_t h);
 
 /*
+ * Where the last error that eqlin_get_error reported (other than EQLIN_OK)
+ * came from, for diagnosis: detail[0] the device status (1 = timeout),
+ * detail[1] the site of the first wait that ran out, (kernel << 8) |
+ * (role << 4) | barrier (kernels: 1 forward/dx, 2 dW from x and gy, 3 dW from
+ * spectra), detail[2] that CTA's index | (its stage or tile counter << 12),
+ * detail[3] the polls it made | (milliseconds it waited << 20).  All zero if
+ * no error has been read on this handle.
+ */
+EQLIN_API eqlin_status_t eqlin_error_detail(eqlin_t h, uint32_t detail[4]);
+
+/*
  * Cap, in polling iterations, on every wait inside this handle's kernels
  * (0 restores the default).  A wait that reaches the cap records
  * EQLIN_ERR_TIMEOUT and its kernel returns early instead of spinning.
