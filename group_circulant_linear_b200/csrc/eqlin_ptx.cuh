@@ -45,14 +45,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// Elapsed time of a wait, from the SM's cycle counter (monotonic on its SM,
+// unlike the global timer, which follows the host clock and can step).
+__device__ __forceinline__ uint64_t cycles_now() { return (uint64_t)clock64(); }
 
-// Upper bound on the wall time of any single wait, whatever the poll limit.
-constexpr uint64_t kWaitTimeNs = 2000000000ull;
+// Upper bound on any single wait, whatever the poll limit: 4e9 cycles, about
+// 2 s at the 1965 MHz maximum SM clock (longer at lower clocks).
+constexpr uint64_t kWaitCycles = 4000000000ull;
+constexpr uint64_t kCyclesPerMs = 1965000ull;
 
 // Non-blocking check that the phase with the given parity has completed.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
@@ -66,16 +66,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed; false after
-// `limit` polls or kWaitTimeNs, whichever comes first.
+// `limit` polls or kWaitCycles, whichever comes first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  uint64_t t0 = 0;
+  const uint64_t t0 = cycles_now();
   for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 15u) {
-      const uint64_t t = globaltimer_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > kWaitTimeNs) return false;
-    }
+    if ((i & 15u) == 15u && cycles_now() - t0 > kWaitCycles) return false;
   }
   return false;
 }

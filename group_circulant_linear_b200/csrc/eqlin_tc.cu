@@ -95,14 +95,25 @@ struct Cfg {
   static constexpr int STAGING = 4 * OUT_TILE_BYTES;
   // ring depths: operand slots (the A planes of a stage and its weight
   // planes share one slot and one pair of barriers, so the MMA thread waits
-  // and commits once per stage): three where three raw slots still fit (the
+  // and commits once per stage): three where four raw slots still fit (the
   // transform writes stage k + 2 while the MMAs of k and k + 1 are in
   // flight), else two; the rest of the budget for raw slots (memory latency)
+  //
+  // The raw ring's depth is even.  The two transform groups take alternate
+  // stages, and stages k and k + RAW_ST share a slot.  With an odd depth they
+  // belong to different groups, so one group could wait on the slot's next
+  // phase while the other group's stage k had not yet landed; an mbarrier
+  // parity wait cannot tell a phase from the one two ahead, so that wait would
+  // return at once, read stale data and complete the slot's release early
+  // (a second TMA load into a slot whose first was still in flight).  With an
+  // even depth both uses of a slot are the same group's, which consumes them
+  // in order.
   static constexpr int BUDGET = 224 * 1024;
-  static constexpr int AB_ST = (BUDGET - STAGING - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 3 ? 3 : 2;
+  static constexpr int AB_ST = (BUDGET - STAGING - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 3 : 2;
   static constexpr int RAW_FIT = (BUDGET - STAGING - AB_ST * (A_BYTES + B_BYTES)) / RAW_BYTES;
-  static constexpr int RAW_ST = RAW_FIT > 8 ? 8 : RAW_FIT;
+  static constexpr int RAW_ST = (RAW_FIT > 8 ? 8 : RAW_FIT) & ~1;
   static_assert(RAW_ST >= 2 && AB_ST >= 2, "two slots per ring (the transform groups take alternate stages)");
+  static_assert(RAW_ST % 2 == 0, "both uses of a raw slot belong to one transform group");
   static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + 1;
   // per epilogue half, the bias of the tile's BO channels (FP32)
   static constexpr int BIAS_BYTES = 2 * BO * 4;

@@ -1,6 +1,6 @@
 // eqlin_wait.cuh -- bounded mbarrier waits shared by the tensor-core kernels.
 //
-// Every wait polls at most `limit` times and at most kWaitTimeNs of wall time.
+// Every wait polls at most `limit` times and at most kWaitCycles SM cycles.
 // A wait that runs out records where it gave up in the handle's error record
 // (first writer wins) and returns false; the kernel then raises its CTA-wide
 // abort flag, drains its own in-flight copies and MMAs, frees TMEM and
@@ -12,7 +12,7 @@
 //   [0] status: DEV_OK, or DEV_TIMEOUT
 //   [1] site of the first wait that ran out: (kernel << 8) | (role << 4) | barrier
 //   [2] that CTA's blockIdx.x | (stage or tile counter << 12)
-//   [3] polls made | (milliseconds waited << 20)
+//   [3] polls made | (milliseconds waited, at the maximum SM clock, << 20)
 #pragma once
 
 #include "eqlin_internal.cuh"
@@ -31,10 +31,10 @@ __device__ __forceinline__ uint32_t site(uint32_t kernel, uint32_t role, uint32_
 }
 
 __device__ __forceinline__ void record_timeout(int* err, uint32_t where, uint32_t iter, uint32_t polls,
-                                               uint64_t ns) {
+                                               uint64_t cycles) {
   if (atomicCAS(err + 1, 0, (int)where) == 0) {
     err[2] = (int)((blockIdx.x & 0xFFFu) | (iter << 12));
-    const uint64_t ms = ns / 1000000u;
+    const uint64_t ms = cycles / kCyclesPerMs;
     err[3] = (int)((polls > 0xFFFFFu ? 0xFFFFFu : polls) | ((ms > 0xFFFu ? 0xFFFu : (uint32_t)ms) << 20));
   }
   atomicCAS(err, DEV_OK, DEV_TIMEOUT);
@@ -45,18 +45,18 @@ __device__ __forceinline__ void record_timeout(int* err, uint32_t where, uint32_
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t limit, volatile int* abort_flag,
                                       int* err, uint32_t where, uint32_t iter) {
   if (mbar_test_wait(bar, parity)) return true;     // already complete: no suspension
-  uint64_t t0 = 0, t = 0;
+  const uint64_t t0 = cycles_now();
+  uint64_t t = t0;
   uint32_t i = 0;
   for (; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15u) == 15u) {
       if (*abort_flag) return false;
-      t = globaltimer_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > kWaitTimeNs) break;
+      t = cycles_now();
+      if (t - t0 > kWaitCycles) break;
     }
   }
-  record_timeout(err, where, iter, i, t0 ? t - t0 : 0);
+  record_timeout(err, where, iter, i, t - t0);
   return false;
 }
 
