@@ -18,23 +18,27 @@
 //                    and write the T frequency planes as token-contiguous
 //                    (MN-major, 128B-swizzled) MMA operands; then a
 //                    generic->async proxy fence
-//   MMA warp         (10)   one thread issues tcgen05.mma into TMEM: for each
-//                    real frequency one M=128, N=BO product; for each complex
-//                    frequency two M=128, N=2*BO products that accumulate
+//                    In the stash forms, the threads of each token block's
+//                    first output tile also store the planes they computed --
+//                    the input's spectrum, X = DFT(x) for the forward, G =
+//                    DFT(gy) for the input gradient -- from registers to a
+//                    caller-owned buffer [T planes][channels][tokens] (one
+//                    16-byte store per plane and 8 tokens), which the weight
+//                    gradient then reads instead of transforming x and gy again
+//   MMA warps        (10, 11) lane 0 of each issues tcgen05.mma into TMEM for
+//                    the accumulators it owns: for each real frequency one
+//                    M=128, N=BO product; for each complex frequency two
+//                    M=128, N=2*BO products that accumulate
 //                    [Re Y | Im Y] = Re X [Re W ; Im W] + Im X [-Im W ; Re W]
-//                    -- R(T) real GEMMs, six for p4
-//   epilogue warps   (11-18) tcgen05.ld of the frequency planes, inverse DFT
+//                    -- R(T) real GEMMs, six for p4.  One thread issues at most
+//                    about one MMA per 160 cycles whatever its size, so two
+//                    issuers split the stage's MMAs (p4: the two real
+//                    frequencies, and the complex block product); an
+//                    accumulator is only ever written by one issuer.
+//   epilogue warps   (12-19) tcgen05.ld of the frequency planes, inverse DFT
 //                    (the weight planes carry its 1/T and 2/T scales, so this
 //                    is additions only), bias, cast into a 128B-swizzled
 //                    staging tile, TMA store of 64 output elements x 128 rows
-//   stash warp       (19, stash forms only) TMA stores of the stage's
-//                    transformed A planes -- the input's spectrum, X = DFT(x)
-//                    for the forward, G = DFT(gy) for the input gradient -- to
-//                    a caller-owned buffer [T planes][channels][tokens], for the
-//                    tiles of each token block's first output tile; the weight
-//                    gradient then reads the spectra instead of transforming
-//                    x and gy again.  An operand slot is free once both the
-//                    MMAs and these stores have read it.
 //
 // The two rings are independent: a raw slot is refilled as soon as the
 // transform warps have read it, and an operand slot (the stage's A planes and
@@ -65,7 +69,7 @@ namespace tc {
 using namespace ptx;
 using namespace waits;
 
-template <int T, int BO_, bool STASH_ = false>
+template <int T, int BO_>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
@@ -114,7 +118,16 @@ struct Cfg {
   static constexpr int RAW_ST = (RAW_FIT > 8 ? 8 : RAW_FIT) & ~1;
   static_assert(RAW_ST >= 2 && AB_ST >= 2, "two slots per ring (the transform groups take alternate stages)");
   static_assert(RAW_ST % 2 == 0, "both uses of a raw slot belong to one transform group");
-  static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + 1;
+  // MMA issuers: a group of accumulators (one per real frequency, one per
+  // complex frequency, which takes two MMAs) belongs to one issuer; in order,
+  // groups go to issuer 0 until it holds half of the stage's MMAs.
+  static constexpr int NMMA = (T == 1) ? 1 : 2;
+  static constexpr int MMAS = G::nreal + 2 * G::ncomplex;          // MMAs per stage
+  __host__ __device__ static constexpr int own_real(int f) { return (NMMA == 1 || 2 * f < MMAS) ? 0 : 1; }
+  __host__ __device__ static constexpr int own_cplx(int k) {
+    return (NMMA == 1 || 2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
+  }
+  static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + NMMA;
   // per epilogue half, the bias of the tile's BO channels (FP32)
   static constexpr int BIAS_BYTES = 2 * BO * 4;
   static constexpr int SMEM_BYTES = RAW_ST * RAW_BYTES + AB_ST * (A_BYTES + B_BYTES) + STAGING +
@@ -127,10 +140,9 @@ struct Cfg {
   static constexpr int TR_WARPS = 8;                   // transform: two groups of four warps
   static constexpr int GRP_WARPS = TR_WARPS / 2;       // warps per stage (16 tokens x 16 channels per warp-half)
   static constexpr int RAW_PRODUCER = TR_WARPS, B_PRODUCER = TR_WARPS + 1;
-  static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = TR_WARPS + 3;
+  static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = MMA_WARP + NMMA;
   static constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter
-  static constexpr int STASH_WARP = EPI0 + EPI_WARPS;  // present in the stash forms only
-  static constexpr int THREADS = (EPI0 + EPI_WARPS + (STASH_ ? 1 : 0)) * 32;
+  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
   static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
 };
@@ -147,6 +159,8 @@ struct Params {
   int* err;
   uint32_t wait_limit;
   uint32_t ab_fmt;     // 0 f16, 1 bf16
+  void* stash;         // stash forms: spectra [T][K][ld] of the input, else nullptr
+  int64_t ld;          // its row pitch (tokens)
 };
 
 // Eight floats to eight 16-bit values (round to nearest even), two per conversion.
@@ -179,10 +193,10 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
 }
 
 template <int T, int BO, typename E, bool STASH>
-__global__ void __launch_bounds__(Cfg<T, BO, STASH>::THREADS, 1)
+__global__ void __launch_bounds__(Cfg<T, BO>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
-                const __grid_constant__ CUtensorMap map_stash, Params p) {
-  using C = Cfg<T, BO, STASH>;
+                Params p) {
+  using C = Cfg<T, BO>;
   using G = Group<T>;
   grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -202,8 +216,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   uint64_t* ab_empty = ab_full + C::AB_ST;
   uint64_t* acc_full = ab_empty + C::AB_ST;
   uint64_t* acc_empty = acc_full + C::NACC;
-  uint64_t* drain_bar = acc_empty + C::NACC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* drain_bar = acc_empty + C::NACC;    // [NMMA]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -219,18 +233,17 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     }
     for (int i = 0; i < C::AB_ST; ++i) {
       mbar_init(&ab_full[i], C::GRP_WARPS + 1);
-      mbar_init(&ab_empty[i], STASH ? 2 : 1);     // MMA commit (+ the stash warp)
+      mbar_init(&ab_empty[i], C::NMMA);           // one commit per MMA issuer
     }
     for (int i = 0; i < C::NACC; ++i) {
-      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_full[i], C::NMMA);
       mbar_init(&acc_empty[i], C::EPI_WARPS * 32);
     }
-    mbar_init(drain_bar, 1);
+    for (int i = 0; i < C::NMMA; ++i) mbar_init(&drain_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&map_in);
     prefetch_tensormap(&map_out);
-    if (STASH) prefetch_tensormap(&map_stash);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -326,6 +339,26 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       }
       rs += 2;
       if (rs >= C::RAW_ST) { rs -= C::RAW_ST; rph ^= 1; }
+      if constexpr (STASH) {
+        // the first output tile of each token block stores the spectrum of
+        // its input: 8 tokens of one channel and plane are 16 contiguous bytes
+        const int64_t ti = it / nk;
+        const int kb = (int)(it - ti * nk);
+        const int tile = (int)(blockIdx.x + ti * gridDim.x);
+        const int ch = kb * C::BK + c;
+        if (tile % p.n_otiles == 0 && ch < p.K) {
+          E* dst = reinterpret_cast<E*>(p.stash) + (int64_t)ch * p.ld;
+          const int64_t t0 = (int64_t)(tile / p.n_otiles) * C::BM + m;
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            if (t0 + 8 * b < p.N) {
+#pragma unroll
+              for (int q = 0; q < T; ++q)
+                *reinterpret_cast<uint4*>(dst + (int64_t)q * p.K * p.ld + t0 + 8 * b) =
+                    make_uint4(Pw[b][q][0], Pw[b][q][1], Pw[b][q][2], Pw[b][q][3]);
+            }
+        }
+      }
       // the operand slot must have been consumed by the MMAs issued from it
       if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane, p.err, site(K_APPLY, 1, 4), (uint32_t)it)) { ok = false; break; }
       uint8_t* a_st = a_buf + as * C::A_BYTES;
@@ -404,8 +437,12 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       for (int i = 0; i < C::AB_ST; ++i)
         if (n_b > i) mbar_wait(&ab_full[i], (uint32_t)(((n_b - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
-  } else if (warp == C::MMA_WARP) {
-    // -------------------------------------------------------------- MMA
+  } else if (warp < C::MMA_WARP + C::NMMA) {
+    // ------------------------------------------------------------- MMA
+    // Issuer mi (lane 0 of MMA warp mi) issues the MMAs of the accumulators it
+    // owns and commits them: every operand slot and accumulator barrier takes
+    // one commit per issuer.
+    const int mi = warp - C::MMA_WARP;
     if (lane == 0) {
       int s = 0, ab = 0;
       uint32_t ph = 0, acph = 0;
@@ -418,21 +455,29 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       const uint64_t a_desc0 = smem_desc_mn(smem_u32(a_buf), C::A_LBO, C::A_SBO);
       const uint64_t b_desc0 = smem_desc(smem_u32(b_buf), C::B_ROWB);
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 4, 6), (uint32_t)ti)) { ok = false; break; }
+        if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 4, 6), (uint32_t)ti)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 4, 3), (uint32_t)(ti * nk + kb))) { ok = false; break; }
+          if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 4, 3), (uint32_t)(ti * nk + kb))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint64_t a_d = a_desc0 + (uint64_t)((s * C::A_BYTES) >> 4);
           const uint64_t b_d = b_desc0 + (uint64_t)((s * C::B_BYTES) >> 4);
           const uint32_t first = kb > 0 ? 1u : 0u;
 #pragma unroll
           for (int f = 0; f < G::nreal; ++f)
-            mma_f16_ss(acc + f * C::BO, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + ((f * C::B_PLANE_BYTES) >> 4),
-                       id_real, first);
+            if (C::own_real(f) == mi)
+              mma_f16_ss(acc + f * C::BO, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + ((f * C::B_PLANE_BYTES) >> 4),
+                         id_real, first);
 #pragma unroll
           for (int k = 1; k <= G::ncomplex; ++k) {
+            if (C::own_cplx(k) != mi) continue;
             const int pr = G::nreal + 2 * (k - 1);
             const int q = G::nreal + 3 * (k - 1);
             const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO;
@@ -451,8 +496,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         if (++ab == C::NACC) { ab = 0; acph ^= 1; }
       }
       if (!ok) raise_abort(abort_flag, p.err);
-      mma_commit(drain_bar);              // arrives once every issued MMA has completed
-      mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+      mma_commit(&drain_bar[mi]);         // arrives once every MMA this thread issued has completed
+      mbar_wait(&drain_bar[mi], 0, kDefaultWaitLimit);
       // The last commit of each operand slot fires on the same completion as
       // the drain's, and nothing else waits for it: an arrival that lands
       // after the CTA has left would write into the shared memory of whatever
@@ -461,52 +506,6 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       const int64_t n_st = my_tiles * nk;
       for (int i = 0; i < C::AB_ST; ++i)
         if (n_st > i) mbar_wait(&ab_empty[i], (uint32_t)(((n_st - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
-    }
-  } else if (STASH && warp == C::STASH_WARP) {
-    // --------------------------------------------------------- stash warp
-    // Per stage: once the operand slot is full, the tiles of output tile 0
-    // store the slot's T A planes (each two TMA boxes of 64 tokens x 16
-    // channels, the 128B-swizzled image they already have) to the spectra
-    // buffer; the slot is released (second arrival on its empty barrier) once
-    // the stores have read it.  Other tiles release at once.
-    if (lane == 0) {
-      int s = 0, pend = -1;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const bool store = (tile % p.n_otiles) == 0;
-        const int m0 = (tile / p.n_otiles) * C::BM;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 3), (uint32_t)(ti * nk + kb))) { ok = false; break; }
-          if (store) {
-            const uint8_t* a_st = a_buf + s * C::A_BYTES;
-#pragma unroll
-            for (int q = 0; q < T; ++q)
-#pragma unroll
-              for (int b = 0; b < 2; ++b)
-                tma_store_3d(&map_stash, a_st + q * C::A_PLANE_BYTES + b * C::A_LBO, m0 + 64 * b, kb * C::BK, q);
-            bulk_commit();
-            bulk_wait_read<1>();          // the previous stage's stores have read their slot
-            if (pend >= 0) mbar_arrive(&ab_empty[pend]);
-            pend = s;
-          } else {
-            if (pend >= 0) {
-              bulk_wait_read<0>();
-              mbar_arrive(&ab_empty[pend]);
-              pend = -1;
-            }
-            mbar_arrive(&ab_empty[s]);
-          }
-          if (++s == C::AB_ST) { s = 0; ph ^= 1; }
-        }
-      }
-      if (pend >= 0) {
-        bulk_wait_read<0>();
-        mbar_arrive(&ab_empty[pend]);
-      }
-      if (!ok) raise_abort(abort_flag, p.err);
-      bulk_wait<0>();                     // the stores have completed before the CTA exits
     }
   } else {
     // ------------------------------------------------------ epilogue warps
@@ -626,7 +625,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 template <int T, int BO, typename E, bool STASH>
 static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, void* stash, int64_t N,
                             cudaStream_t st) {
-  using C = Cfg<T, BO, STASH>;
+  using C = Cfg<T, BO>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int K = (int)(backward ? h.Dp : h.Cp);
@@ -655,21 +654,6 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  // spectra of the stash forms: [T planes][K channels][ld tokens], TMA stores of
-  // 64 tokens x 16 channels x 1 plane, 128B swizzle (the A planes' own image);
-  // the token extent N clips the last tile's rows
-  CUtensorMap map_stash = map_out;
-  if (STASH) {
-    const int64_t ld = spectra_ld(N);
-    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)T};
-    cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)K * ld * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)C::BK, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    if (enc(&map_stash, dt, 3, stash, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
   Params p;
   p.N = N;
   p.K = K;
@@ -682,6 +666,8 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
+  p.stash = stash;
+  p.ld = spectra_ld(N);
 
   {
     const cudaError_t e =
@@ -691,7 +677,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
   const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH>, dim3((unsigned)grid), dim3(C::THREADS),
-                                   C::SMEM_BYTES, st, map_in, map_out, map_stash, p);
+                                   C::SMEM_BYTES, st, map_in, map_out, p);
   count_launches(1);
   return e;
 }

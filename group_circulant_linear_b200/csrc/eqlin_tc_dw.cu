@@ -77,13 +77,22 @@ struct Cfg {
   static constexpr int RAW_FIT = (220 * 1024 - OP_STAGES * OP_BYTES) / RAW_BYTES;
   static constexpr int RAW_STAGES = RAW_FIT > 6 ? 6 : RAW_FIT;
   static_assert(RAW_STAGES >= 2, "two raw stages must fit");
-  static constexpr int NBAR = 2 * RAW_STAGES + 2 * OP_STAGES + 2;
+  // MMA issuers: an accumulator group (a real frequency's plane, or a
+  // complex frequency's [Re | Im] block, two MMAs) belongs to one issuer; in
+  // order, groups go to issuer 0 until it holds half of the stage's MMAs.
+  static constexpr int NMMA = (T == 1) ? 1 : 2;
+  static constexpr int MMAS = G::nreal + 2 * G::ncomplex;
+  __host__ __device__ static constexpr int own_real(int f) { return (NMMA == 1 || 2 * f < MMAS) ? 0 : 1; }
+  __host__ __device__ static constexpr int own_cplx(int k) {
+    return (NMMA == 1 || 2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
+  }
+  static constexpr int NBAR = 2 * RAW_STAGES + 2 * OP_STAGES + 1 + NMMA;
   static constexpr int SMEM_BYTES = OP_STAGES * OP_BYTES + RAW_STAGES * RAW_BYTES + NBAR * 8 + 16 +
                                     BM * 4 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
   static constexpr int TR_WARPS = 16;                     // two token groups x (4 A + 4 B warps)
-  static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;
-  static constexpr int THREADS = (TR_WARPS + 2) * 32;
+  static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;   // MMA warps MMA_WARP .. + NMMA - 1
+  static constexpr int THREADS = (TR_WARPS + 1 + NMMA) * 32;
   static constexpr int PF_STAGES = 12;                    // L2 prefetch distance (stages)
   static constexpr int MA_BOX = BM * T <= 256 ? BM * T : 256;   // M-side TMA box width (elements)
   static constexpr int W = packed::Words<T>::n;
@@ -134,8 +143,8 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
   uint64_t* op_full = raw_empty + C::RAW_STAGES;      // the transform warps have written the operands
   uint64_t* op_empty = op_full + C::OP_STAGES;        // MMA commit
   uint64_t* acc_full = op_empty + C::OP_STAGES;
-  uint64_t* drain_bar = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* drain_bar = acc_full + 1;           // [NMMA]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* db_half = reinterpret_cast<float*>(tmem_slot + 4);       // [BM] token group 1's db sums
 
@@ -160,10 +169,10 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
     }
     for (int i = 0; i < C::OP_STAGES; ++i) {
       mbar_init(&op_full[i], C::TR_WARPS);
-      mbar_init(&op_empty[i], 1);
+      mbar_init(&op_empty[i], C::NMMA);   // one commit per MMA issuer
     }
-    mbar_init(acc_full, 1);
-    mbar_init(drain_bar, 1);
+    mbar_init(acc_full, C::NMMA);
+    for (int i = 0; i < C::NMMA; ++i) mbar_init(&drain_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&map_m);
@@ -394,30 +403,34 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
     grid_dep_launch();
   } else {
     // -------------------------------------------------------------- MMA
-    // The whole warp runs the loop and takes the waits together; one lane
-    // issues the tcgen05 instructions.
-    int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    const uint32_t id_real = idesc_f16(p.ab_fmt, (uint32_t)BC);
-    const uint32_t id_cplx = idesc_f16(p.ab_fmt, (uint32_t)(2 * BC));
-    // descriptors of slot 0, advanced by byte offset >> 4 (start-address field)
-    const uint64_t desc0 = smem_desc(smem_u32(op_buf), C::ROWB);
-    // window of the first complex product: M = d uses B planes q+1..q+2, M = c planes q..q+1
-    const int w1 = swap ? 0 : 1, w2 = swap ? 1 : 0;
-    for (int st = 0; st < nst; ++st) {
-      if (!wwait(&op_full[s], ph, limit, abort_flag, lane, p.err, site(K_DW, 3, 3), (uint32_t)st)) { ok = false; break; }
-      tc_fence_after();
-      if (lane == 0) {
+    // Lane 0 of MMA warp mi issues the MMAs of the accumulator groups it
+    // owns and commits them; the operand slot's and the accumulator's
+    // barriers take one commit per issuer.
+    const int mi = warp - C::MMA_WARP;
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      const uint32_t id_real = idesc_f16(p.ab_fmt, (uint32_t)BC);
+      const uint32_t id_cplx = idesc_f16(p.ab_fmt, (uint32_t)(2 * BC));
+      // descriptors of slot 0, advanced by byte offset >> 4 (start-address field)
+      const uint64_t desc0 = smem_desc(smem_u32(op_buf), C::ROWB);
+      // window of the first complex product: M = d uses B planes q+1..q+2, M = c planes q..q+1
+      const int w1 = swap ? 0 : 1, w2 = swap ? 1 : 0;
+      for (int st = 0; st < nst; ++st) {
+        if (!bwait(&op_full[s], ph, limit, abort_flag, p.err, site(K_DW, 3, 3), (uint32_t)st)) { ok = false; break; }
+        tc_fence_after();
         const uint64_t a_d = desc0 + (uint64_t)((s * C::OP_BYTES) >> 4);
         const uint64_t b_d = a_d + (uint64_t)(C::A_BYTES >> 4);
         const uint32_t bp = b_plane >> 4;
         const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
         for (int f = 0; f < G::nreal; ++f)
-          mma_f16_ss(tmem_base + f * BC, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + f * bp, id_real, first);
+          if (C::own_real(f) == mi)
+            mma_f16_ss(tmem_base + f * BC, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + f * bp, id_real, first);
 #pragma unroll
         for (int k = 1; k <= G::ncomplex; ++k) {
+          if (C::own_cplx(k) != mi) continue;
           const int pr = G::nreal + 2 * (k - 1);
           const int q = G::nreal + 3 * (k - 1);
           const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
@@ -426,16 +439,12 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
           mma_f16_ss(col, a_d + (((pr + 1) * C::A_PLANE_BYTES) >> 4), b_d + (q + w2) * bp, id_cplx, 1u);
         }
         mma_commit(&op_empty[s]);
+        if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
       }
-      __syncwarp();
-      if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
-    }
-    grid_dep_launch();
-    if (lane == 0) {
       if (ok) mma_commit(acc_full);
       else raise_abort(abort_flag, p.err);
-      mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, kDefaultWaitLimit);
+      mma_commit(&drain_bar[mi]);
+      mbar_wait(&drain_bar[mi], 0, kDefaultWaitLimit);
       // The last commit of each operand slot fires on the same completion as
       // the drain's, and nothing else waits for it: an arrival that lands
       // after the CTA has left would write into the shared memory of whatever
@@ -445,6 +454,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         if (nst > i) mbar_wait(&op_empty[i], (uint32_t)(((nst - 1 - i) / C::OP_STAGES) & 1), kDefaultWaitLimit);
     }
     __syncwarp();
+    grid_dep_launch();
   }
 
   tc_fence_before();

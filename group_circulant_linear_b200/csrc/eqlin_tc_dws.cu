@@ -25,8 +25,11 @@
 // Work unit of one CTA: 128 M channels x BC N channels x one contiguous chunk
 // of tokens.  The M side is d or c, whichever pads less to a multiple of 128
 // (M = d: A from G, B from X; M = c: A from X, B from G).  Roles:
-//   warp 0      allocates TMEM; lane 0 issues the MMAs
-//   warp 1      lane 0 issues the TMA loads of each stage (T A planes, T B planes)
+//   warps 0-3   MMA issuers: lane 0 of warp i issues the MMAs of the
+//               accumulator planes it owns (plane q belongs to issuer q mod 4;
+//               one thread issues at most about one MMA per 160 cycles whatever
+//               its size, and these MMAs are small); warp 0 allocates TMEM
+//   warp 8      lane 0 issues the TMA loads of each stage (T A planes, T B planes)
 //   warps 4-7   during the main loop, on the CTAs that own db for their d
 //               channels, each thread sums the k = 0 plane of G along tokens for
 //               one channel; after it, the accumulators out of TMEM (one warp per
@@ -64,8 +67,9 @@ struct Cfg {
   static constexpr int NBAR = 2 * STAGES + 1;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NBAR * 8 + 16 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
-  static constexpr int MMA_WARP = 0, PRODUCER = 1, EPI0 = 4, EPI_WARPS = 4;
-  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+  static constexpr int NMMA = T < 4 ? T : 4;            // MMA issuers (warps 0 .. NMMA-1)
+  static constexpr int MMA_WARP = 0, EPI0 = 4, EPI_WARPS = 4, PRODUCER = 8;
+  static constexpr int THREADS = (PRODUCER + 1) * 32;
 };
 
 struct Params {
@@ -126,9 +130,9 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1 + (sums_db ? C::EPI_WARPS : 0));
+      mbar_init(&empty[i], C::NMMA + (sums_db ? C::EPI_WARPS : 0));
     }
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, C::NMMA);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&map_a);
@@ -173,8 +177,10 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     }
     __syncwarp();
     grid_dep_launch();
-  } else if (warp == C::MMA_WARP) {
+  } else if (warp < C::MMA_WARP + C::NMMA) {
     // -------------------------------------------------------------- MMA
+    // Issuer mi owns the accumulator planes q with q % NMMA == mi.
+    const int mi = warp - C::MMA_WARP;
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -195,22 +201,27 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
           const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
           for (int f = 0; f < G::nreal; ++f)
-            mma_f16_ss(tmem_base + f * BC, ka + f * ap, kb + f * bp, id, acc);
+            if (f % C::NMMA == mi) mma_f16_ss(tmem_base + f * BC, ka + f * ap, kb + f * bp, id, acc);
 #pragma unroll
           for (int k = 1; k <= G::ncomplex; ++k) {
             const int pr = G::nreal + 2 * (k - 1), pi = pr + 1;
-            const uint32_t re = tmem_base + pr * BC, im = tmem_base + pi * BC;
-            // Re += Ar Br + Ai Bi (both orientations)
-            mma_f16_ss(re, ka + pr * ap, kb + pr * bp, id, acc);
-            mma_f16_ss(re, ka + pi * ap, kb + pi * bp, id, 1u);
-            if (!swap) {
-              // M = d (A = G, B = X): Im += Gi Xr - Gr Xi
-              mma_f16_ss(im, ka + pi * ap, kb + pr * bp, id, acc);
-              mma_f16_ss(im, ka + pr * ap, kb + pi * bp, id_neg, 1u);
-            } else {
-              // M = c (A = X, B = G): Im += Xr Gi - Xi Gr
-              mma_f16_ss(im, ka + pr * ap, kb + pi * bp, id, acc);
-              mma_f16_ss(im, ka + pi * ap, kb + pr * bp, id_neg, 1u);
+            if (pr % C::NMMA == mi) {
+              // Re += Ar Br + Ai Bi (both orientations)
+              const uint32_t re = tmem_base + pr * BC;
+              mma_f16_ss(re, ka + pr * ap, kb + pr * bp, id, acc);
+              mma_f16_ss(re, ka + pi * ap, kb + pi * bp, id, 1u);
+            }
+            if (pi % C::NMMA == mi) {
+              const uint32_t im = tmem_base + pi * BC;
+              if (!swap) {
+                // M = d (A = G, B = X): Im += Gi Xr - Gr Xi
+                mma_f16_ss(im, ka + pi * ap, kb + pr * bp, id, acc);
+                mma_f16_ss(im, ka + pr * ap, kb + pi * bp, id_neg, 1u);
+              } else {
+                // M = c (A = X, B = G): Im += Xr Gi - Xi Gr
+                mma_f16_ss(im, ka + pr * ap, kb + pi * bp, id, acc);
+                mma_f16_ss(im, ka + pi * ap, kb + pr * bp, id_neg, 1u);
+              }
             }
           }
         }
@@ -299,7 +310,7 @@ tc_dws_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
-  if (warp == 2 || warp == 3) grid_dep_launch();
+  if (warp >= C::MMA_WARP + C::NMMA && warp < C::EPI0) grid_dep_launch();   // idle warps
 }
 
 struct Plan {
