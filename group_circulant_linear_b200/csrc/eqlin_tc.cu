@@ -18,13 +18,6 @@
 //                    and write the T frequency planes as token-contiguous
 //                    (MN-major, 128B-swizzled) MMA operands; then a
 //                    generic->async proxy fence
-//                    In the stash forms, the threads of each token block's
-//                    first output tile also store the planes they computed --
-//                    the input's spectrum, X = DFT(x) for the forward, G =
-//                    DFT(gy) for the input gradient -- from registers to a
-//                    caller-owned buffer [T planes][channels][tokens] (one
-//                    16-byte store per plane and 8 tokens), which the weight
-//                    gradient then reads instead of transforming x and gy again
 //   MMA warps        (10, 11) lane 0 of each issues tcgen05.mma into TMEM for
 //                    the accumulators it owns: for each real frequency one
 //                    M=128, N=BO product; for each complex frequency two
@@ -39,6 +32,16 @@
 //                    (the weight planes carry its 1/T and 2/T scales, so this
 //                    is additions only), bias, cast into a 128B-swizzled
 //                    staging tile, TMA store of 64 output elements x 128 rows
+//   stash warp       (20, stash forms only) for the tiles of each token
+//                    block's first output tile, TMA stores of the stage's
+//                    transformed A planes -- the input's spectrum, X = DFT(x)
+//                    for the forward, G = DFT(gy) for the input gradient -- to
+//                    a caller-owned buffer [T planes][channels][tokens]; the
+//                    weight gradient then reads the spectra instead of
+//                    transforming x and gy again.  It starts as soon as the
+//                    transform has written the planes (its own barrier), so
+//                    the stores read them while the weights load and the MMAs
+//                    run; an operand slot is free once both have read it.
 //
 // The two rings are independent: a raw slot is refilled as soon as the
 // transform warps have read it, and an operand slot (the stage's A planes and
@@ -69,7 +72,7 @@ namespace tc {
 using namespace ptx;
 using namespace waits;
 
-template <int T, int BO_>
+template <int T, int BO_, bool STASH_ = false>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
@@ -127,7 +130,7 @@ struct Cfg {
   __host__ __device__ static constexpr int own_cplx(int k) {
     return (NMMA == 1 || 2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
   }
-  static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + NMMA;
+  static constexpr int NBAR = 2 * RAW_ST + 3 * AB_ST + 2 * NACC + NMMA;
   // per epilogue half, the bias of the tile's BO channels (FP32)
   static constexpr int BIAS_BYTES = 2 * BO * 4;
   static constexpr int SMEM_BYTES = RAW_ST * RAW_BYTES + AB_ST * (A_BYTES + B_BYTES) + STAGING +
@@ -142,7 +145,8 @@ struct Cfg {
   static constexpr int RAW_PRODUCER = TR_WARPS, B_PRODUCER = TR_WARPS + 1;
   static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = MMA_WARP + NMMA;
   static constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter
-  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+  static constexpr int STASH_WARP = EPI0 + EPI_WARPS;  // present in the stash forms only
+  static constexpr int THREADS = (EPI0 + EPI_WARPS + (STASH_ ? 1 : 0)) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
   static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
 };
@@ -159,8 +163,6 @@ struct Params {
   int* err;
   uint32_t wait_limit;
   uint32_t ab_fmt;     // 0 f16, 1 bf16
-  void* stash;         // stash forms: spectra [T][K][ld] of the input, else nullptr
-  int64_t ld;          // its row pitch (tokens)
 };
 
 // Eight floats to eight 16-bit values (round to nearest even), two per conversion.
@@ -193,10 +195,10 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
 }
 
 template <int T, int BO, typename E, bool STASH>
-__global__ void __launch_bounds__(Cfg<T, BO>::THREADS, 1)
+__global__ void __launch_bounds__(Cfg<T, BO, STASH>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
-                Params p) {
-  using C = Cfg<T, BO>;
+                const __grid_constant__ CUtensorMap map_stash, Params p) {
+  using C = Cfg<T, BO, STASH>;
   using G = Group<T>;
   grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -214,7 +216,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   // planes' bulk-copy bytes have landed; ab_empty: MMA commit
   uint64_t* ab_full = raw_empty + C::RAW_ST;
   uint64_t* ab_empty = ab_full + C::AB_ST;
-  uint64_t* acc_full = ab_empty + C::AB_ST;
+  uint64_t* a_ready = ab_empty + C::AB_ST;     // the transform has written the A planes (stash forms)
+  uint64_t* acc_full = a_ready + C::AB_ST;
   uint64_t* acc_empty = acc_full + C::NACC;
   uint64_t* drain_bar = acc_empty + C::NACC;    // [NMMA]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
@@ -233,7 +236,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     }
     for (int i = 0; i < C::AB_ST; ++i) {
       mbar_init(&ab_full[i], C::GRP_WARPS + 1);
-      mbar_init(&ab_empty[i], C::NMMA);           // one commit per MMA issuer
+      mbar_init(&ab_empty[i], C::NMMA + (STASH ? 1 : 0));   // a commit per MMA issuer (+ the stash warp)
+      mbar_init(&a_ready[i], C::GRP_WARPS);
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], C::NMMA);
@@ -244,6 +248,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     fence_barrier_init();
     prefetch_tensormap(&map_in);
     prefetch_tensormap(&map_out);
+    if (STASH) prefetch_tensormap(&map_stash);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -339,26 +344,6 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       }
       rs += 2;
       if (rs >= C::RAW_ST) { rs -= C::RAW_ST; rph ^= 1; }
-      if constexpr (STASH) {
-        // the first output tile of each token block stores the spectrum of
-        // its input: 8 tokens of one channel and plane are 16 contiguous bytes
-        const int64_t ti = it / nk;
-        const int kb = (int)(it - ti * nk);
-        const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const int ch = kb * C::BK + c;
-        if (tile % p.n_otiles == 0 && ch < p.K) {
-          E* dst = reinterpret_cast<E*>(p.stash) + (int64_t)ch * p.ld;
-          const int64_t t0 = (int64_t)(tile / p.n_otiles) * C::BM + m;
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-            if (t0 + 8 * b < p.N) {
-#pragma unroll
-              for (int q = 0; q < T; ++q)
-                *reinterpret_cast<uint4*>(dst + (int64_t)q * p.K * p.ld + t0 + 8 * b) =
-                    make_uint4(Pw[b][q][0], Pw[b][q][1], Pw[b][q][2], Pw[b][q][3]);
-            }
-        }
-      }
       // the operand slot must have been consumed by the MMAs issued from it
       if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane, p.err, site(K_APPLY, 1, 4), (uint32_t)it)) { ok = false; break; }
       uint8_t* a_st = a_buf + as * C::A_BYTES;
@@ -370,7 +355,10 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
               make_uint4(Pw[b][q][0], Pw[b][q][1], Pw[b][q][2], Pw[b][q][3]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ab_full[as]);
+      if (lane == 0) {
+        mbar_arrive(&ab_full[as]);
+        if (STASH) mbar_arrive(&a_ready[as]);
+      }
       as += 2;
       if (as >= C::AB_ST) { as -= C::AB_ST; aph ^= 1; }
     }
@@ -507,6 +495,55 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       for (int i = 0; i < C::AB_ST; ++i)
         if (n_st > i) mbar_wait(&ab_empty[i], (uint32_t)(((n_st - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
+  } else if (STASH && warp == C::STASH_WARP) {
+    // --------------------------------------------------------- stash warp
+    // Per stage, once the transform has written the A planes: the tiles of
+    // output tile 0 store the slot's T planes (each two TMA boxes of 64 tokens
+    // x 16 channels, the 128B-swizzled image they already have) to the
+    // spectra buffer, and release the slot (its last arrival) once the stores
+    // have read it; other tiles release at once.
+    if (lane == 0) {
+      int s = 0, pend = -1;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
+        const int tile = (int)(blockIdx.x + ti * gridDim.x);
+        const bool store = (tile % p.n_otiles) == 0;
+        const int m0 = (tile / p.n_otiles) * C::BM;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!bwait(&a_ready[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 7), (uint32_t)(ti * nk + kb))) {
+            ok = false;
+            break;
+          }
+          if (store) {
+            const uint8_t* a_st = a_buf + s * C::A_BYTES;
+#pragma unroll
+            for (int q = 0; q < T; ++q)
+#pragma unroll
+              for (int b = 0; b < 2; ++b)
+                tma_store_3d(&map_stash, a_st + q * C::A_PLANE_BYTES + b * C::A_LBO, m0 + 64 * b, kb * C::BK, q);
+            bulk_commit();
+            bulk_wait_read<1>();          // the previous stage's stores have read their slot
+            if (pend >= 0) mbar_arrive(&ab_empty[pend]);
+            pend = s;
+          } else {
+            if (pend >= 0) {
+              bulk_wait_read<0>();
+              mbar_arrive(&ab_empty[pend]);
+              pend = -1;
+            }
+            mbar_arrive(&ab_empty[s]);
+          }
+          if (++s == C::AB_ST) { s = 0; ph ^= 1; }
+        }
+      }
+      if (pend >= 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(&ab_empty[pend]);
+      }
+      if (!ok) raise_abort(abort_flag, p.err);
+      bulk_wait<0>();                     // the stores have completed before the CTA exits
+    }
   } else {
     // ------------------------------------------------------ epilogue warps
     // Two halves of four warps (one per TMEM lane quarter); half h takes the
@@ -625,7 +662,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 template <int T, int BO, typename E, bool STASH>
 static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, void* stash, int64_t N,
                             cudaStream_t st) {
-  using C = Cfg<T, BO>;
+  using C = Cfg<T, BO, STASH>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int K = (int)(backward ? h.Dp : h.Cp);
@@ -654,6 +691,21 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // spectra of the stash forms: [T planes][K channels][ld tokens], TMA stores of
+  // 64 tokens x 16 channels x 1 plane, 128B swizzle (the A planes' own image);
+  // the token extent N clips the last tile's rows
+  CUtensorMap map_stash = map_out;
+  if (STASH) {
+    const int64_t ld = spectra_ld(N);
+    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)K * ld * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)C::BK, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&map_stash, dt, 3, stash, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   Params p;
   p.N = N;
   p.K = K;
@@ -666,8 +718,6 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
-  p.stash = stash;
-  p.ld = spectra_ld(N);
 
   {
     const cudaError_t e =
@@ -677,7 +727,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
   const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH>, dim3((unsigned)grid), dim3(C::THREADS),
-                                   C::SMEM_BYTES, st, map_in, map_out, p);
+                                   C::SMEM_BYTES, st, map_in, map_out, map_stash, p);
   count_launches(1);
   return e;
 }
