@@ -2,8 +2,11 @@
 // forward pass and the input gradient, f16/bf16 in, f32 accumulation.
 //
 // One persistent CTA per SM walks output tiles of 128 tokens x BO output
-// channels (all T group positions).  Per tile and per K stage of 16 input
-// channels:
+// channels (all T group positions), tile t = (output tile t / token blocks,
+// token block t % token blocks), CTA b taking tiles b, b + grid, ...: the CTAs
+// of one wave share an output tile's weights, and the stash forms' stores
+// (output tile 0 only) spread over the CTAs.  Per tile and per K stage of 16
+// input channels:
 //
 //   raw producer     (8)    TMA: the raw input tile of the stage [128 tokens x
 //                    16*T elements] into the raw ring; L2 prefetches of raw
@@ -156,6 +159,7 @@ struct Params {
   int K;           // input channels per group element (C' forward, D' for dx)
   int O;           // output channels per group element
   int n_otiles;
+  int n_tb;        // 128-token blocks; tile t covers token block t % n_tb, output tile t / n_tb
   int64_t n_tiles;
   const void* in;
   const void* wtiles;  // tensor-core weight tiles (rows O, K) of this pass
@@ -376,13 +380,13 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       auto prefetch_next = [&]() {
         if (pf_ti >= my_tiles) return;
         const int tile = (int)(blockIdx.x + pf_ti * gridDim.x);
-        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, (tile / p.n_otiles) * C::BM);
+        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, (tile % p.n_tb) * C::BM);
         if (++pf_kb == nk) { pf_kb = 0; ++pf_ti; }
       };
       for (int i = 0; i < C::PF_STAGES; ++i) prefetch_next();
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const int m0 = (tile / p.n_otiles) * C::BM;
+        const int m0 = (tile % p.n_tb) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
           if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 2, 2), (uint32_t)n_raw)) { ok = false; break; }
@@ -407,7 +411,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       bool ok = true;
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)(tile % p.n_otiles) * nk * C::B_BYTES;
+        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)(tile / p.n_tb) * nk * C::B_BYTES;
         for (int kb = 0; kb < nk; ++kb) {
           if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 3, 4), (uint32_t)n_b)) { ok = false; break; }
           // the stage's Q weight planes are one contiguous, pre-swizzled tile
@@ -508,8 +512,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       bool ok = true;
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const bool store = (tile % p.n_otiles) == 0;
-        const int m0 = (tile / p.n_otiles) * C::BM;
+        const bool store = tile < p.n_tb;          // output tile 0
+        const int m0 = (tile % p.n_tb) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
           if (!bwait(&a_ready[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 7), (uint32_t)(ti * nk + kb))) {
             ok = false;
@@ -565,7 +569,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       // this half's copy of the tile's bias, loaded while the MMAs run (the
       // half's previous tile has finished reading it)
       {
-        const int ob = (tile % p.n_otiles) * C::BO;
+        const int ob = (tile / p.n_tb) * C::BO;
         for (int i = (e & 3) * 32 + lane; i < C::BO; i += 128)
           s_bias[half * C::BO + i] = (p.bias && ob + i < p.O) ? __ldg(p.bias + ob + i) : 0.f;
       }
@@ -574,8 +578,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane, p.err, site(K_APPLY, 5, 5), (uint32_t)ti));
       if (!got) { ok = false; break; }
       tc_fence_after();
-      const int m0 = (tile / p.n_otiles) * C::BM;
-      const int o0 = (tile % p.n_otiles) * C::BO;
+      const int m0 = (tile % p.n_tb) * C::BM;
+      const int o0 = (tile / p.n_tb) * C::BO;
       const uint32_t acc = tmem_base + lane_addr + ab * C::ACC_COLS;
 #pragma unroll 1
       for (int ci = half; ci < C::NCHUNK; ci += 2) {
@@ -711,7 +715,8 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.K = K;
   p.O = O;
   p.n_otiles = (O + C::BO - 1) / C::BO;
-  p.n_tiles = ((N + C::BM - 1) / C::BM) * p.n_otiles;
+  p.n_tb = (int)((N + C::BM - 1) / C::BM);
+  p.n_tiles = (int64_t)p.n_tb * p.n_otiles;
   p.in = in;
   p.wtiles = backward ? h.wt_bwd : h.wt_fwd;
   p.bias = backward ? nullptr : h.bias;
