@@ -145,3 +145,94 @@ void eqlin_oracle_backward_dw(int64_t T, int64_t Cp, int64_t Dp, int64_t N,
         }
     }
 }
+
+/*
+ * The same layer over any finite group G of order n given by its
+ * multiplication table, for the reflection (dihedral) groups the paper names
+ * as future work (technical summary, section "Limitacoes e Trabalho Futuro")
+ * and which it does not spell out.  The plainest generalisation of the
+ * cyclic formula above -- whose kernel index (s - t) mod T is h^-1 g for the
+ * group elements g = s, h = t of Z_T -- is the group convolution
+ *
+ *     y[n, d*n+g]  = b[d] + sum_c sum_h W[d, c, h^-1 g] * x[n, c*n+h]
+ *
+ * which commutes with the left action (L_u x)[h] = x[u^-1 h] of every u in G.
+ * Its exact gradients (derived from this definition):
+ *
+ *     dx[n, c*n+h] = sum_d sum_g W[d, c, h^-1 g] * gy[n, d*n+g]
+ *     dW[d, c, u]  = sum_n sum_h x[n, c*n+h] * gy[n, d*n + h u]
+ *     db[d]        = sum_n sum_g gy[n, d*n+g]
+ *
+ * mul[g*n + h] is the index of the product g h and inv[g] that of g^-1.
+ */
+void eqlin_oracle_forward_group(int64_t G, const int64_t *mul, const int64_t *inv,
+                                int64_t Cp, int64_t Dp,
+                                const double *x, const double *W, const double *b,
+                                const int64_t *rows, int64_t n_out, double *y)
+{
+    int64_t i;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < n_out; ++i) {
+        const int64_t n = rows ? rows[i] : i;
+        for (int64_t d = 0; d < Dp; ++d) {
+            for (int64_t g = 0; g < G; ++g) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < Cp; ++c)
+                    for (int64_t h = 0; h < G; ++h)
+                        acc += W[(d * Cp + c) * G + mul[inv[h] * G + g]] *
+                               x[n * Cp * G + c * G + h];
+                y[i * Dp * G + d * G + g] = (b ? b[d] : 0.0) + acc;
+            }
+        }
+    }
+}
+
+void eqlin_oracle_backward_dx_group(int64_t G, const int64_t *mul, const int64_t *inv,
+                                    int64_t Cp, int64_t Dp,
+                                    const double *gy, const double *W,
+                                    const int64_t *rows, int64_t n_out, double *dx)
+{
+    int64_t i;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < n_out; ++i) {
+        const int64_t n = rows ? rows[i] : i;
+        for (int64_t c = 0; c < Cp; ++c) {
+            for (int64_t h = 0; h < G; ++h) {
+                double acc = 0.0;
+                for (int64_t d = 0; d < Dp; ++d)
+                    for (int64_t g = 0; g < G; ++g)
+                        acc += W[(d * Cp + c) * G + mul[inv[h] * G + g]] *
+                               gy[n * Dp * G + d * G + g];
+                dx[i * Cp * G + c * G + h] = acc;
+            }
+        }
+    }
+}
+
+void eqlin_oracle_backward_dw_group(int64_t G, const int64_t *mul, int64_t Cp, int64_t Dp, int64_t N,
+                                    const double *x, const double *gy, double *dW, double *db)
+{
+    int64_t j;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (j = 0; j < Dp * Cp; ++j) {
+        const int64_t d = j / Cp, c = j % Cp;
+        for (int64_t u = 0; u < G; ++u) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                for (int64_t h = 0; h < G; ++h)
+                    acc += x[n * Cp * G + c * G + h] * gy[n * Dp * G + d * G + mul[h * G + u]];
+            dW[j * G + u] = acc;
+        }
+    }
+    if (db) {
+        int64_t d;
+#pragma omp parallel for schedule(static)
+        for (d = 0; d < Dp; ++d) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                for (int64_t g = 0; g < G; ++g)
+                    acc += gy[n * Dp * G + d * G + g];
+            db[d] = acc;
+        }
+    }
+}
