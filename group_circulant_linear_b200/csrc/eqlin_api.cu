@@ -117,11 +117,20 @@ const char* eqlin_status_string(eqlin_status_t s) {
 }
 
 eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, eqlin_t* out) {
+  return eqlin_create_group(EQLIN_GROUP_CYCLIC, T, Cp, Dp, dtype, out);
+}
+
+eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype,
+                                  eqlin_t* out) {
   if (!out) return EQLIN_ERR_INVALID_ARG;
   *out = nullptr;
   if (dtype != EQLIN_F32 && dtype != EQLIN_F16 && dtype != EQLIN_BF16) return EQLIN_ERR_INVALID_ARG;
+  if (group != EQLIN_GROUP_CYCLIC && group != EQLIN_GROUP_DIHEDRAL) return EQLIN_ERR_INVALID_ARG;
   if (Cp < 1 || Dp < 1) return EQLIN_ERR_INVALID_ARG;
-  if (T != 1 && T != 2 && T != 3 && T != 4 && T != 6 && T != 8) return EQLIN_ERR_UNSUPPORTED;
+  const bool dihedral = group == EQLIN_GROUP_DIHEDRAL;
+  if (dihedral && !eqlin::dihedral_supported(m)) return EQLIN_ERR_UNSUPPORTED;
+  const int T = dihedral ? 2 * m : m;      // group order
+  if (!dihedral && T != 1 && T != 2 && T != 3 && T != 4 && T != 6 && T != 8) return EQLIN_ERR_UNSUPPORTED;
   if (Cp > 65536 || Dp > 65536) return EQLIN_ERR_UNSUPPORTED;
   const size_t e = elem_size(dtype);
   if ((Cp * T * e) % 16 || (Dp * T * e) % 16) return EQLIN_ERR_MISALIGNED;
@@ -130,6 +139,8 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
   if (!hh) return EQLIN_ERR_OOM;
   Handle& h = hh->h;
   h.T = T;
+  h.group = group;
+  h.m = m;
   h.Cp = Cp;
   h.Dp = Dp;
   h.dtype = dtype;
@@ -140,7 +151,7 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
   }
   const size_t planes = (size_t)T * Cp * Dp;
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
-  if (dtype != EQLIN_F32 && T != 3 && T != 6) {
+  if (!dihedral && dtype != EQLIN_F32 && T != 3 && T != 6) {
     const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
     if (tcb > h.ws_bytes) h.ws_bytes = tcb;
     const size_t tcs = eqlin::tc_dws_workspace_bytes(T, Cp, Dp, h.sm_count);
@@ -152,7 +163,7 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
             cudaMalloc(&h.ws, h.ws_bytes) == cudaSuccess &&
             cudaMalloc(&h.err, 4 * sizeof(int)) == cudaSuccess;
   // tensor-core weight tiles only where a tensor-core pass exists (T | 8)
-  if (ok && dtype != EQLIN_F32 && (eqlin::tc_supported(h, false) || eqlin::tc_supported(h, true))) {
+  if (ok && !dihedral && dtype != EQLIN_F32 && (eqlin::tc_supported(h, false) || eqlin::tc_supported(h, true))) {
     h.bo_fwd = eqlin::tc_pick_bo(T, Dp);
     h.bo_bwd = eqlin::tc_pick_bo(T, Cp);
     const size_t nf = (size_t)eqlin::wtile_elems(T, h.bo_fwd, Dp, Cp);
@@ -168,8 +179,8 @@ eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype, 
     delete hh;
     return EQLIN_ERR_OOM;
   }
-  h.need_simt_fwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, false);
-  h.need_simt_bwd = dtype == EQLIN_F32 || !eqlin::tc_supported(h, true);
+  h.need_simt_fwd = dihedral || dtype == EQLIN_F32 || !eqlin::tc_supported(h, false);
+  h.need_simt_bwd = dihedral || dtype == EQLIN_F32 || !eqlin::tc_supported(h, true);
   snprintf(h.backend, sizeof(h.backend), "fwd=%s dx=%s dw=%s", h.need_simt_fwd ? "simt" : "tcgen05",
            h.need_simt_bwd ? "simt" : "tcgen05", eqlin::tc_dw_supported(h) ? "tcgen05" : "simt");
   *out = hh;
@@ -190,7 +201,8 @@ eqlin_status_t eqlin_set_weights(eqlin_t hh, const void* W, const void* b, void*
   if (!aligned16(W) || (b && ((uintptr_t)b % elem_size(h.dtype)))) return EQLIN_ERR_MISALIGNED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
-  cudaError_t e = eqlin::launch_pretransform(h, W, b, (cudaStream_t)stream);
+  cudaError_t e = h.group == EQLIN_GROUP_DIHEDRAL ? eqlin::launch_dihedral_pretransform(h, W, b, (cudaStream_t)stream)
+                                                  : eqlin::launch_pretransform(h, W, b, (cudaStream_t)stream);
   if (e != cudaSuccess) return EQLIN_ERR_CUDA;
   h.has_weights = true;
   return EQLIN_OK;
@@ -204,7 +216,9 @@ eqlin_status_t eqlin_forward(eqlin_t hh, const void* x, void* y, int64_t N, void
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
   cudaError_t e;
-  if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, false))
+  if (h.group == EQLIN_GROUP_DIHEDRAL)
+    e = eqlin::launch_dihedral_apply(h, false, x, y, N, (cudaStream_t)stream);
+  else if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, false))
     e = eqlin::launch_tc_apply(h, false, x, y, nullptr, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, false, x, y, N, (cudaStream_t)stream);
@@ -219,7 +233,9 @@ eqlin_status_t eqlin_backward_dx(eqlin_t hh, const void* gy, void* dx, int64_t N
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
   cudaError_t e;
-  if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, true))
+  if (h.group == EQLIN_GROUP_DIHEDRAL)
+    e = eqlin::launch_dihedral_apply(h, true, gy, dx, N, (cudaStream_t)stream);
+  else if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, true))
     e = eqlin::launch_tc_apply(h, true, gy, dx, nullptr, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, true, gy, dx, N, (cudaStream_t)stream);
@@ -241,9 +257,9 @@ eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, floa
   }
   eqlin_status_t s = check_io(h, x, gy, N);
   if (s != EQLIN_OK) return s;
-  cudaError_t e = eqlin::tc_dw_supported(h)
-                      ? eqlin::launch_tc_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
-                      : eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
+  cudaError_t e = h.group == EQLIN_GROUP_DIHEDRAL ? eqlin::launch_dihedral_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
+                  : eqlin::tc_dw_supported(h)      ? eqlin::launch_tc_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
+                                                   : eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }
 
@@ -256,7 +272,8 @@ eqlin_status_t eqlin_forward_stash(eqlin_t hh, const void* x, void* y, void* xs,
   if (s != EQLIN_OK || N == 0) return s;
   if (!xs) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(xs)) return EQLIN_ERR_MISALIGNED;
-  if (h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, false)) return EQLIN_ERR_UNSUPPORTED;
+  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, false))
+    return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
   const cudaError_t e = eqlin::launch_tc_apply(h, false, x, y, xs, N, (cudaStream_t)stream);
@@ -270,7 +287,8 @@ eqlin_status_t eqlin_backward_dx_stash(eqlin_t hh, const void* gy, void* dx, voi
   if (s != EQLIN_OK || N == 0) return s;
   if (!gs) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(gs)) return EQLIN_ERR_MISALIGNED;
-  if (h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, true)) return EQLIN_ERR_UNSUPPORTED;
+  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, true))
+    return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
   const cudaError_t e = eqlin::launch_tc_apply(h, true, gy, dx, gs, N, (cudaStream_t)stream);
@@ -283,7 +301,8 @@ eqlin_status_t eqlin_backward_dw_spectra(eqlin_t hh, const void* xs, const void*
   Handle& h = hh->h;
   if (!dW || N < 0) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(dW) || (db && !aligned16(db))) return EQLIN_ERR_MISALIGNED;
-  if (h.dtype == EQLIN_F32 || !eqlin::tc_dw_supported(h)) return EQLIN_ERR_UNSUPPORTED;
+  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_dw_supported(h))
+    return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
   if (N == 0) {

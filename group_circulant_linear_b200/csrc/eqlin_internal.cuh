@@ -200,7 +200,9 @@ inline int64_t spectra_ld(int64_t N) { return (N + 63) / 64 * 64; }
 
 // ------------------------------------------------------------------ handle
 struct Handle {
-  int T = 0;
+  int T = 0;                      // group order (cyclic: T; dihedral D_m: 2m)
+  int group = EQLIN_GROUP_CYCLIC;
+  int m = 0;                      // dihedral groups: D_m
   int64_t Cp = 0, Dp = 0;
   eqlin_dtype_t dtype = EQLIN_F32;
   int device = 0;
@@ -283,6 +285,16 @@ cudaError_t launch_simt_apply(const Handle& h, bool backward, const void* in, vo
 cudaError_t launch_simt_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db,
                            int64_t N, cudaStream_t st);
 size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp);
+// Token splits of the SIMT weight gradients (32 x 32 channel tiles).
+int simt_dw_splits(int64_t Cp, int64_t Dp, int64_t N);
+
+// Dihedral groups D_m (eqlin_dihedral.cu), FP32 CUDA-core kernels, every dtype.
+bool dihedral_supported(int m);
+cudaError_t launch_dihedral_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st);
+cudaError_t launch_dihedral_apply(const Handle& h, bool backward, const void* in, void* out, int64_t N,
+                                  cudaStream_t st);
+cudaError_t launch_dihedral_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db, int64_t N,
+                               cudaStream_t st);
 // Sum per-split partial Fourier planes ([splits][T][Dp][Cp], or
 // [splits][T][Cp][Dp] when cd_layout) and db partials [splits][Dp] in split
 // order and apply the inverse DFT -> dW [Dp][Cp][T].

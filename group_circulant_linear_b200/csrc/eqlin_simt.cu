@@ -445,6 +445,8 @@ static int dw_splits(int64_t Cp, int64_t Dp, int64_t N) {
   return s < 1 ? 1 : (int)s;
 }
 
+int simt_dw_splits(int64_t Cp, int64_t Dp, int64_t N) { return dw_splits(Cp, Dp, N); }
+
 size_t simt_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp) {
   const int64_t s = dw_splits(Cp, Dp, INT64_MAX / 2);
   return (size_t)s * ((size_t)T * Cp * Dp + Dp) * sizeof(float);

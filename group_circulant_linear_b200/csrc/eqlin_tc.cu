@@ -767,6 +767,7 @@ static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out
 }  // namespace tc
 
 bool tc_supported(const Handle& h, bool backward) {
+  if (h.group != EQLIN_GROUP_CYCLIC) return false;
   if (h.dtype != EQLIN_F16 && h.dtype != EQLIN_BF16) return false;
   if (h.T != 1 && h.T != 2 && h.T != 4 && h.T != 8) return false;
   const int64_t K = backward ? h.Dp : h.Cp;

@@ -573,7 +573,7 @@ static cudaError_t launch_e(const Handle& h, const void* x, const void* gy, floa
 }  // namespace tcdw
 
 bool tc_dw_supported(const Handle& h) {
-  return (h.dtype == EQLIN_F16 || h.dtype == EQLIN_BF16) &&
+  return h.group == EQLIN_GROUP_CYCLIC && (h.dtype == EQLIN_F16 || h.dtype == EQLIN_BF16) &&
          (h.T == 1 || h.T == 2 || h.T == 4 || h.T == 8);
 }
 

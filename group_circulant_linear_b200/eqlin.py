@@ -18,6 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libeqlin.so")
 
 F32, F16, BF16 = 0, 1, 2
+CYCLIC, DIHEDRAL = 0, 1
+_GROUPS = {"cyclic": CYCLIC, "dihedral": DIHEDRAL}
 _DT = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 _TORCH_DT = {v: k for k, v in _DT.items()}
 _NAMES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
@@ -30,6 +32,7 @@ STATUS = {0: "EQLIN_OK", -1: "EQLIN_ERR_INVALID_ARG", -2: "EQLIN_ERR_UNSUPPORTED
 _vp, _i64, _int, _u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32
 SIGNATURES = {
     "eqlin_create": ([_int, _i64, _i64, _int, ctypes.POINTER(_vp)], _int),
+    "eqlin_create_group": ([_int, _int, _i64, _i64, _int, ctypes.POINTER(_vp)], _int),
     "eqlin_set_weights": ([_vp, _vp, _vp, _vp], _int),
     "eqlin_forward": ([_vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_backward_dx": ([_vp, _vp, _vp, _i64, _vp], _int),
@@ -99,15 +102,26 @@ def _dev_ptr(t: torch.Tensor, dtype, shape, name):
 
 
 class Handle:
-    """An eqlin_t plus the layer shape it was created for."""
+    """An eqlin_t plus the layer shape it was created for.
 
-    def __init__(self, T: int, Cp: int, Dp: int, dtype):
+    ``T`` is the group order (the length of the group axis).  For
+    ``group="dihedral"`` pass ``m`` (D_m, order 2m) and T = 2m, or T = None."""
+
+    def __init__(self, T, Cp: int, Dp: int, dtype, group="cyclic", m: int | None = None):
         if isinstance(dtype, str):
             dtype = _NAMES[dtype]
+        self.group = _GROUPS[group] if isinstance(group, str) else int(group)
+        if self.group == DIHEDRAL:
+            if m is None:
+                m = int(T) // 2
+            self.m = int(m)
+            T = 2 * self.m
+        else:
+            self.m = int(T)
         self.T, self.Cp, self.Dp, self.dtype = int(T), int(Cp), int(Dp), dtype
         out = ctypes.c_void_p()
-        _check(lib().eqlin_create(self.T, self.Cp, self.Dp, _DT[dtype], ctypes.byref(out)),
-               "eqlin_create")
+        _check(lib().eqlin_create_group(self.group, self.m, self.Cp, self.Dp, _DT[dtype], ctypes.byref(out)),
+               "eqlin_create_group")
         self._h = out
 
     @property
@@ -133,13 +147,19 @@ class Handle:
 
     def __deepcopy__(self, memo):
         # a new handle of the same shape; it holds no weights until set_weights
-        return Handle(self.T, self.Cp, self.Dp, self.dtype)
+        return Handle(self.T, self.Cp, self.Dp, self.dtype, group=self.group, m=self.m)
 
 
 # ------------------------------------------------------------------ the ABI
 
 def create(T: int, Cp: int, Dp: int, dtype) -> Handle:
     return Handle(T, Cp, Dp, dtype)
+
+
+def create_group(group, m: int, Cp: int, Dp: int, dtype) -> Handle:
+    """A layer over the cyclic group Z_m or the dihedral group D_m (order 2m)."""
+    g = _GROUPS[group] if isinstance(group, str) else int(group)
+    return Handle(m if g == CYCLIC else 2 * m, Cp, Dp, dtype, group=g, m=m)
 
 
 def set_weights(h: Handle, W: torch.Tensor, b: torch.Tensor | None = None, stream=None):
@@ -278,9 +298,12 @@ def destroy(h: Handle):
 class EQLinear:
     """Convenience wrapper: owns a handle and allocates outputs with torch."""
 
-    def __init__(self, W: torch.Tensor, b: torch.Tensor | None = None):
+    def __init__(self, W: torch.Tensor, b: torch.Tensor | None = None, group="cyclic"):
         Dp, Cp, T = W.shape
-        self.h = create(T, Cp, Dp, W.dtype)
+        if group == "dihedral":
+            self.h = create_group("dihedral", T // 2, Cp, Dp, W.dtype)
+        else:
+            self.h = create(T, Cp, Dp, W.dtype)
         self.set_weights(W, b)
 
     def set_weights(self, W, b=None, stream=None):

@@ -74,6 +74,11 @@ typedef enum {
     EQLIN_ERR_OOM = -7           /* device allocation failed */
 } eqlin_status_t;
 
+typedef enum {
+    EQLIN_GROUP_CYCLIC = 0,     /* Z_T, rotations by multiples of 2 pi / T (p4: T = 4) */
+    EQLIN_GROUP_DIHEDRAL = 1    /* D_m, rotations and reflections of a regular m-gon, order 2m */
+} eqlin_group_t;
+
 typedef struct eqlin_handle *eqlin_t;
 
 /*
@@ -85,6 +90,32 @@ typedef struct eqlin_handle *eqlin_t;
  */
 EQLIN_API eqlin_status_t eqlin_create(int T, int64_t Cp, int64_t Dp, eqlin_dtype_t dtype,
                             eqlin_t *out);
+
+/*
+ * A layer over another group: the group convolution
+ *
+ *   y[n, d*|G|+g] = b[d] + sum_c sum_h W[d, c, h^-1 g] * x[n, c*|G|+h]
+ *
+ * which for the cyclic group is the formula above ((s - t) mod T = h^-1 g).
+ * The paper names reflection groups as future work (technical summary,
+ * section "Limitacoes e Trabalho Futuro") without a formula; this is the
+ * plainest reading.
+ *   group = EQLIN_GROUP_CYCLIC, m = T: the same as eqlin_create(T, ...).
+ *   group = EQLIN_GROUP_DIHEDRAL, m in {1, 2, 3, 4, 5, 6, 8}: D_m of order
+ *     |G| = 2m, element r^a s^f (rotation by 2 pi a / m after f reflections)
+ *     at group index g = f*m + a; products follow from s r = r^-1 s.
+ *     Evaluated by the Fourier transform over D_m's real irreducible
+ *     representations (12 real channel GEMMs for D_4 against 64), in FP32
+ *     CUDA-core kernels for every dtype; the stash forms and
+ *     eqlin_backward_dw_noalloc are for cyclic groups only.
+ * Layouts and every other call are those of the cyclic layer with T = |G|:
+ * x [N, C'*|G|], y [N, D'*|G|], W [D', C', |G|], dW [D', C', |G|] with
+ *   dx[n, c*|G|+h] = sum_d sum_g W[d, c, h^-1 g] gy[n, d*|G|+g]
+ *   dW[d, c, u]    = sum_n sum_h x[n, c*|G|+h] gy[n, d*|G| + h u]
+ *   db[d]          = sum_n sum_g gy[n, d*|G|+g]
+ */
+EQLIN_API eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_t Dp,
+                                            eqlin_dtype_t dtype, eqlin_t *out);
 
 /*
  * Load weights: W [D', C', T] and b [D'] (b may be NULL: zero bias), device

@@ -56,6 +56,11 @@ def test_create_rejects_bad_arguments_before_touching_cuda():
     assert L.eqlin_create(4, 16, -1, eqlin.F32, ctypes.byref(out)) == -1
     assert L.eqlin_create(4, 16, 16, 7, ctypes.byref(out)) == -1
     assert L.eqlin_create(4, 16, 16, eqlin.F32, None) == -1
+    assert L.eqlin_create_group(2, 4, 16, 16, eqlin.F32, ctypes.byref(out)) == -1   # no such group
+    assert L.eqlin_create_group(eqlin.DIHEDRAL, 7, 16, 16, eqlin.F32, ctypes.byref(out)) == -2
+    assert L.eqlin_create_group(eqlin.DIHEDRAL, 0, 16, 16, eqlin.F32, ctypes.byref(out)) == -2
+    assert L.eqlin_create_group(eqlin.CYCLIC, 5, 16, 16, eqlin.F32, ctypes.byref(out)) == -2
+    assert L.eqlin_create_group(eqlin.DIHEDRAL, 1, 3, 8, eqlin.F16, ctypes.byref(out)) == -3  # 12-byte rows
     assert L.eqlin_create(1, 3, 8, eqlin.F16, ctypes.byref(out)) == -3     # 6-byte rows
     assert out.value is None
 
