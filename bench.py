@@ -461,11 +461,12 @@ def main(argv=None):
     eqlin = state.eqlin
     st = state.st
 
-    # dW/db of a layer runs on a second stream.  Plain path: it reads the same
-    # inputs as dx and writes nothing dx reads, so it starts beside dx and its
-    # CTAs take the SMs of dx's last, partial wave.  Fused path: it reads the
-    # spectrum dx writes, so it starts after dx and runs beside the next
-    # layer's weight transform and forward.  The main stream waits for it
+    # A step runs in training order: every layer's weight transform and
+    # forward, then the layers' backward passes in reverse.  dW/db of a layer
+    # runs on a second stream.  Plain path: it reads the same inputs as dx and
+    # writes nothing dx reads, so it starts beside that dx.  Fused path: it
+    # reads the spectrum its dx writes, so it starts after that dx and runs
+    # beside the next backward layer's dx.  The main stream waits for it
     # before each step ends (and before an all-reduce of dW/db).
     side = torch.cuda.Stream(device=dev)
 
@@ -473,6 +474,7 @@ def main(argv=None):
         for s in st:
             state.call(s, "set_weights", i)
             state.call(s, "fwd", i)
+        for s in reversed(st):
             if not fused:
                 side.wait_stream(stream)
             state.call(s, "dx", i)
@@ -611,11 +613,12 @@ def main(argv=None):
         "workload": args.workload,
         "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes)) for L in layers],
         "path": args.path,
-        "step": ("per layer: set_weights (weight DFT) + forward writing X = DFT(x) + dx writing G = DFT(gy) "
-                 "+ dW/db from the spectra on a second stream beside the next layer"
+        "step": ("every layer: set_weights (weight DFT) + forward writing X = DFT(x); then in reverse layer "
+                 "order: dx writing G = DFT(gy), and dW/db from the spectra on a second stream beside the next "
+                 "layer's dx"
                  if fused else
-                 "per layer: set_weights (weight DFT) + forward + dx + dW/db (transforming x and gy), "
-                 "dW/db on a second stream beside dx") + (" + NCCL all-reduce of dW/db" if dist else ""),
+                 "every layer: set_weights (weight DFT) + forward; then in reverse layer order: dx, and dW/db "
+                 "(transforming x and gy) on a second stream beside it") + (" + NCCL all-reduce of dW/db" if dist else ""),
         "tokens_per_gpu": layers[0].N,
         "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
               f"({N_SETS * set_bytes / 1e6:.0f} MB > 126 MB L2)",

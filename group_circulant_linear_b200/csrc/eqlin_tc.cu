@@ -2,11 +2,8 @@
 // forward pass and the input gradient, f16/bf16 in, f32 accumulation.
 //
 // One persistent CTA per SM walks output tiles of 128 tokens x BO output
-// channels (all T group positions), tile t = (output tile t / token blocks,
-// token block t % token blocks), CTA b taking tiles b, b + grid, ...: the CTAs
-// of one wave share an output tile's weights, and the stash forms' stores
-// (output tile 0 only) spread over the CTAs.  Per tile and per K stage of 16
-// input channels:
+// channels (all T group positions).  Per tile and per K stage of 16 input
+// channels:
 //
 //   raw producer     (8)    TMA: the raw input tile of the stage [128 tokens x
 //                    16*T elements] into the raw ring; L2 prefetches of raw
@@ -159,7 +156,7 @@ struct Params {
   int K;           // input channels per group element (C' forward, D' for dx)
   int O;           // output channels per group element
   int n_otiles;
-  int n_tb;        // 128-token blocks; tile t covers token block t % n_tb, output tile t / n_tb
+  int n_tb;        // 128-token blocks
   int64_t n_tiles;
   const void* in;
   const void* wtiles;  // tensor-core weight tiles (rows O, K) of this pass
@@ -230,8 +227,16 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t limit = p.wait_limit;
   const int nk = (p.K + C::BK - 1) / C::BK;
-  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...  Tile t covers
+  // (token block, output tile) = (t / n_otiles, t % n_otiles): the output tiles
+  // of one token block run side by side and share its input tile in L2.  The
+  // stash forms order them (t % n_tb, t / n_tb) instead: only output tile 0
+  // stores, and with the first order a CTA's tiles b, b + grid, ... all have
+  // the same output tile whenever n_otiles divides the grid, so half of the
+  // CTAs would do every store.
   const int64_t my_tiles = p.n_tiles > blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto tile_tb = [&](int tile) { return STASH ? tile % p.n_tb : tile / p.n_otiles; };
+  auto tile_ot = [&](int tile) { return STASH ? tile / p.n_tb : tile % p.n_otiles; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::RAW_ST; ++i) {
@@ -380,13 +385,13 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       auto prefetch_next = [&]() {
         if (pf_ti >= my_tiles) return;
         const int tile = (int)(blockIdx.x + pf_ti * gridDim.x);
-        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, (tile % p.n_tb) * C::BM);
+        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, tile_tb(tile) * C::BM);
         if (++pf_kb == nk) { pf_kb = 0; ++pf_ti; }
       };
       for (int i = 0; i < C::PF_STAGES; ++i) prefetch_next();
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const int m0 = (tile % p.n_tb) * C::BM;
+        const int m0 = tile_tb(tile) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
           prefetch_next();
           if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 2, 2), (uint32_t)n_raw)) { ok = false; break; }
@@ -411,7 +416,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       bool ok = true;
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)(tile / p.n_tb) * nk * C::B_BYTES;
+        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)tile_ot(tile) * nk * C::B_BYTES;
         for (int kb = 0; kb < nk; ++kb) {
           if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 3, 4), (uint32_t)n_b)) { ok = false; break; }
           // the stage's Q weight planes are one contiguous, pre-swizzled tile
@@ -512,8 +517,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       bool ok = true;
       for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
         const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const bool store = tile < p.n_tb;          // output tile 0
-        const int m0 = (tile % p.n_tb) * C::BM;
+        const bool store = tile_ot(tile) == 0;
+        const int m0 = tile_tb(tile) * C::BM;
         for (int kb = 0; kb < nk; ++kb) {
           if (!bwait(&a_ready[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 7), (uint32_t)(ti * nk + kb))) {
             ok = false;
@@ -569,7 +574,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       // this half's copy of the tile's bias, loaded while the MMAs run (the
       // half's previous tile has finished reading it)
       {
-        const int ob = (tile / p.n_tb) * C::BO;
+        const int ob = tile_ot(tile) * C::BO;
         for (int i = (e & 3) * 32 + lane; i < C::BO; i += 128)
           s_bias[half * C::BO + i] = (p.bias && ob + i < p.O) ? __ldg(p.bias + ob + i) : 0.f;
       }
@@ -578,8 +583,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane, p.err, site(K_APPLY, 5, 5), (uint32_t)ti));
       if (!got) { ok = false; break; }
       tc_fence_after();
-      const int m0 = (tile % p.n_tb) * C::BM;
-      const int o0 = (tile / p.n_tb) * C::BO;
+      const int m0 = tile_tb(tile) * C::BM;
+      const int o0 = tile_ot(tile) * C::BO;
       const uint32_t acc = tmem_base + lane_addr + ab * C::ACC_COLS;
 #pragma unroll 1
       for (int ci = half; ci < C::NCHUNK; ci += 2) {
