@@ -65,9 +65,12 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="skip the sub-measurements")
-    ap.add_argument("--path", choices=("fused", "plain"), default="fused",
+    ap.add_argument("--path", choices=("fused", "plain"), default="plain",
                     help="fused: forward and dx stash the spectra, dW from the spectra; "
                          "plain: dW transforms x and gy itself")
+    ap.add_argument("--order", choices=("layer", "training"), default="layer",
+                    help="layer: each layer's forward and backward in turn; training: every forward, "
+                         "then the backward passes in reverse layer order")
     return ap.parse_args(argv)
 
 
@@ -461,29 +464,39 @@ def main(argv=None):
     eqlin = state.eqlin
     st = state.st
 
-    # A step runs in training order: every layer's weight transform and
-    # forward, then the layers' backward passes in reverse.  dW/db of a layer
-    # runs on a second stream.  Plain path: it reads the same inputs as dx and
-    # writes nothing dx reads, so it starts beside that dx.  Fused path: it
-    # reads the spectrum its dx writes, so it starts after that dx and runs
-    # beside the next backward layer's dx.  The main stream waits for it
+    # A step runs every layer's weight transform, forward, dx and dW/db:
+    # layer by layer (--order layer), or every forward first and then the
+    # backward passes in reverse layer order (--order training).  dW/db of a
+    # layer runs on a second stream.  Plain path: it reads the same inputs as
+    # dx and writes nothing dx reads, so it starts beside that dx.  Fused path:
+    # it reads the spectrum its dx writes, so it starts after that dx and runs
+    # beside what follows on the main stream.  The main stream waits for it
     # before each step ends (and before an all-reduce of dW/db).
     side = torch.cuda.Stream(device=dev)
 
+    def backward(s, i):
+        if not fused:
+            side.wait_stream(stream)
+        state.call(s, "dx", i)
+        if fused:
+            side.wait_stream(stream)
+        state.call(s, "dw", i, stream=side)
+        if dist:
+            stream.wait_stream(side)
+            dp.allreduce_grads((s["dW"], s["db"]))
+
     def step(i):
-        for s in st:
-            state.call(s, "set_weights", i)
-            state.call(s, "fwd", i)
-        for s in reversed(st):
-            if not fused:
-                side.wait_stream(stream)
-            state.call(s, "dx", i)
-            if fused:
-                side.wait_stream(stream)
-            state.call(s, "dw", i, stream=side)
-            if dist:
-                stream.wait_stream(side)
-                dp.allreduce_grads((s["dW"], s["db"]))
+        if args.order == "layer":
+            for s in st:
+                state.call(s, "set_weights", i)
+                state.call(s, "fwd", i)
+                backward(s, i)
+        else:
+            for s in st:
+                state.call(s, "set_weights", i)
+                state.call(s, "fwd", i)
+            for s in reversed(st):
+                backward(s, i)
         stream.wait_stream(side)
 
     def barrier():
@@ -613,12 +626,15 @@ def main(argv=None):
         "workload": args.workload,
         "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes)) for L in layers],
         "path": args.path,
-        "step": ("every layer: set_weights (weight DFT) + forward writing X = DFT(x); then in reverse layer "
-                 "order: dx writing G = DFT(gy), and dW/db from the spectra on a second stream beside the next "
-                 "layer's dx"
-                 if fused else
-                 "every layer: set_weights (weight DFT) + forward; then in reverse layer order: dx, and dW/db "
-                 "(transforming x and gy) on a second stream beside it") + (" + NCCL all-reduce of dW/db" if dist else ""),
+        "order": args.order,
+        "step": ("per layer: set_weights (weight DFT), forward"
+                 + (" writing X = DFT(x)" if fused else "")
+                 + ", dx" + (" writing G = DFT(gy)" if fused else "")
+                 + ", dW/db" + (" from the spectra, after dx" if fused else " transforming x and gy, beside dx")
+                 + " on a second stream; "
+                 + ("layer by layer" if args.order == "layer"
+                    else "every forward first, then the backward passes in reverse layer order")
+                 + (" + NCCL all-reduce of dW/db" if dist else "")),
         "tokens_per_gpu": layers[0].N,
         "l2": f"inputs rotate over {N_SETS} sets of {set_bytes / 1e6:.0f} MB each "
               f"({N_SETS * set_bytes / 1e6:.0f} MB > 126 MB L2)",
