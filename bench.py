@@ -542,7 +542,8 @@ def main(argv=None):
     dom = max(per, key=per.get)
     Ld = layers[dom[0]]
     roof = roofline_of(Ld, dom[1], per[dom], pk, fused)
-    kernel_of = {"fwd": "tc_apply", "dx": "tc_apply", "dw": "dws" if fused else "dw", "set_weights": "pretransform"}
+    apply_k = "tc_apply_stash" if fused else "tc_apply"
+    kernel_of = {"fwd": apply_k, "dx": apply_k, "dw": "dws" if fused else "dw", "set_weights": "pretransform"}
     key = f"{kernel_of[dom[1]]}:{Ld.name}:{dom[1]}"
     roof["kernel"] = key
     roof["peak_kind"] = (f"{pk['source']} " + ("bf16 dense, burst (call timed in a sub-second region)"
