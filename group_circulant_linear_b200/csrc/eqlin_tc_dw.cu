@@ -54,13 +54,20 @@ namespace tcdw {
 using namespace ptx;
 using namespace waits;
 
-template <int T>
+// BCM caps the N-side tile width: 128 in general; 32 for small-channel shapes
+// (an N side of at most 32 channels, as the EQ-Swin-T stage-1 layers have).
+// Those take 32 tokens per stage for T <= 4 (two MMA K steps, 64-byte K-major
+// rows with the 64B swizzle): each stage then carries twice the work for the same fixed
+// cost of its barriers and commit, which is what bounds a stage whose MMAs
+// are this small.
+template <int T, int BCM = 128>
 struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                          // M channels per tile (MMA M)
-  static constexpr int BKN = 16;                          // tokens per stage (one MMA K step)
-  static constexpr int ROWB = BKN * 2;                    // 32-byte K-major rows, 32B swizzle
-  static constexpr int BC_MAX = (512 / T) < 128 ? (512 / T) : 128;
+  static constexpr int BKN = BCM <= 32 && T <= 4 ? 32 : 16;   // tokens per stage (BKN / 16 MMA K steps)
+  static constexpr int NSB = BKN / 16;                    // 8-token blocks per transform thread and stage
+  static constexpr int ROWB = BKN * 2;                    // K-major rows of 32 or 64 bytes, swizzled as wide
+  static constexpr int BC_MAX = (512 / T) < BCM ? (512 / T) : BCM;
   static constexpr int Q = G::nreal + 3 * G::ncomplex;    // B planes
   static constexpr int A_PLANE_BYTES = BM * ROWB;
   static constexpr int A_BYTES = T * A_PLANE_BYTES;
@@ -71,9 +78,12 @@ struct Cfg {
   static constexpr int NB_ROWB_MAX = BC_MAX * T * 2;
   static constexpr int RAW_BYTES = BKN * (MA_ROWB + NB_ROWB_MAX);
   // three operand slots where three raw slots still fit (the transform writes
-  // stage k + 2 while the MMAs of k and k + 1 are in flight), else two; the
-  // rest of 220 KB for raw slots (memory latency)
-  static constexpr int OP_STAGES = (220 * 1024 - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3 : 2;
+  // stage k + 2 while the MMAs of k and k + 1 are in flight), four where four
+  // raw slots still fit beside them, else two; the rest of 220 KB for raw
+  // slots (memory latency)
+  static constexpr int OP_STAGES = (220 * 1024 - 4 * OP_BYTES) / RAW_BYTES >= 4   ? 4
+                                   : (220 * 1024 - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3
+                                                                                  : 2;
   static constexpr int RAW_FIT = (220 * 1024 - OP_STAGES * OP_BYTES) / RAW_BYTES;
   static constexpr int RAW_STAGES = RAW_FIT > 6 ? 6 : RAW_FIT;
   static_assert(RAW_STAGES >= 2, "two raw stages must fit");
@@ -123,15 +133,19 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return u;
 }
 
-// Byte offset of the 16-byte chunk j (8 tokens) of row r in a 32B-swizzled K-major plane.
+// Byte offset of the 16-byte chunk j (8 tokens) of row r in a K-major plane
+// with ROWB-byte rows: 32B swizzle (chunk bit 0 XOR row bit 2) for 32-byte
+// rows, 64B swizzle (chunk bits 0-1 XOR row bits 1-2) for 64-byte rows.
+template <int ROWB>
 __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
-  return (uint32_t)(r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+  if constexpr (ROWB == 32) return (uint32_t)(r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+  else return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
-template <int T, typename E>
-__global__ void __launch_bounds__(Cfg<T>::THREADS, 1)
+template <int T, typename E, int BCM>
+__global__ void __launch_bounds__(Cfg<T, BCM>::THREADS, 1)
 tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_n, Params p) {
-  using C = Cfg<T>;
+  using C = Cfg<T, BCM>;
   using G = Group<T>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -190,7 +204,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
 
   if (warp < C::TR_WARPS) {
     // --------------------------------------------------- transform warps
-    const int grp = warp >> 3;                             // token group: tokens 8*grp .. 8*grp+7
+    const int grp = warp >> 3;                             // token group: tokens 8*NSB*grp .. 8*NSB*(grp+1)-1
     const bool is_a = (warp & 7) < 4;
     const int r = (warp & 3) * 32 + lane;                  // operand row: M channel (A) or N channel (B)
     const bool active = is_a || r < BC;
@@ -202,17 +216,20 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
                                   : (uint32_t)((r * T / p.nb_box) * C::BKN * p.nb_box * 2 +
                                                ((r * T) % p.nb_box) * 2);
     const uint32_t raw_rowb = is_a ? (uint32_t)(C::MA_BOX * 2) : (uint32_t)(p.nb_box * 2);
-    const uint32_t raw_base = (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + grp * 8 * raw_rowb;
-    const uint32_t off = kmajor_off(r, grp);
+    const uint32_t raw_base =
+        (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + grp * C::NSB * 8 * raw_rowb;
     float dbacc = 0.f;
     int rs = 0, os = 0;
     uint32_t rph = 0, oph = 0;
     bool ok = true;
     for (int st = 0; st < nst; ++st) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_DW, 1, 1), (uint32_t)st)) { ok = false; break; }
+      uint32_t Pw[C::NSB][T][4];
+#pragma unroll
+      for (int sb = 0; sb < C::NSB; ++sb) {
       uint32_t wv[8][C::W];
       if (active) {
-        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
+        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base + sb * 8 * raw_rowb;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint8_t* src = raw + j * raw_rowb;
@@ -229,7 +246,6 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
           }
         }
       }
-      uint32_t Pw[T][4];
       if (active) {
         if constexpr (T <= 4) {
 #pragma unroll
@@ -237,7 +253,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
             uint32_t P[T];
             packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
 #pragma unroll
-            for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
+            for (int q = 0; q < T; ++q) Pw[sb][q][pr] = P[q];
             if (sums_db) {
               const float2 f = packed::Pair<E>::to_f2(P[0]);
               dbacc += f.x + f.y;
@@ -258,36 +274,42 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
 #pragma unroll
             for (int q = 0; q < T; ++q) {
               E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
-              Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
+              Pw[sb][q][pr] = *reinterpret_cast<const uint32_t*>(two);
             }
           }
         }
+      }
       }
       // the operand slot must have been consumed by the MMAs issued from it
       if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
       if (active) {
         uint8_t* a_st = op_buf + os * C::OP_BYTES;
         uint8_t* b_st = a_st + C::A_BYTES;
-        if (is_a) {
 #pragma unroll
-          for (int q = 0; q < T; ++q)
-            *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
-                make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
-        } else {
+        for (int sb = 0; sb < C::NSB; ++sb) {
+          const uint32_t off = kmajor_off<C::ROWB>(r, grp * C::NSB + sb);
+          if (is_a) {
 #pragma unroll
-          for (int f = 0; f < G::nreal; ++f)
-            *reinterpret_cast<uint4*>(b_st + f * b_plane + off) = make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
+            for (int q = 0; q < T; ++q)
+              *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
+                  make_uint4(Pw[sb][q][0], Pw[sb][q][1], Pw[sb][q][2], Pw[sb][q][3]);
+          } else {
 #pragma unroll
-          for (int k = 1; k <= G::ncomplex; ++k) {
-            const int pr = G::nreal + 2 * (k - 1);
-            const int q = G::nreal + 3 * (k - 1);
-            // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G)
-            const uint32_t* u0 = swap ? Pw[pr] : Pw[pr + 1];
-            const uint32_t* u1 = swap ? Pw[pr + 1] : Pw[pr];
-            *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-            *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-            *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
-                make_uint4(packed::neg2(u0[0]), packed::neg2(u0[1]), packed::neg2(u0[2]), packed::neg2(u0[3]));
+            for (int f = 0; f < G::nreal; ++f)
+              *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
+                  make_uint4(Pw[sb][f][0], Pw[sb][f][1], Pw[sb][f][2], Pw[sb][f][3]);
+#pragma unroll
+            for (int k = 1; k <= G::ncomplex; ++k) {
+              const int pr = G::nreal + 2 * (k - 1);
+              const int q = G::nreal + 3 * (k - 1);
+              // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G)
+              const uint32_t* u0 = swap ? Pw[sb][pr] : Pw[sb][pr + 1];
+              const uint32_t* u1 = swap ? Pw[sb][pr + 1] : Pw[sb][pr];
+              *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+              *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(u1[0], u1[1], u1[2], u1[3]);
+              *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
+                  make_uint4(packed::neg2(u0[0]), packed::neg2(u0[1]), packed::neg2(u0[2]), packed::neg2(u0[3]));
+            }
           }
         }
       }
@@ -423,20 +445,25 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         const uint64_t a_d = desc0 + (uint64_t)((s * C::OP_BYTES) >> 4);
         const uint64_t b_d = a_d + (uint64_t)(C::A_BYTES >> 4);
         const uint32_t bp = b_plane >> 4;
-        const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
-        for (int f = 0; f < G::nreal; ++f)
-          if (C::own_real(f) == mi)
-            mma_f16_ss(tmem_base + f * BC, a_d + ((f * C::A_PLANE_BYTES) >> 4), b_d + f * bp, id_real, first);
+        for (int kk = 0; kk < C::BKN / 16; ++kk) {
+          // K step kk: 16 tokens = 32 bytes further along the swizzled rows
+          const uint64_t ka = a_d + (uint64_t)(kk * 2), kb = b_d + (uint64_t)(kk * 2);
+          const uint32_t first = (st > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
-        for (int k = 1; k <= G::ncomplex; ++k) {
-          if (C::own_cplx(k) != mi) continue;
-          const int pr = G::nreal + 2 * (k - 1);
-          const int q = G::nreal + 3 * (k - 1);
-          const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
-          // [Re | Im] += (Re plane of A) [first window] + (Im plane of A) [second window]
-          mma_f16_ss(col, a_d + ((pr * C::A_PLANE_BYTES) >> 4), b_d + (q + w1) * bp, id_cplx, first);
-          mma_f16_ss(col, a_d + (((pr + 1) * C::A_PLANE_BYTES) >> 4), b_d + (q + w2) * bp, id_cplx, 1u);
+          for (int f = 0; f < G::nreal; ++f)
+            if (C::own_real(f) == mi)
+              mma_f16_ss(tmem_base + f * BC, ka + ((f * C::A_PLANE_BYTES) >> 4), kb + f * bp, id_real, first);
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            if (C::own_cplx(k) != mi) continue;
+            const int pr = G::nreal + 2 * (k - 1);
+            const int q = G::nreal + 3 * (k - 1);
+            const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
+            // [Re | Im] += (Re plane of A) [first window] + (Im plane of A) [second window]
+            mma_f16_ss(col, ka + ((pr * C::A_PLANE_BYTES) >> 4), kb + (q + w1) * bp, id_cplx, first);
+            mma_f16_ss(col, ka + (((pr + 1) * C::A_PLANE_BYTES) >> 4), kb + (q + w2) * bp, id_cplx, 1u);
+          }
         }
         mma_commit(&op_empty[s]);
         if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
@@ -473,9 +500,9 @@ struct Plan {
 
 // M side: d, unless c pads less to a multiple of 128.  N side: tiles of BC
 // channels (a multiple of 16, at most BC_MAX) that split it evenly.
-template <int T>
+template <int T, int BCM = 128>
 static Plan plan(int64_t Cp, int64_t Dp, int64_t N, int sm_count) {
-  using C = Cfg<T>;
+  using C = Cfg<T, BCM>;
   Plan pl;
   const int64_t pad_d = (Dp + C::BM - 1) / C::BM * C::BM - Dp;
   const int64_t pad_c = (Cp + C::BM - 1) / C::BM * C::BM - Cp;
@@ -501,11 +528,10 @@ size_t workspace_bytes(int64_t Cp, int64_t Dp, int sm_count) {
   return (size_t)pl.splits * ((size_t)T * Cp * Dp + Dp) * sizeof(float);
 }
 
-template <int T, typename E>
-static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+template <int T, typename E, int BCM>
+static cudaError_t launch_b(const Handle& h, const Plan& pl, const void* x, const void* gy, float* dW, float* db,
                             int64_t N, cudaStream_t st) {
-  using C = Cfg<T>;
-  const Plan pl = plan<T>(h.Cp, h.Dp, N, h.sm_count);
+  using C = Cfg<T, BCM>;
   const size_t need = (size_t)pl.splits * ((size_t)T * h.Cp * h.Dp + h.Dp) * sizeof(float);
   if (need > h.ws_bytes) return cudaErrorInvalidValue;
   Params p;
@@ -547,15 +573,26 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
   }
   p.nb_box = nb_box;
   {
-    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(tc_dw_kernel<T, E>), C::SMEM_BYTES);
+    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(tc_dw_kernel<T, E, BCM>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
   const unsigned grid = (unsigned)(pl.n_mt * pl.n_nt * pl.splits);
-  cudaError_t e = launch_pdl(tc_dw_kernel<T, E>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, map_m, map_n, p);
+  cudaError_t e = launch_pdl(tc_dw_kernel<T, E, BCM>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, map_m, map_n, p);
   if (e != cudaSuccess) return e;
   count_launches(1);
   // partials are [N channel][M channel]: c-major over d when M = d
   return launch_dw_reduce(h, pl.splits, p.part, p.dbpart, dW, db, /*cd_layout=*/!pl.swap, st);
+}
+
+// The small-channel configuration serves N-side tiles of at most 32 channels;
+// the plan (tile widths, splits) is the same for both.
+template <int T, typename E>
+static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, float* dW, float* db,
+                            int64_t N, cudaStream_t st) {
+  const Plan pl = plan<T>(h.Cp, h.Dp, N, h.sm_count);
+  if (pl.BC <= Cfg<T, 32>::BC_MAX && Cfg<T, 32>::BC_MAX < Cfg<T>::BC_MAX)
+    return launch_b<T, E, 32>(h, plan<T, 32>(h.Cp, h.Dp, N, h.sm_count), x, gy, dW, db, N, st);
+  return launch_b<T, E, 128>(h, pl, x, gy, dW, db, N, st);
 }
 
 template <typename E>
