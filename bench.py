@@ -292,6 +292,11 @@ def pass_work(L, kind, fused=False):
     (fused path) also write the input's spectrum, as many elements as the input."""
     if kind == "set_weights":
         return 0, L.Dp * L.Cp * L.T * 2 * 2
+    if kind == "fwd_gauss":
+        # the three-product form: per complex frequency 3 real GEMMs, not 4
+        R = workloads.real_gemms(L.T)
+        n_complex = (L.T - 1) // 2
+        return L.actual_flop() * (R - n_complex) // R, L.bytes_fwd()
     e = workloads.BYTES[L.dtype]
     extra = 0
     if fused and kind == "fwd":
@@ -369,6 +374,8 @@ class Layers:
         inp = s["sets"][j]
         if kind == "set_weights":
             e.set_weights(s["h"], s["W"], s["b"], stream)
+        elif kind == "fwd_gauss":
+            e.forward_gauss(s["h"], inp["x"], s["y"], stream)
         elif kind == "fwd":
             if self.fused:
                 e.forward_stash(s["h"], inp["x"], s["y"], s["xs"][j], stream)
@@ -414,8 +421,12 @@ def sub_measurements(dev, pk, reps, fused):
     vit_b_f16 = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd",))
                  for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
     t8 = [L for L in workloads.WORKLOADS["cyclic-sweep-fwdbwd"] if L.T == 8 and L.dtype == "f16"]
+    gauss = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd", "fwd_gauss"))
+             for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
     subs = {
         "p4 FP16 forward, EQ-ViT-B MLP shapes": vit_b_f16,
+        # the complex products as four real GEMMs (fwd) or three (fwd_gauss, tiles of <= 96 channels)
+        "p4 FP16 forward, four- against three-product complex products": gauss,
         "EQ-Swin-T stage-1 step (f16)": workloads.WORKLOADS["eq-swin-t-s1-f16-fwdbwd"],
         "cyclic T=8 f16 layer": t8,
     }

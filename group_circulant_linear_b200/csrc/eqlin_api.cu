@@ -83,6 +83,8 @@ void free_all(Handle& h) {
   cudaFree(h.bias);
   cudaFree(h.ws);
   cudaFree(h.err);
+  cudaFree(h.wt_gauss);
+  h.wt_gauss = nullptr;
   h.wf_fwd = h.wf_bwd = nullptr;
   h.wt_fwd = h.wt_bwd = nullptr;
   h.bias = h.ws = nullptr;
@@ -171,6 +173,12 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
     ok = cudaMalloc(&h.wt_fwd, nf * e) == cudaSuccess && cudaMalloc(&h.wt_bwd, nb * e) == cudaSuccess;
     // padding rows and K columns of the tiles stay zero
     if (ok) ok = cudaMemset(h.wt_fwd, 0, nf * e) == cudaSuccess && cudaMemset(h.wt_bwd, 0, nb * e) == cudaSuccess;
+    // the p4 three-product forward image (eqlin_forward_gauss)
+    if (ok && T == 4 && eqlin::tc_supported(h, false) && eqlin::tc_supported(h, true)) {
+      h.bo_gauss = eqlin::tc_pick_bo_gauss(Dp);
+      const size_t ng = (size_t)eqlin::wtile_elems(T, h.bo_gauss, Dp, Cp);
+      ok = cudaMalloc(&h.wt_gauss, ng * e) == cudaSuccess && cudaMemset(h.wt_gauss, 0, ng * e) == cudaSuccess;
+    }
   }
   if (ok) ok = cudaMemset(h.err, 0, 4 * sizeof(int)) == cudaSuccess;
   if (!ok) {
@@ -222,6 +230,18 @@ eqlin_status_t eqlin_forward(eqlin_t hh, const void* x, void* y, int64_t N, void
     e = eqlin::launch_tc_apply(h, false, x, y, nullptr, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, false, x, y, N, (cudaStream_t)stream);
+  return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
+}
+
+eqlin_status_t eqlin_forward_gauss(eqlin_t hh, const void* x, void* y, int64_t N, void* stream) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  if (h.group != EQLIN_GROUP_CYCLIC || h.T != 4 || !h.wt_gauss) return EQLIN_ERR_UNSUPPORTED;
+  eqlin_status_t s = check_io(h, x, y, N);
+  if (s != EQLIN_OK || N == 0) return s;
+  DeviceGuard g(h.device);
+  if (!g.ok) return EQLIN_ERR_CUDA;
+  const cudaError_t e = eqlin::launch_tc_apply_gauss(h, x, y, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }
 

@@ -163,6 +163,17 @@ constexpr int TC_BK = 16;
 __host__ __device__ constexpr int tc_planes(int T) {
   return (T % 2 ? 1 : 2) + 3 * ((T - (T % 2 ? 1 : 2)) / 2);
 }
+// Tile width of the p4 three-product form: 96, 64 or 32, padding O least
+// (wider on a tie).
+inline int tc_pick_bo_gauss(int64_t O) {
+  int best = 96;
+  int64_t best_pad = (O + 95) / 96 * 96;
+  for (int bo : {64, 32}) {
+    const int64_t pad = (O + bo - 1) / bo * bo;
+    if (pad < best_pad) { best = bo; best_pad = pad; }
+  }
+  return best;
+}
 inline int tc_pick_bo(int T, int64_t O) {
   if (T == 1) return 256;
   if (T == 2) return 128;
@@ -219,6 +230,11 @@ struct Handle {
   void* wt_fwd = nullptr;
   void* wt_bwd = nullptr;
   int bo_fwd = 0, bo_bwd = 0;     // tile widths (output channels) of the two layouts
+  // p4 forward image for the three-product (Gauss) complex products, tile
+  // width bo_gauss (its five accumulators fit TMEM up to 96 channels);
+  // present for T = 4 handles whose passes both run on the tensor cores
+  void* wt_gauss = nullptr;
+  int bo_gauss = 0;
   bool need_simt_fwd = true;      // FP32 planes needed (SIMT serves forward / dx)
   bool need_simt_bwd = true;
   float* bias = nullptr;          // [Dp] float32 (zeros when no bias)
@@ -308,6 +324,9 @@ bool tc_supported(const Handle& h, bool backward);
 // writes the input's spectrum there (see spectra_ld).
 cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out, void* stash,
                             int64_t N, cudaStream_t st);
+// The p4 forward with the complex products in three real GEMMs (Gauss), for
+// comparison; needs the handle's Gauss image (h.wt_gauss).
+cudaError_t launch_tc_apply_gauss(const Handle& h, const void* in, void* out, int64_t N, cudaStream_t st);
 bool tc_dw_supported(const Handle& h);
 // dW, db from the spectra written by the stash forms (eqlin_tc_dws.cu).
 size_t tc_dws_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);

@@ -141,7 +141,8 @@ __device__ __forceinline__ void store8(E* dst, const float (&v)[8]) {
 template <int T, typename E>
 __global__ void __launch_bounds__(256)
 pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __restrict__ wt_fwd,
-                       E* __restrict__ wt_bwd, float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b) {
+                       E* __restrict__ wt_bwd, float* __restrict__ bias, int Cp, int Dp, int bo_f, int bo_b,
+                       E* __restrict__ wt_gauss, int bo_g) {
   using G = Group<T>;
   static_assert(sizeof(E) == 2, "tensor-core images hold 16-bit elements");
   grid_dep_launch();
@@ -231,6 +232,30 @@ pretransform_tc_kernel(const E* __restrict__ W, const E* __restrict__ b, E* __re
     for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? -s0 * (P[i][pr + 1] * sc) : 0.f;
     store8(out + wtile_index(T, bo, nkb, row, k0, q + 2), o);
   }
+  // The forward image for the three-product (Gauss) form of the complex
+  // products: real planes as above; per complex frequency (Re W, Im W - Re W,
+  // Re W + Im W), each formed in FP32 and rounded once.
+  if (fwd && wt_gauss) {
+#pragma unroll
+    for (int f = 0; f < G::nreal; ++f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? P[i][f] * sr : 0.f;
+      store8(wt_gauss + wtile_index(T, bo_g, nkb, row, k0, f), o);
+    }
+#pragma unroll
+    for (int k = 1; k <= G::ncomplex; ++k) {
+      const int pr = G::nreal + 2 * (k - 1), q = G::nreal + 3 * (k - 1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? P[i][pr] * sc : 0.f;
+      store8(wt_gauss + wtile_index(T, bo_g, nkb, row, k0, q + 0), o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? (P[i][pr + 1] - P[i][pr]) * sc : 0.f;
+      store8(wt_gauss + wtile_index(T, bo_g, nkb, row, k0, q + 1), o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = k0 + i < K ? (P[i][pr] + P[i][pr + 1]) * sc : 0.f;
+      store8(wt_gauss + wtile_index(T, bo_g, nkb, row, k0, q + 2), o);
+    }
+  }
 }
 
 template <int T, typename E>
@@ -241,7 +266,8 @@ static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b,
       const int64_t threads = n > h.Dp ? n : h.Dp;
       const cudaError_t e = launch_pdl(pretransform_tc_kernel<T, E>, dim3((unsigned)((threads + 255) / 256)),
                                        dim3(256), 0, st, (const E*)W, (const E*)b, (E*)h.wt_fwd, (E*)h.wt_bwd,
-                                       h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
+                                       h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd, (E*)h.wt_gauss,
+                                       h.bo_gauss);
       count_launches(1);
       return e;
     }

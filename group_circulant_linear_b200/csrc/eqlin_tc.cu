@@ -72,16 +72,25 @@ namespace tc {
 using namespace ptx;
 using namespace waits;
 
-template <int T, int BO_, bool STASH_ = false>
+// GAUSS_: the three-product form of the complex products (p4 only), for
+// comparison with the four-product form the paper counts: per complex
+// frequency k1 = (Re X + Im X) Re W, k2 = Re X (Im W - Re W), k3 = Im X (Re W
+// + Im W), Re Y = k1 - k3, Im Y = k1 + k2 -- five real GEMMs per p4 stage
+// instead of six, each N = BO, into five accumulators; the transform adds a
+// Re X + Im X plane.
+template <int T, int BO_, bool STASH_ = false, bool GAUSS_ = false>
 struct Cfg {
   using G = Group<T>;
+  static constexpr bool GAUSS = GAUSS_;
+  static_assert(!GAUSS || (T == 4 && !STASH_), "the three-product form is the p4 forward's");
+  static constexpr int NCX = GAUSS ? G::ncomplex : 0;      // extra A planes (Re X + Im X)
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
   static constexpr int BK = TC_BK;                     // input channels per stage (one MMA K step)
   // output channels per tile and accumulator buffers: T * BO * NACC <= 512 columns
   static constexpr int BO = BO_;
-  static_assert(T * BO <= 512 && (Group<T>::ncomplex == 0 || 2 * BO <= 256), "TMEM columns, MMA N");
-  static constexpr int NACC = (T * BO * 2 <= 512) ? 2 : 1;
-  static constexpr int ACC_COLS = T * BO;
+  static constexpr int ACC_COLS = (GAUSS ? G::nreal + 3 * G::ncomplex : T) * BO;
+  static_assert(ACC_COLS <= 512 && (Group<T>::ncomplex == 0 || 2 * BO <= 256), "TMEM columns, MMA N");
+  static constexpr int NACC = (ACC_COLS * 2 <= 512) ? 2 : 1;
   static constexpr int TMEM_COLS = NACC * ACC_COLS <= 256 ? 256 : 512;
   static constexpr int Q = G::nreal + 3 * G::ncomplex; // weight planes per stage
   // raw input tile of a stage: 128 tokens x (16 channels x T) elements, row-major (TMA)
@@ -91,7 +100,7 @@ struct Cfg {
   static constexpr int A_SBO = 1024;
   static constexpr int A_LBO = (BK / 8) * A_SBO;       // 2048
   static constexpr int A_PLANE_BYTES = BM * BK * 2;    // 4 KB
-  static constexpr int A_BYTES = T * A_PLANE_BYTES;
+  static constexpr int A_BYTES = (T + NCX) * A_PLANE_BYTES;
   // B: K-major, 32-byte rows (16 channels), 32B swizzle
   static constexpr int B_ROWB = BK * 2;
   static constexpr int B_PLANE_BYTES = BO * B_ROWB;
@@ -126,9 +135,11 @@ struct Cfg {
   // groups go to issuer 0 until it holds half of the stage's MMAs.
   static constexpr int NMMA = (T == 1) ? 1 : 2;
   static constexpr int MMAS = G::nreal + 2 * G::ncomplex;          // MMAs per stage
-  __host__ __device__ static constexpr int own_real(int f) { return (NMMA == 1 || 2 * f < MMAS) ? 0 : 1; }
+  __host__ __device__ static constexpr int own_real(int f) {
+    return (NMMA == 1 || GAUSS || 2 * f < MMAS) ? 0 : 1;
+  }
   __host__ __device__ static constexpr int own_cplx(int k) {
-    return (NMMA == 1 || 2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
+    return NMMA == 1 ? 0 : GAUSS ? 1 : (2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
   }
   static constexpr int NBAR = 2 * RAW_ST + 3 * AB_ST + 2 * NACC + NMMA;
   // per epilogue half, the bias of the tile's BO channels (FP32)
@@ -195,11 +206,11 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, u
   return d;
 }
 
-template <int T, int BO, typename E, bool STASH>
-__global__ void __launch_bounds__(Cfg<T, BO, STASH>::THREADS, 1)
+template <int T, int BO, typename E, bool STASH, bool GAUSS = false>
+__global__ void __launch_bounds__(Cfg<T, BO, STASH, GAUSS>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,
                 const __grid_constant__ CUtensorMap map_stash, Params p) {
-  using C = Cfg<T, BO, STASH>;
+  using C = Cfg<T, BO, STASH, GAUSS>;
   using G = Group<T>;
   grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -362,6 +373,20 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         for (int q = 0; q < T; ++q)
           *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + a_off[b]) =
               make_uint4(Pw[b][q][0], Pw[b][q][1], Pw[b][q][2], Pw[b][q][3]);
+      if constexpr (C::GAUSS) {
+        // Re X + Im X of each complex frequency (packed adds, one rounding)
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const int pr = G::nreal + 2 * (k - 1);
+            uint32_t sw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sw[i] = packed::Pair<E>::add(Pw[b][pr][i], Pw[b][pr + 1][i]);
+            *reinterpret_cast<uint4*>(a_st + (T + k - 1) * C::A_PLANE_BYTES + a_off[b]) =
+                make_uint4(sw[0], sw[1], sw[2], sw[3]);
+          }
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -477,6 +502,17 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
             if (C::own_cplx(k) != mi) continue;
             const int pr = G::nreal + 2 * (k - 1);
             const int q = G::nreal + 3 * (k - 1);
+            if constexpr (C::GAUSS) {
+              // k1 = (Re X + Im X) Re W, k2 = Re X (Im W - Re W), k3 = Im X (Re W + Im W)
+              const uint32_t kc = acc + (G::nreal + 3 * (k - 1)) * C::BO;
+              mma_f16_ss(kc, a_d + (((T + k - 1) * C::A_PLANE_BYTES) >> 4), b_d + ((q * C::B_PLANE_BYTES) >> 4),
+                         id_real, first);
+              mma_f16_ss(kc + C::BO, a_d + ((pr * C::A_PLANE_BYTES) >> 4),
+                         b_d + (((q + 1) * C::B_PLANE_BYTES) >> 4), id_real, first);
+              mma_f16_ss(kc + 2 * C::BO, a_d + (((pr + 1) * C::A_PLANE_BYTES) >> 4),
+                         b_d + (((q + 2) * C::B_PLANE_BYTES) >> 4), id_real, first);
+              continue;
+            }
             const uint32_t col = acc + G::nreal * C::BO + (k - 1) * 2 * C::BO;
             // [Re Y | Im Y] += Re X [Re W ; Im W]
             mma_f16_ss(col, a_d + ((pr * C::A_PLANE_BYTES) >> 4), b_d + (((q + 1) * C::B_PLANE_BYTES) >> 4),
@@ -595,20 +631,50 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
         named_bar_sync(1 + half, 128);
         // the chunk's T planes x CH channels (64 values) in one batch of TMEM loads
         uint32_t rg[T][C::CH];
+        if constexpr (C::GAUSS) {
+          // real planes, then per complex frequency k1 -> Re slot, k2 -> Im slot, k3 aside
+          uint32_t k3[G::ncomplex][C::CH];
 #pragma unroll
-        for (int q = 0; q < T; ++q) {
-          const int k = q < G::nreal ? 0 : 1 + (q - G::nreal) / 2;
-          const uint32_t col = acc + ci * C::CH +
-                               (q < G::nreal ? q * C::BO
-                                             : G::nreal * C::BO + (k - 1) * 2 * C::BO + ((q - G::nreal) & 1) * C::BO);
-          if constexpr (C::CH == 8) {
-            tmem_ld_32x32b_x8(col, *reinterpret_cast<uint32_t(*)[8]>(&rg[q][0]));
-          } else {
+          for (int q = 0; q < T; ++q) {
+            const int k = q < G::nreal ? 0 : 1 + (q - G::nreal) / 2;
+            const uint32_t col = acc + ci * C::CH +
+                                 (q < G::nreal ? q * C::BO : (G::nreal + 3 * (k - 1) + ((q - G::nreal) & 1)) * C::BO);
 #pragma unroll
             for (int h = 0; h < C::CH / 16; ++h) tmem_ld_32x32b_x16(col + 16 * h, &rg[q][16 * h]);
           }
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const uint32_t col = acc + ci * C::CH + (G::nreal + 3 * (k - 1) + 2) * C::BO;
+#pragma unroll
+            for (int h = 0; h < C::CH / 16; ++h) tmem_ld_32x32b_x16(col + 16 * h, &k3[k - 1][16 * h]);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const int pr = G::nreal + 2 * (k - 1);
+#pragma unroll
+            for (int j = 0; j < C::CH; ++j) {
+              const float k1 = __uint_as_float(rg[pr][j]), k2 = __uint_as_float(rg[pr + 1][j]);
+              rg[pr][j] = __float_as_uint(k1 - __uint_as_float(k3[k - 1][j]));     // Re Y
+              rg[pr + 1][j] = __float_as_uint(k1 + k2);                            // Im Y
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < T; ++q) {
+            const int k = q < G::nreal ? 0 : 1 + (q - G::nreal) / 2;
+            const uint32_t col = acc + ci * C::CH +
+                                 (q < G::nreal ? q * C::BO
+                                               : G::nreal * C::BO + (k - 1) * 2 * C::BO + ((q - G::nreal) & 1) * C::BO);
+            if constexpr (C::CH == 8) {
+              tmem_ld_32x32b_x8(col, *reinterpret_cast<uint32_t(*)[8]>(&rg[q][0]));
+            } else {
+#pragma unroll
+              for (int h = 0; h < C::CH / 16; ++h) tmem_ld_32x32b_x16(col + 16 * h, &rg[q][16 * h]);
+            }
+          }
+          tmem_wait_ld();
         }
-        tmem_wait_ld();
         if (ci + 2 >= C::NCHUNK) {
           // last TMEM read of this tile by this thread: release the accumulator
           tc_fence_before();
@@ -668,10 +734,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
-template <int T, int BO, typename E, bool STASH>
+template <int T, int BO, typename E, bool STASH, bool GAUSS = false>
 static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void* out, void* stash, int64_t N,
                             cudaStream_t st) {
-  using C = Cfg<T, BO, STASH>;
+  using C = Cfg<T, BO, STASH, GAUSS>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   const int K = (int)(backward ? h.Dp : h.Cp);
@@ -723,7 +789,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.n_tb = (int)((N + C::BM - 1) / C::BM);
   p.n_tiles = (int64_t)p.n_tb * p.n_otiles;
   p.in = in;
-  p.wtiles = backward ? h.wt_bwd : h.wt_fwd;
+  p.wtiles = GAUSS ? h.wt_gauss : backward ? h.wt_bwd : h.wt_fwd;
   p.bias = backward ? nullptr : h.bias;
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
@@ -731,12 +797,12 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
 
   {
     const cudaError_t e =
-        set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E, STASH>), C::SMEM_BYTES);
+        set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E, STASH, GAUSS>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
   int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
   if (grid < 1) grid = 1;
-  const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH>, dim3((unsigned)grid), dim3(C::THREADS),
+  const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH, GAUSS>, dim3((unsigned)grid), dim3(C::THREADS),
                                    C::SMEM_BYTES, st, map_in, map_out, map_stash, p);
   count_launches(1);
   return e;
@@ -780,6 +846,24 @@ bool tc_supported(const Handle& h, bool backward) {
   if (K % 8) return false;
   if (!tc::encode_fn()) return false;
   return true;
+}
+
+// The p4 forward in the three-product form (the handle's Gauss image).
+template <typename E>
+static cudaError_t launch_gauss_e(const Handle& h, const void* in, void* out, int64_t N, cudaStream_t st) {
+  switch (h.bo_gauss) {
+    case 96: return tc::launch_t<4, 96, E, false, true>(h, false, in, out, nullptr, N, st);
+    case 64: return tc::launch_t<4, 64, E, false, true>(h, false, in, out, nullptr, N, st);
+    case 32: return tc::launch_t<4, 32, E, false, true>(h, false, in, out, nullptr, N, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc_apply_gauss(const Handle& h, const void* in, void* out, int64_t N, cudaStream_t st) {
+  if (h.T != 4 || !h.wt_gauss) return cudaErrorNotSupported;
+  if (h.dtype == EQLIN_F16) return launch_gauss_e<__half>(h, in, out, N, st);
+  if (h.dtype == EQLIN_BF16) return launch_gauss_e<__nv_bfloat16>(h, in, out, N, st);
+  return cudaErrorNotSupported;
 }
 
 cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void* out, void* stash,

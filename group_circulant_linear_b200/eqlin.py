@@ -35,6 +35,7 @@ SIGNATURES = {
     "eqlin_create_group": ([_int, _int, _i64, _i64, _int, ctypes.POINTER(_vp)], _int),
     "eqlin_set_weights": ([_vp, _vp, _vp, _vp], _int),
     "eqlin_forward": ([_vp, _vp, _vp, _i64, _vp], _int),
+    "eqlin_forward_gauss": ([_vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_backward_dx": ([_vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_backward_dw": ([_vp, _vp, _vp, _vp, _vp, _i64, _vp], _int),
     "eqlin_get_error": ([_vp], _int),
@@ -173,6 +174,14 @@ def forward(h: Handle, x: torch.Tensor, y: torch.Tensor, stream=None):
     px = _dev_ptr(x, h.dtype, (N, h.Cp * h.T), "x")
     py = _dev_ptr(y, h.dtype, (N, h.Dp * h.T), "y")
     _check(lib().eqlin_forward(h.ptr, px, py, N, _stream(stream)), "eqlin_forward")
+
+
+def forward_gauss(h: Handle, x: torch.Tensor, y: torch.Tensor, stream=None):
+    """eqlin_forward with the complex products as three real GEMMs (p4 only)."""
+    N = x.shape[0]
+    px = _dev_ptr(x, h.dtype, (N, h.Cp * h.T), "x")
+    py = _dev_ptr(y, h.dtype, (N, h.Dp * h.T), "y")
+    _check(lib().eqlin_forward_gauss(h.ptr, px, py, N, _stream(stream)), "eqlin_forward_gauss")
 
 
 def backward_dx(h: Handle, gy: torch.Tensor, dx: torch.Tensor, stream=None):

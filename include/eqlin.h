@@ -130,6 +130,22 @@ EQLIN_API eqlin_status_t eqlin_set_weights(eqlin_t h, const void *W, const void 
 EQLIN_API eqlin_status_t eqlin_forward(eqlin_t h, const void *x, void *y, int64_t N, void *stream);
 
 /*
+ * The forward with each complex frequency's product in three real GEMMs
+ * instead of four (Gauss): with X = Xr + i Xi and W = Wr + i Wi,
+ *   k1 = (Xr + Xi) Wr,  k2 = Xr (Wi - Wr),  k3 = Xi (Wr + Wi),
+ *   Re(X W) = k1 - k3,  Im(X W) = k1 + k2,
+ * five real GEMMs per p4 layer instead of the six the paper counts
+ * (technical summary, section "Especializacao para o Grupo de Rotacao p4";
+ * the method's general-T form, section "Abordagem Algoritmica", leaves the
+ * complex product's evaluation open).  Same arguments and result as
+ * eqlin_forward up to rounding: Xr + Xi, Wi - Wr and Wr + Wi are each rounded
+ * to the dtype, and k1 - k3 and k1 + k2 cancel, so the error is somewhat
+ * larger.  Provided for comparison; T = 4, f16/bf16 handles whose passes both
+ * run on the tensor cores, else EQLIN_ERR_UNSUPPORTED.
+ */
+EQLIN_API eqlin_status_t eqlin_forward_gauss(eqlin_t h, const void *x, void *y, int64_t N, void *stream);
+
+/*
  * Input gradient: dx[n, c*T+t] = sum_d sum_s W[d, c, (s-t) mod T] gy[n, d*T+s].
  * gy [N, D'*T] -> dx [N, C'*T]; dx is overwritten.
  */

@@ -161,6 +161,60 @@ def test_integer_inputs_bit_exact(T, Cp, Dp, N, dt, amp):
         check_exact(f"{tag} stashed G", f["gs"][..., :N], np.rint(_spectrum(inp["gy"].double().numpy(), Dp, T)))
 
 
+# The p4 forward with the complex products as three real GEMMs (Gauss): against
+# the oracle (random inputs within the FP16/BF16 tolerance, integer inputs bit
+# for bit: Re X + Im X, Im W - Re W and Re W + Im W stay exact there), and
+# several tiles per CTA at N = 65536.
+GAUSS = [  # (C', D', N, dtype)
+    (192, 768, 1000, "bf16"), (768, 192, 777, "bf16"), (96, 288, 333, "f16"), (64, 96, 700, "bf16"),
+    (24, 96, 3000, "f16"), (16, 40, 129, "f16"),
+]
+GAUSS_EXACT = [  # (C', D', N, dtype, amp)
+    (16, 16, 700, "f16", 4), (16, 96, 65536, "f16", 2), (16, 64, 65536, "f16", 2), (8, 32, 300, "bf16", 1),
+]
+
+
+def _gauss_forward(inp):
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    N = g["x"].shape[0]
+    y = torch.empty((N, layer.h.Dp * 4), dtype=layer.h.dtype, device="cuda")
+    eqlin.forward_gauss(layer.h, g["x"], y)
+    y4 = layer.forward(g["x"])
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    return y.float().cpu().numpy(), y4.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("Cp,Dp,N,dt", GAUSS, ids=lambda v: str(v))
+def test_gauss_forward(Cp, Dp, N, dt):
+    inp = inputs.make_inputs(4, Cp, Dp, N, dt, seed=11, with_gy=False)
+    y3, y4 = _gauss_forward(inp)
+    ref = oracle.forward(inp["x"], inp["W"], inp["b"])
+    tag = f"gauss T=4 C'={Cp} D'={Dp} N={N} {dt}"
+    check(f"{tag} y", y3, ref, TOL[dt])
+    check(f"{tag} y (four-product form)", y4, ref, TOL[dt])
+
+
+@pytest.mark.parametrize("Cp,Dp,N,dt,amp", GAUSS_EXACT, ids=lambda v: str(v))
+def test_gauss_forward_integer_exact(Cp, Dp, N, dt, amp):
+    inp = inputs.make_integer_inputs(4, Cp, Dp, N, dt, seed=13, amp=amp)
+    y3, _ = _gauss_forward(inp)
+    check_exact(f"gauss integer T=4 C'={Cp} D'={Dp} N={N} {dt} y", y3, oracle.forward(inp["x"], inp["W"], inp["b"]))
+
+
+def test_gauss_forward_rejects_what_it_cannot_serve():
+    for T, dt in ((2, torch.bfloat16), (8, torch.float16), (4, torch.float32)):
+        h = eqlin.create(T, 16, 16, dt)
+        W = torch.zeros((16, 16, T), dtype=dt, device="cuda")
+        eqlin.set_weights(h, W, None)
+        x = torch.zeros((4, 16 * T), dtype=dt, device="cuda")
+        y = torch.empty((4, 16 * T), dtype=dt, device="cuda")
+        with pytest.raises(eqlin.EqlinError):
+            eqlin.forward_gauss(h, x, y)
+        h.close()
+
+
 FUSED = [  # (T, C', D', N, dtype): the stash forms and the one-call backward
     (4, 192, 768, 1000, "bf16"), (4, 768, 192, 777, "bf16"), (4, 24, 96, 3000, "f16"),
     (4, 96, 24, 3000, "f16"), (4, 96, 288, 333, "f16"), (2, 64, 48, 515, "bf16"),
