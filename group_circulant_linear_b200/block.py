@@ -120,8 +120,8 @@ class EQLinear(nn.Module):
         else:
             self.register_parameter("bias", None)
         self.h = eqlin.create(T, Cp, Dp, dtype)
-        # the stash forms serve handles whose every pass runs on the tensor cores
-        self.fused = self.h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
+        # the stash forms (fused backward) serve T | 8 layers whose passes all run on tensor cores
+        self.fused = self.h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05" and self.h.T in (1, 2, 4, 8)
         self._seen = None
 
     def sync_weights(self, W: torch.Tensor, b: torch.Tensor | None):

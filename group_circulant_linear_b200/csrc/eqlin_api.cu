@@ -153,7 +153,7 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
   }
   const size_t planes = (size_t)T * Cp * Dp;
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
-  if (!dihedral && dtype != EQLIN_F32 && T != 3 && T != 6) {
+  if (!dihedral && dtype != EQLIN_F32) {
     const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
     if (tcb > h.ws_bytes) h.ws_bytes = tcb;
     const size_t tcs = eqlin::tc_dws_workspace_bytes(T, Cp, Dp, h.sm_count);
@@ -283,6 +283,14 @@ eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, floa
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }
 
+// The stash forms and the weight gradient from spectra serve cyclic f16/bf16
+// layers of order T | 8 (the tensor-core kernels for T = 3 and 6 have no
+// stash form).
+static bool stash_order(const Handle& h) {
+  return h.group == EQLIN_GROUP_CYCLIC && h.dtype != EQLIN_F32 &&
+         (h.T == 1 || h.T == 2 || h.T == 4 || h.T == 8);
+}
+
 int64_t eqlin_spectra_ld(int64_t N) { return N < 0 ? -1 : eqlin::spectra_ld(N); }
 
 eqlin_status_t eqlin_forward_stash(eqlin_t hh, const void* x, void* y, void* xs, int64_t N, void* stream) {
@@ -292,7 +300,7 @@ eqlin_status_t eqlin_forward_stash(eqlin_t hh, const void* x, void* y, void* xs,
   if (s != EQLIN_OK || N == 0) return s;
   if (!xs) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(xs)) return EQLIN_ERR_MISALIGNED;
-  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, false))
+  if (!stash_order(h) || !eqlin::tc_supported(h, false))
     return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
@@ -307,7 +315,7 @@ eqlin_status_t eqlin_backward_dx_stash(eqlin_t hh, const void* gy, void* dx, voi
   if (s != EQLIN_OK || N == 0) return s;
   if (!gs) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(gs)) return EQLIN_ERR_MISALIGNED;
-  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_supported(h, true))
+  if (!stash_order(h) || !eqlin::tc_supported(h, true))
     return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;
@@ -321,7 +329,7 @@ eqlin_status_t eqlin_backward_dw_spectra(eqlin_t hh, const void* xs, const void*
   Handle& h = hh->h;
   if (!dW || N < 0) return EQLIN_ERR_INVALID_ARG;
   if (!aligned16(dW) || (db && !aligned16(db))) return EQLIN_ERR_MISALIGNED;
-  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32 || !eqlin::tc_dw_supported(h))
+  if (!stash_order(h) || !eqlin::tc_dw_supported(h))
     return EQLIN_ERR_UNSUPPORTED;
   DeviceGuard g(h.device);
   if (!g.ok) return EQLIN_ERR_CUDA;

@@ -177,6 +177,8 @@ inline int tc_pick_bo_gauss(int64_t O) {
 inline int tc_pick_bo(int T, int64_t O) {
   if (T == 1) return 256;
   if (T == 2) return 128;
+  if (T == 3) return 128;
+  if (T == 6) return 64;
   if (T == 8) return 32;
   int best = 128;
   int64_t best_pad = (O + 127) / 128 * 128;

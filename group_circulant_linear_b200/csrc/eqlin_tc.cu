@@ -105,9 +105,13 @@ struct Cfg {
   static constexpr int B_ROWB = BK * 2;
   static constexpr int B_PLANE_BYTES = BO * B_ROWB;
   static constexpr int B_BYTES = Q * B_PLANE_BYTES;
-  // output staging for the TMA stores: per epilogue half two [128 rows x 128 B] tiles
-  static constexpr int OUT_EL = 64;                    // output elements per row per store
-  static constexpr int OUT_TILE_BYTES = BM * OUT_EL * 2;
+  // output staging for the TMA stores: per epilogue half two [128 rows x
+  // OUT_EL elements] tiles; 64 elements (128 bytes, 128B swizzle) for T | 8,
+  // 48 (96 bytes, unswizzled) for T = 3 and 6
+  static constexpr bool POW2 = (T & (T - 1)) == 0;
+  static constexpr int OUT_EL = POW2 ? 64 : 48;        // output elements per row per store
+  static constexpr int OUT_ROWB = OUT_EL * 2;
+  static constexpr int OUT_TILE_BYTES = BM * OUT_ROWB;
   static constexpr int STAGING = 4 * OUT_TILE_BYTES;
   // ring depths: operand slots (the A planes of a stage and its weight
   // planes share one slot and one pair of barriers, so the MMA thread waits
@@ -148,6 +152,7 @@ struct Cfg {
                                     BIAS_BYTES + NBAR * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
   static constexpr int CH = OUT_EL / T;                // output channels per store chunk
+  static_assert(OUT_EL % T == 0 && CH % 8 == 0, "whole channels per store chunk, 8 at a time");
   static constexpr int NCHUNK = BO / CH;               // store chunks per tile (even)
   static_assert(NCHUNK % 2 == 0, "chunks alternate between the two epilogue halves");
   // roles
@@ -305,7 +310,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_APPLY, 1, 1), (uint32_t)it)) { ok = false; break; }
       const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_off;
       uint32_t Pw[2][T][4];
-      if constexpr (T <= 4) {
+      if constexpr (T == 1 || T == 2 || T == 4) {
         // all 16 tokens' words first, so the raw slot is released early
         uint32_t wv[16][C::W];
 #pragma unroll
@@ -334,7 +339,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
 #pragma unroll
             for (int q = 0; q < T; ++q) Pw[b][q][pr] = P[q];
           }
-      } else {
+      } else if constexpr (T == 8) {
         // T = 8: one block of 8 tokens at a time (registers), FP32 butterflies
         // with the sqrt(2)/2 twiddles, one rounding per value
 #pragma unroll
@@ -350,6 +355,28 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
             float Pa[T], Pb[T], va[T], vb[T];
             const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
             const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
+#pragma unroll
+            for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
+            G::dft(va, Pa);
+            G::dft(vb, Pb);
+#pragma unroll
+            for (int q = 0; q < T; ++q) Pw[b][q][pr] = pack2<E>(Pa[q], Pb[q]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
+      } else {
+        // T = 3, 6: a channel's T values are 6 or 12 bytes, read element by
+        // element, a pair of tokens at a time; FP32 butterflies with the
+        // sqrt(3)/2 twiddles, one rounding per value
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) {
+            const E* ea = reinterpret_cast<const E*>(raw + (8 * b + 2 * pr) * C::RAW_ROWB);
+            const E* eb = reinterpret_cast<const E*>(raw + (8 * b + 2 * pr + 1) * C::RAW_ROWB);
+            float Pa[T], Pb[T], va[T], vb[T];
 #pragma unroll
             for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
             G::dft(va, Pa);
@@ -625,7 +652,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
 #pragma unroll 1
       for (int ci = half; ci < C::NCHUNK; ci += 2) {
         uint8_t* stage_tile = o_buf + (half * 2 + sb) * C::OUT_TILE_BYTES;
-        uint8_t* my_row = stage_tile + r * 128;
+        uint8_t* my_row = stage_tile + r * C::OUT_ROWB;
         // the TMA store issued from this staging tile two chunks ago must have read it
         if (issuer) bulk_wait_read<1>();
         named_bar_sync(1 + half, 128);
@@ -690,21 +717,37 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
             bo8[0] = b0.x; bo8[1] = b0.y; bo8[2] = b0.z; bo8[3] = b0.w;
             bo8[4] = b1.x; bo8[5] = b1.y; bo8[6] = b1.z; bo8[7] = b1.w;
           }
-          // 8 channels x T outputs = T 16-byte chunks of this row's 128 bytes;
-          // chunk v holds the outputs of channels v*8/T .. (v+1)*8/T - 1
+          if constexpr (C::POW2) {
+            // 8 channels x T outputs = T 16-byte chunks of this row's 128 bytes;
+            // chunk v holds the outputs of channels v*8/T .. (v+1)*8/T - 1
 #pragma unroll
-          for (int v = 0; v < T; ++v) {
-            float vals[8];
+            for (int v = 0; v < T; ++v) {
+              float vals[8];
 #pragma unroll
-            for (int cc = 0; cc < 8 / T; ++cc) {
-              const int c = v * (8 / T) + cc;
+              for (int cc = 0; cc < 8 / T; ++cc) {
+                const int c = v * (8 / T) + cc;
+                float Pc[T];
+#pragma unroll
+                for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][sub * 8 + c]);
+                G::idft_scaled(Pc, bo8[c], vals + cc * T);
+              }
+              const int j = sub * T + v;
+              *reinterpret_cast<uint4*>(my_row + ((j ^ (r & 7)) << 4)) = pack8<E>(vals);
+            }
+          } else {
+            // T = 3, 6: the 8 channels' 8T outputs, then T 16-byte chunks of
+            // consecutive outputs (unswizzled rows of 96 bytes)
+            float vals[8 * T];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
               float Pc[T];
 #pragma unroll
               for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][sub * 8 + c]);
-              G::idft_scaled(Pc, bo8[c], vals + cc * T);
+              G::idft_scaled(Pc, bo8[c], vals + c * T);
             }
-            const int j = sub * T + v;
-            *reinterpret_cast<uint4*>(my_row + ((j ^ (r & 7)) << 4)) = pack8<E>(vals);
+#pragma unroll
+            for (int v = 0; v < T; ++v)
+              *reinterpret_cast<uint4*>(my_row + (sub * T + v) * 16) = pack8<E>(vals + 8 * v);
           }
         }
         fence_proxy_async_smem();
@@ -762,7 +805,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
     cuuint32_t box[2] = {(cuuint32_t)C::OUT_EL, (cuuint32_t)C::BM};
     cuuint32_t es[2] = {1, 1};
     if (enc(&map_out, dt, 2, out, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            C::POW2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
@@ -831,6 +874,9 @@ static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out
       }
       return cudaErrorInvalidValue;
     case 8: return bo == 32 ? launch_s<8, 32, E>(h, bwd, in, out, stash, N, st) : cudaErrorInvalidValue;
+    // T = 3, 6: no stash form
+    case 3: return bo == 128 && !stash ? launch_t<3, 128, E, false>(h, bwd, in, out, nullptr, N, st) : cudaErrorInvalidValue;
+    case 6: return bo == 64 && !stash ? launch_t<6, 64, E, false>(h, bwd, in, out, nullptr, N, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }
@@ -840,7 +886,7 @@ static cudaError_t launch_e(const Handle& h, bool bwd, const void* in, void* out
 bool tc_supported(const Handle& h, bool backward) {
   if (h.group != EQLIN_GROUP_CYCLIC) return false;
   if (h.dtype != EQLIN_F16 && h.dtype != EQLIN_BF16) return false;
-  if (h.T != 1 && h.T != 2 && h.T != 4 && h.T != 8) return false;
+  if (h.T != 1 && h.T != 2 && h.T != 3 && h.T != 4 && h.T != 6 && h.T != 8) return false;
   const int64_t K = backward ? h.Dp : h.Cp;
   // TMA row pitch of the weight planes (K * 2 bytes) must be a 16-byte multiple
   if (K % 8) return false;

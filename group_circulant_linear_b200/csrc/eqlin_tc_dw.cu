@@ -67,7 +67,8 @@ struct Cfg {
   static constexpr int BKN = BCM <= 32 && T <= 4 ? 32 : 16;   // tokens per stage (BKN / 16 MMA K steps)
   static constexpr int NSB = BKN / 16;                    // 8-token blocks per transform thread and stage
   static constexpr int ROWB = BKN * 2;                    // K-major rows of 32 or 64 bytes, swizzled as wide
-  static constexpr int BC_MAX = (512 / T) < BCM ? (512 / T) : BCM;
+  // T * BC_MAX TMEM columns; tile widths are multiples of 16
+  static constexpr int BC_MAX = (512 / T / 16 * 16) < BCM ? (512 / T / 16 * 16) : BCM;
   static constexpr int Q = G::nreal + 3 * G::ncomplex;    // B planes
   static constexpr int A_PLANE_BYTES = BM * ROWB;
   static constexpr int A_BYTES = T * A_PLANE_BYTES;
@@ -104,7 +105,9 @@ struct Cfg {
   static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;   // MMA warps MMA_WARP .. + NMMA - 1
   static constexpr int THREADS = (TR_WARPS + 1 + NMMA) * 32;
   static constexpr int PF_STAGES = 12;                    // L2 prefetch distance (stages)
-  static constexpr int MA_BOX = BM * T <= 256 ? BM * T : 256;   // M-side TMA box width (elements)
+  // M-side TMA box width (elements): a whole number of channels, at most 256
+  static constexpr int MA_BOX = BM * T <= 256 ? BM * T : (T & (T - 1)) == 0 ? 256 : 192;
+  static_assert((BM * T) % MA_BOX == 0 && MA_BOX % T == 0, "whole channels per box, whole boxes per tile");
   static constexpr int W = packed::Words<T>::n;
 };
 
@@ -228,8 +231,8 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
 #pragma unroll
       for (int sb = 0; sb < C::NSB; ++sb) {
       uint32_t wv[8][C::W];
-      if (active) {
-        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base + sb * 8 * raw_rowb;
+      const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base + sb * 8 * raw_rowb;
+      if (active && (T == 1 || T == 2 || T == 4 || T == 8)) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint8_t* src = raw + j * raw_rowb;
@@ -247,7 +250,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         }
       }
       if (active) {
-        if constexpr (T <= 4) {
+        if constexpr (T == 1 || T == 2 || T == 4) {
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
             uint32_t P[T];
@@ -260,12 +263,16 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
             }
           }
         } else {
-          // T = 8: FP32 butterflies (sqrt(2)/2 twiddles), one rounding per value
+          // T = 3, 6, 8: FP32 butterflies (sqrt(3)/2 or sqrt(2)/2 twiddles), one
+          // rounding per value; for T = 3, 6 (6 or 12 bytes per channel) the
+          // elements are read one by one
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
             float Pa[T], Pb[T], va[T], vb[T];
-            const E* ea = reinterpret_cast<const E*>(wv[2 * pr]);
-            const E* eb = reinterpret_cast<const E*>(wv[2 * pr + 1]);
+            const E* ea = T == 8 ? reinterpret_cast<const E*>(wv[2 * pr])
+                                 : reinterpret_cast<const E*>(raw + (2 * pr) * raw_rowb);
+            const E* eb = T == 8 ? reinterpret_cast<const E*>(wv[2 * pr + 1])
+                                 : reinterpret_cast<const E*>(raw + (2 * pr + 1) * raw_rowb);
 #pragma unroll
             for (int t = 0; t < T; ++t) { va[t] = Elem<E>::to_f(ea[t]); vb[t] = Elem<E>::to_f(eb[t]); }
             G::dft(va, Pa);
@@ -553,9 +560,17 @@ static cudaError_t launch_b(const Handle& h, const Plan& pl, const void* x, cons
   if (!enc) return cudaErrorNotSupported;
   const CUtensorMapDataType dt = std::is_same<E, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  // N-side box: the largest power-of-two width <= 256 elements that divides BC * T
+  // N-side box: whole channels, at most 256 elements, a multiple of 16 bytes,
+  // dividing BC * T: the largest power of two for T | 8; for T = 3, 6 the
+  // channels of the largest divisor of BC that fits
   int nb_box = 256;
-  while ((pl.BC * T) % nb_box) nb_box >>= 1;
+  if ((T & (T - 1)) == 0) {
+    while ((pl.BC * T) % nb_box) nb_box >>= 1;
+  } else {
+    int d = pl.BC;
+    while (d > 1 && (pl.BC % d || d * T > 256 || (d * T * 2) % 16)) --d;
+    nb_box = d * T;
+  }
   CUtensorMap map_m, map_n;
   const void* srcs[2] = {pl.swap ? x : gy, pl.swap ? gy : x};
   const int64_t widths[2] = {(pl.swap ? h.Cp : h.Dp) * T, (pl.swap ? h.Dp : h.Cp) * T};
@@ -601,7 +616,9 @@ static cudaError_t launch_e(const Handle& h, const void* x, const void* gy, floa
   switch (h.T) {
     case 1: return launch_t<1, E>(h, x, gy, dW, db, N, st);
     case 2: return launch_t<2, E>(h, x, gy, dW, db, N, st);
+    case 3: return launch_t<3, E>(h, x, gy, dW, db, N, st);
     case 4: return launch_t<4, E>(h, x, gy, dW, db, N, st);
+    case 6: return launch_t<6, E>(h, x, gy, dW, db, N, st);
     case 8: return launch_t<8, E>(h, x, gy, dW, db, N, st);
   }
   return cudaErrorInvalidValue;
@@ -611,14 +628,16 @@ static cudaError_t launch_e(const Handle& h, const void* x, const void* gy, floa
 
 bool tc_dw_supported(const Handle& h) {
   return h.group == EQLIN_GROUP_CYCLIC && (h.dtype == EQLIN_F16 || h.dtype == EQLIN_BF16) &&
-         (h.T == 1 || h.T == 2 || h.T == 4 || h.T == 8);
+         (h.T == 1 || h.T == 2 || h.T == 3 || h.T == 4 || h.T == 6 || h.T == 8);
 }
 
 size_t tc_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count) {
   switch (T) {
     case 1: return tcdw::workspace_bytes<1>(Cp, Dp, sm_count);
     case 2: return tcdw::workspace_bytes<2>(Cp, Dp, sm_count);
+    case 3: return tcdw::workspace_bytes<3>(Cp, Dp, sm_count);
     case 4: return tcdw::workspace_bytes<4>(Cp, Dp, sm_count);
+    case 6: return tcdw::workspace_bytes<6>(Cp, Dp, sm_count);
     case 8: return tcdw::workspace_bytes<8>(Cp, Dp, sm_count);
   }
   return 0;

@@ -36,8 +36,9 @@
  *   after the caller has synchronised the stream.
  * - N = 0 is a no-op that returns EQLIN_OK (dW and db are then zeroed).
  * - Supported T: 1, 2, 3, 4, 6, 8.  Other values give EQLIN_ERR_UNSUPPORTED.
- *   T = 3 and 6 (twiddles with sqrt(3)/2) run the FP32 SIMT kernels in every
- *   dtype; the tensor-core kernels serve f16/bf16 for T = 1, 2, 4, 8.
+ *   The tensor-core kernels serve f16/bf16 for every supported T (T = 3 and 6
+ *   with FP32 butterflies and the sqrt(3)/2 twiddles); FP32 handles run the
+ *   SIMT kernels.  The stash forms (fused backward) take T = 1, 2, 4, 8.
  *   eqlin_backward_dw_noalloc takes T = 1, 2, 4, 8 only.
  * - Nothing is thrown across the ABI; every call returns a status.
  * - A handle may be used from one host thread at a time.
@@ -288,9 +289,8 @@ EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
  * "fwd=<k> dx=<k> dw=<k>", where <k> is "tcgen05" (the tensor-core kernels)
  * or "simt" (the FP32 CUDA-core kernels).  f32 handles run simt for every
  * pass.  f16/bf16 handles run tcgen05 except where the shape rules it out:
- * T = 3 or 6 (all passes), or a forward (dx) whose K = C' (D') is not a
- * multiple of 8 -- the row pitch of that pass's weight tiles would not be a
- * TMA stride.  For logging and tests; the string lives as long as the handle.
+ * a forward (dx) whose K = C' (D') is not a multiple of 8 -- the row pitch of
+ * that pass's weight tiles would not be a TMA stride.  For logging and tests; the string lives as long as the handle.
  */
 EQLIN_API const char *eqlin_backend_name(eqlin_t h);
 

@@ -95,8 +95,12 @@ SMALL = [  # (T, C', D', N, dtype)
     (1, 64, 48, 200, "f32"), (1, 64, 48, 200, "bf16"),
     (8, 64, 16, 130, "bf16"), (2, 40, 72, 129, "bf16"),
     (4, 8, 8, 1, "f16"), (4, 200, 40, 131, "f16"),
-    # T = 3 and 6: sqrt(3)/2 twiddles, one real frequency for odd T (SIMT kernels)
+    # T = 3 and 6: sqrt(3)/2 twiddles, one real frequency for odd T (tensor cores
+    # for f16/bf16 with 8-aligned channels, SIMT otherwise), several tiles per CTA
     (3, 64, 48, 257, "f32"), (6, 32, 40, 130, "f32"), (3, 40, 64, 300, "bf16"), (6, 48, 24, 200, "f16"),
+    (3, 192, 768, 3000, "bf16"), (3, 768, 192, 1000, "f16"), (6, 128, 256, 5000, "f16"), (6, 256, 64, 777, "bf16"),
+    (3, 24, 96, 4000, "f16"), (6, 96, 24, 3000, "bf16"),
+    (6, 20, 36, 300, "bf16"),       # K not a multiple of 8: forward and dx on the SIMT kernels
 ]
 
 
@@ -304,12 +308,14 @@ def test_back_to_back_dependencies():
 
 @pytest.mark.parametrize("T,dt", [(3, "f32"), (6, "f32"), (3, "bf16"), (6, "f16")], ids=str)
 def test_odd_and_sixfold_groups_are_equivariant(T, dt):
-    """T = 3 and 6 run the SIMT kernels; a cyclic shift of the input's group
-    axis shifts the output's, and the backend says so."""
+    """T = 3 and 6 run the tensor-core kernels in f16/bf16 (the SIMT ones in
+    FP32); a cyclic shift of the input's group axis shifts the output's, and
+    the backend says which kernels ran."""
     Cp, Dp, N = 16, 24, 150
     inp = _dev(inputs.make_inputs(T, Cp, Dp, N, dt, seed=15))
     layer = eqlin.EQLinear(inp["W"], inp["b"])
-    assert layer.h.backend() == "fwd=simt dx=simt dw=simt"
+    want = "fwd=simt dx=simt dw=simt" if dt == "f32" else "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
+    assert layer.h.backend() == want
     y = layer.forward(inp["x"])
     tol = 1e-5 if dt == "f32" else TOL[dt]
     for r in range(1, T):
@@ -506,7 +512,7 @@ def test_backend_is_reported_per_pass():
     every pass; a pass whose K is not a multiple of 8 runs the SIMT kernels, and
     the handle says which pass."""
     for dt in ("f16", "bf16"):
-        for T in (1, 2, 4, 8):
+        for T in (1, 2, 3, 4, 6, 8):
             h = eqlin.create(T, 64, 64, dt)
             assert h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", (T, dt, h.backend())
             h.close()
