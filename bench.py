@@ -421,6 +421,9 @@ def sub_measurements(dev, pk, reps, fused):
     vit_b_f16 = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd",))
                  for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
     t8 = [L for L in workloads.WORKLOADS["cyclic-sweep-fwdbwd"] if L.T == 8 and L.dtype == "f16"]
+    # the orders with sqrt(3)/2 twiddles, at the sweep's N and about its width (C = C'T near 1024)
+    t36 = [workloads.Layer(f"cyclic T={T} f16", T, C, C, 16384, "f16", ("fwd", "dx", "dw"))
+           for T, C in ((3, 336), (6, 168))]
     gauss = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd", "fwd_gauss"))
              for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
     subs = {
@@ -429,6 +432,7 @@ def sub_measurements(dev, pk, reps, fused):
         "p4 FP16 forward, four- against three-product complex products": gauss,
         "EQ-Swin-T stage-1 step (f16)": workloads.WORKLOADS["eq-swin-t-s1-f16-fwdbwd"],
         "cyclic T=8 f16 layer": t8,
+        "cyclic T=3 and T=6 f16 layers": t36,
     }
     stream = torch.cuda.current_stream()
     for name, layers in subs.items():
