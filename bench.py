@@ -321,11 +321,26 @@ def roofline_of(L, kind, us, pk, fused=False):
     r = {"us": round(us, 2), "tflops": flop / t / 1e12 if flop else 0.0, "gbs": byt / t / 1e9,
          "frac_tensor": flop / t / tens if flop else 0.0, "frac_hbm": byt / t / hbm,
          "frac_roofline": max(flop / tens, byt / hbm) / t}
-    ridge = tens / hbm
-    if flop and flop / byt >= ridge / 2:
-        r.update(bound="tensor", achieved=r["tflops"], peak=pk["bf16"], unit="TFLOP/s", frac=r["frac_tensor"])
+    if L.dtype == "f32" and L.T in (1, 2, 4) and kind in ("fwd", "dx"):
+        # 3xTF32: three kind::tf32 MMAs per real product, against the TF32
+        # peak (the measured bf16 peak x the nominal TF32/BF16 ratio of 1/2)
+        mma_flop, peak = 3 * flop, pk["bf16"] / 2
+        r.update(bound="tensor", achieved=mma_flop / t / 1e12, peak=peak, unit="TFLOP/s (tf32 MMA)",
+                 frac=mma_flop / t / (peak * 1e12), fp32_equiv_tflops=r["tflops"],
+                 frac_hbm=byt / t / hbm)
+        r["frac_roofline"] = max(mma_flop / (peak * 1e12), byt / hbm) / t
+    elif L.dtype == "f32":
+        # FP32 on the CUDA cores: FFMA peak 148 SMs x 128 lanes x 2 x 1965 MHz (nominal)
+        ffma = 148 * 128 * 2 * 1.965e9
+        r.update(bound="alu", achieved=r["tflops"], peak=ffma / 1e12, unit="TFLOP/s (FFMA)",
+                 frac=flop / t / ffma)
+        r["frac_roofline"] = max(flop / ffma, byt / hbm) / t
     else:
-        r.update(bound="hbm", achieved=r["gbs"], peak=pk["hbm_gbs"], unit="GB/s", frac=r["frac_hbm"])
+        ridge = tens / hbm
+        if flop and flop / byt >= ridge / 2:
+            r.update(bound="tensor", achieved=r["tflops"], peak=pk["bf16"], unit="TFLOP/s", frac=r["frac_tensor"])
+        else:
+            r.update(bound="hbm", achieved=r["gbs"], peak=pk["hbm_gbs"], unit="GB/s", frac=r["frac_hbm"])
     r["intensity_flop_per_byte"] = flop / byt
     return r
 
@@ -421,6 +436,7 @@ def sub_measurements(dev, pk, reps, fused):
     vit_b_f16 = [workloads.Layer(L.name + " f16", L.T, L.Cp, L.Dp, L.N, "f16", ("fwd",))
                  for L in workloads.WORKLOADS["eq-vit-b-mlp-bf16-fwdbwd"]]
     t8 = [L for L in workloads.WORKLOADS["cyclic-sweep-fwdbwd"] if L.T == 8 and L.dtype == "f16"]
+    f32 = [L for L in workloads.WORKLOADS["cyclic-sweep-fwdbwd"] if L.dtype == "f32"]
     # the orders with sqrt(3)/2 twiddles, at the sweep's N and about its width (C = C'T near 1024)
     t36 = [workloads.Layer(f"cyclic T={T} f16", T, C, C, 16384, "f16", ("fwd", "dx", "dw"))
            for T, C in ((3, 336), (6, 168))]
@@ -433,6 +449,9 @@ def sub_measurements(dev, pk, reps, fused):
         "EQ-Swin-T stage-1 step (f16)": workloads.WORKLOADS["eq-swin-t-s1-f16-fwdbwd"],
         "cyclic T=8 f16 layer": t8,
         "cyclic T=3 and T=6 f16 layers": t36,
+        # FP32: forward and dx on 3xTF32 tensor cores for T = 2, 4; T = 8 and
+        # every dW on the CUDA cores
+        "cyclic FP32 layers (3xTF32 forward and dx)": f32,
     }
     stream = torch.cuda.current_stream()
     for name, layers in subs.items():

@@ -180,6 +180,16 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
       ok = cudaMalloc(&h.wt_gauss, ng * e) == cudaSuccess && cudaMemset(h.wt_gauss, 0, ng * e) == cudaSuccess;
     }
   }
+  // FP32: the 3xTF32 hi/lo images (both passes or neither)
+  const bool tc32 = ok && eqlin::tc32_supported(h);
+  if (tc32) {
+    h.bo_fwd = eqlin::tc32_pick_bo(T, Dp);
+    h.bo_bwd = eqlin::tc32_pick_bo(T, Cp);
+    const size_t nf = (size_t)eqlin::wtile32_elems(T, h.bo_fwd, Dp, Cp);
+    const size_t nb = (size_t)eqlin::wtile32_elems(T, h.bo_bwd, Cp, Dp);
+    ok = cudaMalloc(&h.wt_fwd, nf * 4) == cudaSuccess && cudaMalloc(&h.wt_bwd, nb * 4) == cudaSuccess;
+    if (ok) ok = cudaMemset(h.wt_fwd, 0, nf * 4) == cudaSuccess && cudaMemset(h.wt_bwd, 0, nb * 4) == cudaSuccess;
+  }
   if (ok) ok = cudaMemset(h.err, 0, 4 * sizeof(int)) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -187,8 +197,8 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
     delete hh;
     return EQLIN_ERR_OOM;
   }
-  h.need_simt_fwd = dihedral || dtype == EQLIN_F32 || !eqlin::tc_supported(h, false);
-  h.need_simt_bwd = dihedral || dtype == EQLIN_F32 || !eqlin::tc_supported(h, true);
+  h.need_simt_fwd = dihedral || (dtype == EQLIN_F32 ? !tc32 : !eqlin::tc_supported(h, false));
+  h.need_simt_bwd = dihedral || (dtype == EQLIN_F32 ? !tc32 : !eqlin::tc_supported(h, true));
   snprintf(h.backend, sizeof(h.backend), "fwd=%s dx=%s dw=%s", h.need_simt_fwd ? "simt" : "tcgen05",
            h.need_simt_bwd ? "simt" : "tcgen05", eqlin::tc_dw_supported(h) ? "tcgen05" : "simt");
   *out = hh;
@@ -228,6 +238,8 @@ eqlin_status_t eqlin_forward(eqlin_t hh, const void* x, void* y, int64_t N, void
     e = eqlin::launch_dihedral_apply(h, false, x, y, N, (cudaStream_t)stream);
   else if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, false))
     e = eqlin::launch_tc_apply(h, false, x, y, nullptr, N, (cudaStream_t)stream);
+  else if (h.dtype == EQLIN_F32 && !h.need_simt_fwd)
+    e = eqlin::launch_tc32_apply(h, false, x, y, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, false, x, y, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
@@ -257,6 +269,8 @@ eqlin_status_t eqlin_backward_dx(eqlin_t hh, const void* gy, void* dx, int64_t N
     e = eqlin::launch_dihedral_apply(h, true, gy, dx, N, (cudaStream_t)stream);
   else if (h.dtype != EQLIN_F32 && eqlin::tc_supported(h, true))
     e = eqlin::launch_tc_apply(h, true, gy, dx, nullptr, N, (cudaStream_t)stream);
+  else if (h.dtype == EQLIN_F32 && !h.need_simt_bwd)
+    e = eqlin::launch_tc32_apply(h, true, gy, dx, N, (cudaStream_t)stream);
   else
     e = eqlin::launch_simt_apply(h, true, gy, dx, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;

@@ -203,6 +203,30 @@ __host__ __device__ inline int64_t wtile_elems(int T, int bo, int64_t rows, int6
   return ((rows + bo - 1) / bo) * ((kdim + TC_BK - 1) / TC_BK) * tc_planes(T) * bo * TC_BK;
 }
 
+// FP32 handles (the 3xTF32 kernel, eqlin_tc32.cu): K stages of 8 input
+// channels (one kind::tf32 MMA step, 32-byte rows of f32), and per stage 2Q
+// planes: the Q planes above rounded to TF32 ("hi", planes 0 .. Q-1), then
+// the TF32 rounding of what that rounding left over ("lo", planes Q .. 2Q-1).
+// Same 32-byte-swizzled row image: 16-byte chunk j (4 floats) of row r at
+// chunk j ^ ((r >> 2) & 1).  Tile widths: 256 (T = 1), 128 (T = 2), and for
+// T = 4 64 or 32, the one that pads O least (64 on a tie).
+constexpr int TC32_BK = 8;
+inline int tc32_pick_bo(int T, int64_t O) {
+  if (T == 1) return 256;
+  if (T == 2) return 128;
+  return (O + 31) / 32 * 32 < (O + 63) / 64 * 64 ? 32 : 64;
+}
+__host__ __device__ inline int64_t wtile32_index(int T, int bo, int64_t n_kb, int64_t row, int64_t k, int plane) {
+  const int64_t ot = row / bo, kb = k / TC32_BK;
+  const int r = (int)(row % bo), kk = (int)(k % TC32_BK);
+  const int64_t tile = (ot * n_kb + kb) * 2 * tc_planes(T) + plane;
+  const int64_t byte = tile * bo * 32 + r * 32 + ((((kk >> 2) ^ ((r >> 2) & 1))) << 4) + (kk & 3) * 4;
+  return byte / 4;
+}
+__host__ __device__ inline int64_t wtile32_elems(int T, int bo, int64_t rows, int64_t kdim) {
+  return ((rows + bo - 1) / bo) * ((kdim + TC32_BK - 1) / TC32_BK) * 2 * tc_planes(T) * bo * TC32_BK;
+}
+
 // ------------------------------------------------------------ spectra
 // The stash forms of the forward and the input gradient also write the group
 // DFT of their input -- X = DFT(x) [T][C'][ld], G = DFT(gy) [T][D'][ld] --
@@ -228,7 +252,8 @@ struct Handle {
   // Fourier planes in the handle dtype for the tensor-core kernels, tiled as
   // above: fwd rows D' x K C', bwd rows C' x K D' (conjugated); Q = real
   // freqs + 3 per complex freq (-Im, Re, Im stacked so that [Re;Im] and
-  // [-Im;Re] are contiguous windows of a stage).
+  // [-Im;Re] are contiguous windows of a stage).  FP32 handles hold the
+  // 3xTF32 hi/lo images here instead (wtile32_index).
   void* wt_fwd = nullptr;
   void* wt_bwd = nullptr;
   int bo_fwd = 0, bo_bwd = 0;     // tile widths (output channels) of the two layouts
@@ -329,6 +354,12 @@ cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void
 // The p4 forward with the complex products in three real GEMMs (Gauss), for
 // comparison; needs the handle's Gauss image (h.wt_gauss).
 cudaError_t launch_tc_apply_gauss(const Handle& h, const void* in, void* out, int64_t N, cudaStream_t st);
+// FP32 handles on the tensor cores, 3xTF32 (eqlin_tc32.cu): T in {1, 2, 4};
+// forward and input gradient, and the pretransform into the hi/lo images.
+bool tc32_supported(const Handle& h);
+cudaError_t launch_tc32_apply(const Handle& h, bool backward, const void* in, void* out, int64_t N,
+                              cudaStream_t st);
+cudaError_t launch_tc32_pretransform(const Handle& h, const float* W, const float* b, cudaStream_t st);
 bool tc_dw_supported(const Handle& h);
 // dW, db from the spectra written by the stash forms (eqlin_tc_dws.cu).
 size_t tc_dws_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);

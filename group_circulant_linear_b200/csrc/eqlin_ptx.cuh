@@ -190,6 +190,26 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::tf32 (32-bit operands of
+// which the tensor core reads sign, exponent and the top 10 mantissa bits;
+// f32 accumulate).  One instruction covers K = 8.
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// f32 -> the nearest TF32 value (ties away from zero), as an f32 bit pattern
+// with the low 13 mantissa bits clear.
+__device__ __forceinline__ uint32_t f32_to_tf32(float v) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return r;
+}
+
 // Arrive on `bar` once every tcgen05 op this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -226,11 +246,41 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, int row_bytes) {
   return d;
 }
 
+// MN-major, 128B-swizzled operand descriptor (A side): leading byte offset =
+// stride between MN blocks of 128 bytes (64 16-bit elements), stride byte
+// offset = stride between 8-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;                                   // 128B swizzle
+  return d;
+}
+
+// MN-major 32-bit (TF32) operands take the 128-byte swizzle with 32-byte
+// atomicity (layout type 1): an atom is 4 K rows of 128 bytes (32 elements),
+// and 32-byte chunk j of row r sits at chunk j ^ r.  Leading byte offset =
+// stride between 128-byte MN blocks, stride byte offset = stride between
+// 4-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_mn_tf32(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)1u << 61;                                   // 128B swizzle, 32B atoms
+  return d;
+}
+
 // Instruction descriptor, kind::f16: D f32, A/B f16 (fmt 0) or bf16 (fmt 1),
 // both K-major, M = 128, N given.
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_fmt, uint32_t N) {
   return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((N >> 3) << 17) | ((128u >> 4) << 24);
 }
+// kind::tf32: the same fields with A/B format 2 (TF32).
+__host__ __device__ constexpr uint32_t idesc_tf32(uint32_t N) { return idesc_f16(2u, N); }
 
 }  // namespace ptx
 }  // namespace eqlin

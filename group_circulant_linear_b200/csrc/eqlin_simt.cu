@@ -297,7 +297,11 @@ static cudaError_t pretransform_e(const Handle& h, const void* W, const void* b,
 
 cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st) {
   switch (h.dtype) {
-    case EQLIN_F32: return pretransform_e<float>(h, W, b, st);
+    case EQLIN_F32:
+      // 3xTF32 tensor-core images (and the bias) only, when both passes use them
+      if (!h.need_simt_fwd && !h.need_simt_bwd && h.wt_fwd && h.wt_bwd)
+        return launch_tc32_pretransform(h, (const float*)W, (const float*)b, st);
+      return pretransform_e<float>(h, W, b, st);
     case EQLIN_F16: return pretransform_e<__half>(h, W, b, st);
     case EQLIN_BF16: return pretransform_e<__nv_bfloat16>(h, W, b, st);
   }

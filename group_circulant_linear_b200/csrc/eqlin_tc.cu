@@ -198,19 +198,6 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return make_uint4(pack2<E>(f[0], f[1]), pack2<E>(f[2], f[3]), pack2<E>(f[4], f[5]), pack2<E>(f[6], f[7]));
 }
 
-// MN-major, 128B-swizzled operand descriptor (A side): leading byte offset =
-// stride between 64-element MN blocks, stride byte offset = stride between
-// 8-row K groups.
-__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1u << 46;
-  d |= (uint64_t)2u << 61;                                   // 128B swizzle
-  return d;
-}
-
 template <int T, int BO, typename E, bool STASH, bool GAUSS = false>
 __global__ void __launch_bounds__(Cfg<T, BO, STASH, GAUSS>::THREADS, 1)
 tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constant__ CUtensorMap map_out,

@@ -101,6 +101,11 @@ SMALL = [  # (T, C', D', N, dtype)
     (3, 192, 768, 3000, "bf16"), (3, 768, 192, 1000, "f16"), (6, 128, 256, 5000, "f16"), (6, 256, 64, 777, "bf16"),
     (3, 24, 96, 4000, "f16"), (6, 96, 24, 3000, "bf16"),
     (6, 20, 36, 300, "bf16"),       # K not a multiple of 8: forward and dx on the SIMT kernels
+    # FP32 on the tensor cores (3xTF32) for T = 1, 2, 4: every tile width
+    # (T = 4: 64 and 32), several output tiles per persistent CTA, ragged N,
+    # and K not a multiple of the 8-channel stage (zero-filled tail)
+    (4, 64, 128, 40000, "f32"), (4, 40, 96, 20000, "f32"), (2, 128, 256, 30000, "f32"),
+    (1, 256, 512, 20000, "f32"), (4, 20, 36, 300, "f32"), (2, 6, 10, 130, "f32"), (1, 12, 20, 99, "f32"),
 ]
 
 
@@ -516,7 +521,10 @@ def test_backend_is_reported_per_pass():
             h = eqlin.create(T, 64, 64, dt)
             assert h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", (T, dt, h.backend())
             h.close()
-    assert eqlin.create(4, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt"
+    for T in (1, 2, 4):      # FP32: 3xTF32 tensor cores for forward and dx, SIMT dW
+        assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=simt", T
+    for T in (3, 6, 8):
+        assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt", T
     assert eqlin.create(4, 6, 16, "f16").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
     assert eqlin.create(4, 16, 6, "bf16").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
 
