@@ -120,8 +120,10 @@ class EQLinear(nn.Module):
         else:
             self.register_parameter("bias", None)
         self.h = eqlin.create(T, Cp, Dp, dtype)
-        # the stash forms (fused backward) serve T | 8 layers whose passes all run on tensor cores
-        self.fused = self.h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05" and self.h.T in (1, 2, 4, 8)
+        # the stash forms (fused backward) serve f16/bf16 layers of order T | 8
+        # whose passes all run on tensor cores
+        self.fused = (self.h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05" and self.h.T in (1, 2, 4, 8)
+                      and self.dtype != torch.float32)
         self._seen = None
 
     def sync_weights(self, W: torch.Tensor, b: torch.Tensor | None):

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libeqlin.so")
-SOURCES = ["eqlin_api.cu", "eqlin_simt.cu", "eqlin_tc.cu", "eqlin_tc32.cu", "eqlin_tc_dw.cu", "eqlin_tc_dws.cu",
+SOURCES = ["eqlin_api.cu", "eqlin_simt.cu", "eqlin_tc.cu", "eqlin_tc32.cu", "eqlin_tc32_dw.cu", "eqlin_tc_dw.cu", "eqlin_tc_dws.cu",
            "eqlin_dihedral.cu", "eqlin_noalloc.cu"]
 HEADERS = ["eqlin_internal.cuh", "eqlin_ptx.cuh", "eqlin_packed.cuh", "eqlin_wait.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")

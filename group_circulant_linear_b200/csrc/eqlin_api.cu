@@ -153,6 +153,10 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
   }
   const size_t planes = (size_t)T * Cp * Dp;
   h.ws_bytes = eqlin::simt_dw_workspace_bytes(T, Cp, Dp);
+  if (!dihedral && dtype == EQLIN_F32 && eqlin::tc32_dw_supported(h)) {
+    const size_t tcb = eqlin::tc32_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
+    if (tcb > h.ws_bytes) h.ws_bytes = tcb;
+  }
   if (!dihedral && dtype != EQLIN_F32) {
     const size_t tcb = eqlin::tc_dw_workspace_bytes(T, Cp, Dp, h.sm_count);
     if (tcb > h.ws_bytes) h.ws_bytes = tcb;
@@ -180,9 +184,10 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
       ok = cudaMalloc(&h.wt_gauss, ng * e) == cudaSuccess && cudaMemset(h.wt_gauss, 0, ng * e) == cudaSuccess;
     }
   }
-  // FP32: the 3xTF32 hi/lo images (both passes or neither)
-  const bool tc32 = ok && eqlin::tc32_supported(h);
-  if (tc32) {
+  // FP32: the 3xTF32 hi/lo images, for the passes whose reduction is short
+  // enough (tc32_pass_ok); the other pass keeps the FP32 SIMT planes
+  const bool tc32_f = ok && eqlin::tc32_pass_ok(h, false), tc32_b = ok && eqlin::tc32_pass_ok(h, true);
+  if (tc32_f || tc32_b) {
     h.bo_fwd = eqlin::tc32_pick_bo(T, Dp);
     h.bo_bwd = eqlin::tc32_pick_bo(T, Cp);
     const size_t nf = (size_t)eqlin::wtile32_elems(T, h.bo_fwd, Dp, Cp);
@@ -197,10 +202,11 @@ eqlin_status_t eqlin_create_group(eqlin_group_t group, int m, int64_t Cp, int64_
     delete hh;
     return EQLIN_ERR_OOM;
   }
-  h.need_simt_fwd = dihedral || (dtype == EQLIN_F32 ? !tc32 : !eqlin::tc_supported(h, false));
-  h.need_simt_bwd = dihedral || (dtype == EQLIN_F32 ? !tc32 : !eqlin::tc_supported(h, true));
+  h.need_simt_fwd = dihedral || (dtype == EQLIN_F32 ? !tc32_f : !eqlin::tc_supported(h, false));
+  h.need_simt_bwd = dihedral || (dtype == EQLIN_F32 ? !tc32_b : !eqlin::tc_supported(h, true));
   snprintf(h.backend, sizeof(h.backend), "fwd=%s dx=%s dw=%s", h.need_simt_fwd ? "simt" : "tcgen05",
-           h.need_simt_bwd ? "simt" : "tcgen05", eqlin::tc_dw_supported(h) ? "tcgen05" : "simt");
+           h.need_simt_bwd ? "simt" : "tcgen05",
+           eqlin::tc_dw_supported(h) || eqlin::tc32_dw_supported(h) ? "tcgen05" : "simt");
   *out = hh;
   return EQLIN_OK;
 }
@@ -293,6 +299,7 @@ eqlin_status_t eqlin_backward_dw(eqlin_t hh, const void* x, const void* gy, floa
   if (s != EQLIN_OK) return s;
   cudaError_t e = h.group == EQLIN_GROUP_DIHEDRAL ? eqlin::launch_dihedral_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
                   : eqlin::tc_dw_supported(h)      ? eqlin::launch_tc_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
+                  : eqlin::tc32_dw_supported(h)    ? eqlin::launch_tc32_dw(h, x, gy, dW, db, N, (cudaStream_t)stream)
                                                    : eqlin::launch_simt_dw(h, x, gy, dW, db, N, (cudaStream_t)stream);
   return e == cudaSuccess ? EQLIN_OK : EQLIN_ERR_CUDA;
 }

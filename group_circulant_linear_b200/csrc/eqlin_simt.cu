@@ -276,7 +276,8 @@ static cudaError_t pretransform_t(const Handle& h, const void* W, const void* b,
   dim3 block(pt::TILE, pt::ROWS);
   const cudaError_t e = launch_pdl(
       pretransform_kernel<T, E>, grid, block, 0, st, (const E*)W, (const E*)b,
-      h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr, (E*)h.wt_fwd, (E*)h.wt_bwd,
+      h.need_simt_fwd ? h.wf_fwd : nullptr, h.need_simt_bwd ? h.wf_bwd : nullptr,
+      sizeof(E) == 2 ? (E*)h.wt_fwd : nullptr, sizeof(E) == 2 ? (E*)h.wt_bwd : nullptr,   // f32: 3xTF32 images
       h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
   count_launches(1);
   return e;
@@ -298,9 +299,12 @@ static cudaError_t pretransform_e(const Handle& h, const void* W, const void* b,
 cudaError_t launch_pretransform(const Handle& h, const void* W, const void* b, cudaStream_t st) {
   switch (h.dtype) {
     case EQLIN_F32:
-      // 3xTF32 tensor-core images (and the bias) only, when both passes use them
-      if (!h.need_simt_fwd && !h.need_simt_bwd && h.wt_fwd && h.wt_bwd)
-        return launch_tc32_pretransform(h, (const float*)W, (const float*)b, st);
+      // the 3xTF32 tensor-core images (and the bias); the FP32 planes as well
+      // when a pass runs on the SIMT kernels
+      if (h.wt_fwd && h.wt_bwd) {
+        const cudaError_t e = launch_tc32_pretransform(h, (const float*)W, (const float*)b, st);
+        if (e != cudaSuccess || (!h.need_simt_fwd && !h.need_simt_bwd)) return e;
+      }
       return pretransform_e<float>(h, W, b, st);
     case EQLIN_F16: return pretransform_e<__half>(h, W, b, st);
     case EQLIN_BF16: return pretransform_e<__nv_bfloat16>(h, W, b, st);

@@ -627,9 +627,20 @@ bool tc32_supported(const Handle& h) {
          tensor_map_encoder() != nullptr;
 }
 
+// The tensor core rounds as it adds each MMA's products into the FP32
+// accumulator, and the error of a product sum grows with the number of MMAs
+// that feed one accumulator (measured: about 1.5e-8 to 1.9e-8 relative
+// Frobenius error per MMA); 384 MMAs keep it below 1e-5 with room to spare.
+bool tc32_pass_ok(const Handle& h, bool backward) {
+  if (!tc32_supported(h)) return false;
+  const int64_t K = backward ? h.Dp : h.Cp;
+  const int64_t per_stage = h.T == 4 ? 6 : 3;     // MMAs into one accumulator per 8-channel stage
+  return per_stage * ((K + TC32_BK - 1) / TC32_BK) <= 384;
+}
+
 cudaError_t launch_tc32_apply(const Handle& h, bool backward, const void* in, void* out, int64_t N,
                               cudaStream_t st) {
-  if (!tc32_supported(h) || !h.wt_fwd || !h.wt_bwd) return cudaErrorNotSupported;
+  if (!tc32_pass_ok(h, backward) || !h.wt_fwd || !h.wt_bwd) return cudaErrorNotSupported;
   const int bo = backward ? h.bo_bwd : h.bo_fwd;
   switch (h.T) {
     case 1: return bo == 256 ? tc32::launch_t<1, 256>(h, backward, in, out, N, st) : cudaErrorInvalidValue;

@@ -106,6 +106,8 @@ SMALL = [  # (T, C', D', N, dtype)
     # and K not a multiple of the 8-channel stage (zero-filled tail)
     (4, 64, 128, 40000, "f32"), (4, 40, 96, 20000, "f32"), (2, 128, 256, 30000, "f32"),
     (1, 256, 512, 20000, "f32"), (4, 20, 36, 300, "f32"), (2, 6, 10, 130, "f32"), (1, 12, 20, 99, "f32"),
+    # FP32 dW with c on the MMA's M side (C' a multiple of 128, D' not)
+    (2, 128, 72, 5000, "f32"), (4, 128, 40, 9000, "f32"),
 ]
 
 
@@ -132,6 +134,8 @@ def test_small_parity(T, Cp, Dp, N, dt):
 # exact in the FP32 accumulator.
 EXACT = [
     (4, 64, 64, 1024, "f32", 4), (2, 64, 48, 515, "f32", 4), (1, 32, 64, 300, "f32", 4),
+    # FP32 dW over two token passes (the second adds to the first's partials)
+    (4, 64, 64, 100000, "f32", 1),
     (4, 16, 16, 700, "f16", 4), (2, 16, 16, 300, "f16", 4), (4, 16, 8, 129, "f16", 4),
     (4, 8, 8, 400, "bf16", 2), (2, 8, 8, 200, "bf16", 2),
     # 512 token tiles: 3-4 output tiles per persistent CTA of the forward and
@@ -521,10 +525,15 @@ def test_backend_is_reported_per_pass():
             h = eqlin.create(T, 64, 64, dt)
             assert h.backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", (T, dt, h.backend())
             h.close()
-    for T in (1, 2, 4):      # FP32: 3xTF32 tensor cores for forward and dx, SIMT dW
-        assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=simt", T
+    for T in (1, 2, 4):      # FP32: 3xTF32 tensor cores
+        assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", T
     for T in (3, 6, 8):
         assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt", T
+    # FP32 passes whose reduction is too long for the 3xTF32 error bound
+    # (more than 384 MMAs into one accumulator) run on the SIMT kernels
+    assert eqlin.create(4, 520, 16, "f32").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
+    assert eqlin.create(2, 16, 1032, "f32").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
+    assert eqlin.create(1, 1024, 1024, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
     assert eqlin.create(4, 6, 16, "f16").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
     assert eqlin.create(4, 16, 6, "bf16").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
 
