@@ -24,16 +24,20 @@
 // (launch_dw_reduce).
 //
 // Work unit of one CTA: 128 M channels (d, or c when that pads less) x BC
-// N channels x one chunk of tokens, in stages of 8 tokens (one TF32 K step,
-// 32-byte K-major rows with the 32B swizzle):
+// N channels x one chunk of tokens, in stages of 16 tokens for T = 1, 2 (two
+// TF32 K steps, 64-byte K-major rows with the 64B swizzle; a stage's fixed
+// costs -- barrier waits, commits, proxy fences -- then cover twice the work)
+// and 8 for T = 4 (one K step, 32-byte rows with the 32B swizzle; a 16-token
+// stage's operands would not fit twice in shared memory):
 //   warp 16    (producer)  TMA of the stage's raw rows (M side, N side) into
 //              the raw ring, L2 prefetches ahead
-//   warps 0-15 (transform) two token groups (tokens 0-3, 4-7 of a stage) x
-//              (4 A warps, one M channel per thread; 4 B warps, one N channel
-//              per thread): the channel's T values of its 4 tokens, the group
-//              DFT in FP32, db sums of G_0 on the gy side, the hi/lo split,
-//              one 16-byte chunk per plane; after the loop the A warps read
-//              the accumulators out of TMEM into the partial planes
+//   warps 0-15 (transform) two groups of eight warps on alternate stages, so
+//              two stages are in flight; in a group 4 A warps (one M channel
+//              per thread) and 4 B warps (one N channel per thread): the
+//              channel's T values of the stage's 8 tokens, the group DFT in
+//              FP32, db sums of G_0 on the gy side, the hi/lo split, two
+//              16-byte chunks per plane; after the loop the A warps read the
+//              accumulators out of TMEM into the partial planes
 //   warp 17(+18) MMA issue, an accumulator group per issuer as in the
 //              f16/bf16 kernel; for a complex frequency the block products
 //   M = d:  [Re | Im] = Re G [Re X ; -Im X] + Im G [Im X ; Re X]   (B planes Im X, Re X, -Im X)
@@ -56,8 +60,9 @@ struct Cfg {
   using G = Group<T>;
   static_assert(T == 1 || T == 2 || T == 4, "3xTF32 tiles for T in {1, 2, 4}");
   static constexpr int BM = 128;                          // M channels per tile (MMA M)
-  static constexpr int BKN = 8;                           // tokens per stage (one TF32 K step)
-  static constexpr int ROWB = BKN * 4;                    // K-major rows of 32 bytes
+  static constexpr int BKN = T <= 2 ? 16 : 8;             // tokens per stage (BKN / 8 TF32 K steps)
+  static constexpr int KSTEPS = BKN / 8;
+  static constexpr int ROWB = BKN * 4;                    // K-major rows of 64 or 32 bytes
   static constexpr int BC_MAX = 128;                      // N channels per tile (T * 128 <= 512 columns)
   static constexpr int Q = G::nreal + 3 * G::ncomplex;    // B planes per part (hi / lo)
   static constexpr int A_PLANE_BYTES = BM * ROWB;
@@ -73,8 +78,13 @@ struct Cfg {
   static constexpr int BUDGET = 220 * 1024;
   static constexpr int OP_STAGES = (BUDGET - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3 : 2;
   static constexpr int RAW_FIT = (BUDGET - OP_STAGES * OP_BYTES) / RAW_BYTES;
-  static constexpr int RAW_STAGES = RAW_FIT > 6 ? 6 : RAW_FIT;
+  // even: the transform groups take alternate stages, and both uses of a raw
+  // slot k and k + RAW_STAGES then belong to the same group, which consumes
+  // them in order (an mbarrier parity wait cannot tell a phase from the one
+  // two ahead)
+  static constexpr int RAW_STAGES = (RAW_FIT > 6 ? 6 : RAW_FIT) & ~1;
   static_assert(RAW_STAGES >= 2, "two raw stages must fit");
+  static constexpr int GRP_WARPS = 8;                     // warps per transform group
   static constexpr int NMMA = (T == 1) ? 1 : 2;
   static constexpr int MMAS = G::nreal + 2 * G::ncomplex;
   __host__ __device__ static constexpr int own_real(int f) { return (NMMA == 1 || 2 * f < MMAS) ? 0 : 1; }
@@ -89,8 +99,10 @@ struct Cfg {
   static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;
   static constexpr int THREADS = (TR_WARPS + 1 + NMMA) * 32;
   static constexpr int PF_STAGES = 16;
-  // tokens one accumulator takes: 384 MMAs
-  static constexpr int CHUNK_MAX = 384 / (3 * (G::ncomplex > 0 ? 2 : 1)) * BKN;
+  // tokens one accumulator takes: 384 MMAs (three, or six into a complex
+  // accumulator, per 8-token K step)
+  static constexpr int CHUNK_MAX = 384 / (3 * (G::ncomplex > 0 ? 2 : 1)) * 8;
+  static_assert(CHUNK_MAX % BKN == 0, "whole stages per chunk");
 };
 
 struct Params {
@@ -110,9 +122,13 @@ struct Params {
   uint32_t wait_limit;
 };
 
-// 16-byte chunk j (4 tokens) of row r in a K-major plane of 32-byte rows, 32B swizzle
+// 16-byte chunk j (4 tokens) of row r in a K-major plane with ROWB-byte rows:
+// 32B swizzle (chunk bit 0 XOR row bit 2) for 32-byte rows, 64B swizzle
+// (chunk bits 0-1 XOR row bits 1-2) for 64-byte rows
+template <int ROWB>
 __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
-  return (uint32_t)(r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+  if constexpr (ROWB == 32) return (uint32_t)(r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+  else return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
 template <int N_>
@@ -165,10 +181,10 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::RAW_STAGES; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], C::TR_WARPS);
+      mbar_init(&raw_empty[i], C::GRP_WARPS);
     }
     for (int i = 0; i < C::OP_STAGES; ++i) {
-      mbar_init(&op_full[i], C::TR_WARPS);
+      mbar_init(&op_full[i], C::GRP_WARPS);
       mbar_init(&op_empty[i], C::NMMA);
     }
     mbar_init(acc_full, C::NMMA);
@@ -190,7 +206,7 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
 
   if (warp < C::TR_WARPS) {
     // --------------------------------------------------- transform warps
-    const int grp = warp >> 3;                             // tokens 4*grp .. 4*grp+3 of a stage
+    const int grp = warp >> 3;                             // stages grp, grp + 2, ...
     const bool is_a = (warp & 7) < 4;
     const int r = (warp & 3) * 32 + lane;                  // operand row: M channel (A) or N channel (B)
     const bool active = is_a || r < BC;
@@ -200,64 +216,66 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
                                   : (uint32_t)((r * T / p.nb_box) * C::BKN * p.nb_box * 4 +
                                                ((r * T) % p.nb_box) * 4);
     const uint32_t raw_rowb = is_a ? (uint32_t)(C::MA_BOX * 4) : (uint32_t)(p.nb_box * 4);
-    const uint32_t raw_base =
-        (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + grp * 4 * raw_rowb;
-    const uint32_t off = kmajor_off(r, grp);
+    const uint32_t raw_base = (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col;
     float dbacc = 0.f;
-    int rs = 0, os = 0;
+    int rs = grp % C::RAW_STAGES, os = grp % C::OP_STAGES;
     uint32_t rph = 0, oph = 0;
     bool ok = true;
-    for (int st = 0; st < nst; ++st) {
+    for (int st = grp; st < nst; st += 2) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_DW, 1, 1), (uint32_t)st)) { ok = false; break; }
-      uint32_t hi[T][4], lo[T][4];
-      if (active) {
-        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float v[T], P[T];
-          load_group<T>(raw + j * raw_rowb, v);
-          G::dft(v, P);
-          if (sums_db) dbacc += P[0];
-#pragma unroll
-          for (int q = 0; q < T; ++q) {
-            hi[q][j] = f32_to_tf32(P[q]);
-            lo[q][j] = f32_to_tf32(P[q] - __uint_as_float(hi[q][j]));
-          }
-        }
-      }
       if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
       if (active) {
+        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
         uint8_t* a_st = op_buf + os * C::OP_BYTES;
         uint8_t* b_st = a_st + C::A_BYTES;
-        auto put = [&](uint8_t* plane_base, const uint32_t (&w)[4], uint32_t sign) {
-          *reinterpret_cast<uint4*>(plane_base + off) = make_uint4(w[0] ^ sign, w[1] ^ sign, w[2] ^ sign, w[3] ^ sign);
-        };
-        if (is_a) {
+        // the stage's tokens as 16-byte chunks of 4 tokens per plane row
 #pragma unroll
-          for (int q = 0; q < T; ++q) {
-            put(a_st + q * C::A_PLANE_BYTES, hi[q], 0u);
-            put(a_st + (T + q) * C::A_PLANE_BYTES, lo[q], 0u);
+        for (int c4 = 0; c4 < C::BKN / 4; ++c4) {
+          uint32_t hi[T][4], lo[T][4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float v[T], P[T];
+            load_group<T>(raw + (4 * c4 + j) * raw_rowb, v);
+            G::dft(v, P);
+            if (sums_db) dbacc += P[0];
+#pragma unroll
+            for (int q = 0; q < T; ++q) {
+              hi[q][j] = f32_to_tf32(P[q]);
+              lo[q][j] = f32_to_tf32(P[q] - __uint_as_float(hi[q][j]));
+            }
           }
-        } else {
+          const uint32_t off = kmajor_off<C::ROWB>(r, c4);
+          auto put = [&](uint8_t* plane_base, const uint32_t (&w)[4], uint32_t sign) {
+            *reinterpret_cast<uint4*>(plane_base + off) =
+                make_uint4(w[0] ^ sign, w[1] ^ sign, w[2] ^ sign, w[3] ^ sign);
+          };
+          if (is_a) {
 #pragma unroll
-          for (int f = 0; f < G::nreal; ++f) {
-            put(b_st + f * b_plane, hi[f], 0u);
-            put(b_st + (C::Q + f) * b_plane, lo[f], 0u);
-          }
+            for (int q = 0; q < T; ++q) {
+              put(a_st + q * C::A_PLANE_BYTES, hi[q], 0u);
+              put(a_st + (T + q) * C::A_PLANE_BYTES, lo[q], 0u);
+            }
+          } else {
 #pragma unroll
-          for (int k = 1; k <= G::ncomplex; ++k) {
-            const int pr = G::nreal + 2 * (k - 1);
-            const int q = G::nreal + 3 * (k - 1);
-            // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G).  The split
-            // rounds to nearest (ties away), symmetric in sign: a negated
-            // plane is the hi and lo of the plane with their signs flipped.
-            const int i0 = swap ? pr : pr + 1, i1 = swap ? pr + 1 : pr;
-            put(b_st + (q + 0) * b_plane, hi[i0], 0u);
-            put(b_st + (q + 1) * b_plane, hi[i1], 0u);
-            put(b_st + (q + 2) * b_plane, hi[i0], 0x80000000u);
-            put(b_st + (C::Q + q + 0) * b_plane, lo[i0], 0u);
-            put(b_st + (C::Q + q + 1) * b_plane, lo[i1], 0u);
-            put(b_st + (C::Q + q + 2) * b_plane, lo[i0], 0x80000000u);
+            for (int f = 0; f < G::nreal; ++f) {
+              put(b_st + f * b_plane, hi[f], 0u);
+              put(b_st + (C::Q + f) * b_plane, lo[f], 0u);
+            }
+#pragma unroll
+            for (int k = 1; k <= G::ncomplex; ++k) {
+              const int pr = G::nreal + 2 * (k - 1);
+              const int q = G::nreal + 3 * (k - 1);
+              // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G).  The split
+              // rounds to nearest (ties away), symmetric in sign: a negated
+              // plane is the hi and lo of the plane with their signs flipped.
+              const int i0 = swap ? pr : pr + 1, i1 = swap ? pr + 1 : pr;
+              put(b_st + (q + 0) * b_plane, hi[i0], 0u);
+              put(b_st + (q + 1) * b_plane, hi[i1], 0u);
+              put(b_st + (q + 2) * b_plane, hi[i0], 0x80000000u);
+              put(b_st + (C::Q + q + 0) * b_plane, lo[i0], 0u);
+              put(b_st + (C::Q + q + 1) * b_plane, lo[i1], 0u);
+              put(b_st + (C::Q + q + 2) * b_plane, lo[i0], 0x80000000u);
+            }
           }
         }
       }
@@ -269,14 +287,16 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
         mbar_arrive(&raw_empty[rs]);
         mbar_arrive(&op_full[os]);
       }
-      if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
-      if (++os == C::OP_STAGES) { os = 0; oph ^= 1; }
+      rs += 2;
+      if (rs >= C::RAW_STAGES) { rs -= C::RAW_STAGES; rph ^= 1; }
+      os += 2;
+      if (os >= C::OP_STAGES) { os -= C::OP_STAGES; oph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
     grid_dep_launch();
 
     // db: the side that sums G_0 writes (or adds) its channels' sums; group 1
-    // hands its sums to group 0 through shared memory.  Only the tiles of the
+    // (the odd stages) hands its sums to group 0 through shared memory.  Only the tiles of the
     // other side's first tile write, so each d is written once per chunk.
     const bool db_tile = swap ? (mt == 0) : (nt == 0);
     if (sums_db && db_tile) {
@@ -295,8 +315,8 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
     if (is_a) {
       // ------------------------------------------------------- epilogue
       // Partial planes [z][T][N channel][M channel]: a warp stores 32
-      // consecutive M channels of one N channel; token group g takes the N
-      // columns [g * BC/2, (g+1) * BC/2).
+      // consecutive M channels of one N channel; transform group g takes the
+      // N columns [g * BC/2, (g+1) * BC/2).
       const bool all_ok = named_bar_and(3, 256, ok);
       const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
       bool got = all_ok && wwait_all(acc_full, 0, limit, abort_flag, p.err, site(K_DW, 4, 5), 0u);
@@ -391,26 +411,31 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
         const uint64_t a_d = desc0 + (uint64_t)((s * C::OP_BYTES) >> 4);
         const uint64_t b_d = a_d + (uint64_t)(C::A_BYTES >> 4);
         const uint32_t bp = b_plane >> 4;
-        auto A = [&](int plane) { return a_d + (uint64_t)((plane * C::A_PLANE_BYTES) >> 4); };
-        auto B = [&](int plane) { return b_d + (uint64_t)plane * bp; };
-        // a * b = hi(a) hi(b) + hi(a) lo(b) + lo(a) hi(b)
-        auto prod3 = [&](uint32_t d, int pa, int pb, uint32_t id, uint32_t acc_first) {
-          mma_tf32_ss(d, A(pa), B(pb), id, acc_first);
-          mma_tf32_ss(d, A(pa), B(C::Q + pb), id, 1u);
-          mma_tf32_ss(d, A(T + pa), B(pb), id, 1u);
-        };
-        const uint32_t first = st > 0 ? 1u : 0u;
 #pragma unroll
-        for (int f = 0; f < G::nreal; ++f)
-          if (C::own_real(f) == mi) prod3(tmem_base + f * BC, f, f, id_real, first);
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          // K step kk: 8 tokens = 32 bytes further along the swizzled rows
+          const uint64_t ka = a_d + (uint64_t)(kk * 2), kb = b_d + (uint64_t)(kk * 2);
+          auto A = [&](int plane) { return ka + (uint64_t)((plane * C::A_PLANE_BYTES) >> 4); };
+          auto B = [&](int plane) { return kb + (uint64_t)plane * bp; };
+          // a * b = hi(a) hi(b) + hi(a) lo(b) + lo(a) hi(b)
+          auto prod3 = [&](uint32_t d, int pa, int pb, uint32_t id, uint32_t acc_first) {
+            mma_tf32_ss(d, A(pa), B(pb), id, acc_first);
+            mma_tf32_ss(d, A(pa), B(C::Q + pb), id, 1u);
+            mma_tf32_ss(d, A(T + pa), B(pb), id, 1u);
+          };
+          const uint32_t first = (st > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
-        for (int k = 1; k <= G::ncomplex; ++k) {
-          if (C::own_cplx(k) != mi) continue;
-          const int pr = G::nreal + 2 * (k - 1);
-          const int q = G::nreal + 3 * (k - 1);
-          const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
-          prod3(col, pr, q + w1, id_cplx, first);
-          prod3(col, pr + 1, q + w2, id_cplx, 1u);
+          for (int f = 0; f < G::nreal; ++f)
+            if (C::own_real(f) == mi) prod3(tmem_base + f * BC, f, f, id_real, first);
+#pragma unroll
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            if (C::own_cplx(k) != mi) continue;
+            const int pr = G::nreal + 2 * (k - 1);
+            const int q = G::nreal + 3 * (k - 1);
+            const uint32_t col = tmem_base + G::nreal * BC + (k - 1) * 2 * BC;
+            prod3(col, pr, q + w1, id_cplx, first);
+            prod3(col, pr + 1, q + w2, id_cplx, 1u);
+          }
         }
         mma_commit(&op_empty[s]);
         if (++s == C::OP_STAGES) { s = 0; ph ^= 1; }
