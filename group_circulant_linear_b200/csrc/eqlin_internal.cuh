@@ -208,13 +208,20 @@ __host__ __device__ inline int64_t wtile_elems(int T, int bo, int64_t rows, int6
 // planes: the Q planes above rounded to TF32 ("hi", planes 0 .. Q-1), then
 // the TF32 rounding of what that rounding left over ("lo", planes Q .. 2Q-1).
 // Same 32-byte-swizzled row image: 16-byte chunk j (4 floats) of row r at
-// chunk j ^ ((r >> 2) & 1).  Tile widths: 256 (T = 1), 128 (T = 2), and for
-// T = 4 64 or 32, the one that pads O least (64 on a tie).
+// chunk j ^ ((r >> 2) & 1).  Tile widths: the widest MMAs that fit (an
+// N = 128 TF32 MMA already reads its operands at the SM's shared-memory rate,
+// so narrower tiles are bandwidth-bound): 256 (T = 1), 256 or 128 (T = 2),
+// 128, 64 or 32 (T = 4), the one that pads O least, the wider on a tie.
 constexpr int TC32_BK = 8;
 inline int tc32_pick_bo(int T, int64_t O) {
   if (T == 1) return 256;
-  if (T == 2) return 128;
-  return (O + 31) / 32 * 32 < (O + 63) / 64 * 64 ? 32 : 64;
+  const int widths2[2] = {256, 128}, widths4[3] = {128, 64, 32};
+  const int* w = T == 2 ? widths2 : widths4;
+  const int n = T == 2 ? 2 : 3;
+  int best = w[0];
+  for (int i = 1; i < n; ++i)
+    if ((O + w[i] - 1) / w[i] * w[i] < (O + best - 1) / best * best) best = w[i];
+  return best;
 }
 __host__ __device__ inline int64_t wtile32_index(int T, int bo, int64_t n_kb, int64_t row, int64_t k, int plane) {
   const int64_t ot = row / bo, kb = k / TC32_BK;

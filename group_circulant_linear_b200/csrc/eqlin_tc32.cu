@@ -87,7 +87,8 @@ struct Cfg {
   // epilogue half where four raw slots still fit, else one; the rest raw
   // slots (even, as in the f16/bf16 kernel: both uses of a slot belong to
   // the same transform group)
-  static constexpr int BUDGET = 224 * 1024;
+  static constexpr int BIAS_BYTES = 2 * BO * 4;        // per epilogue half, the tile's bias (FP32)
+  static constexpr int BUDGET = 225 * 1024 - BIAS_BYTES;
   static constexpr int AB_ST = (BUDGET - 2 * OUT_TILE_BYTES - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 3 : 2;
   static constexpr int NSTG = (BUDGET - 4 * OUT_TILE_BYTES - AB_ST * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 2 : 1;
   static constexpr int STAGING = 2 * NSTG * OUT_TILE_BYTES;
@@ -102,7 +103,6 @@ struct Cfg {
     return NMMA == 1 ? 0 : (2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
   }
   static constexpr int NBAR = 2 * RAW_ST + 2 * AB_ST + 2 * NACC + NMMA;
-  static constexpr int BIAS_BYTES = 2 * BO * 4;
   static constexpr int SMEM_BYTES = RAW_ST * RAW_BYTES + AB_ST * (A_BYTES + B_BYTES) + STAGING + BIAS_BYTES +
                                     NBAR * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
@@ -644,9 +644,13 @@ cudaError_t launch_tc32_apply(const Handle& h, bool backward, const void* in, vo
   const int bo = backward ? h.bo_bwd : h.bo_fwd;
   switch (h.T) {
     case 1: return bo == 256 ? tc32::launch_t<1, 256>(h, backward, in, out, N, st) : cudaErrorInvalidValue;
-    case 2: return bo == 128 ? tc32::launch_t<2, 128>(h, backward, in, out, N, st) : cudaErrorInvalidValue;
+    case 2:
+      return bo == 256   ? tc32::launch_t<2, 256>(h, backward, in, out, N, st)
+             : bo == 128 ? tc32::launch_t<2, 128>(h, backward, in, out, N, st)
+                         : cudaErrorInvalidValue;
     case 4:
-      return bo == 64   ? tc32::launch_t<4, 64>(h, backward, in, out, N, st)
+      return bo == 128  ? tc32::launch_t<4, 128>(h, backward, in, out, N, st)
+             : bo == 64 ? tc32::launch_t<4, 64>(h, backward, in, out, N, st)
              : bo == 32 ? tc32::launch_t<4, 32>(h, backward, in, out, N, st)
                         : cudaErrorInvalidValue;
   }

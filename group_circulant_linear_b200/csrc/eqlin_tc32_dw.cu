@@ -24,16 +24,17 @@
 // (launch_dw_reduce).
 //
 // Work unit of one CTA: 128 M channels (d, or c when that pads less) x BC
-// N channels x one chunk of tokens, in stages of 16 tokens for T = 1, 2 (two
-// TF32 K steps, 64-byte K-major rows with the 64B swizzle; a stage's fixed
-// costs -- barrier waits, commits, proxy fences -- then cover twice the work)
-// and 8 for T = 4 (one K step, 32-byte rows with the 32B swizzle; a 16-token
-// stage's operands would not fit twice in shared memory):
+// N channels (BC <= 256 for T = 1, 2, <= 128 for T = 4) x one chunk of
+// tokens, in stages of 16 tokens for T = 1 (two TF32 K steps, 64-byte K-major
+// rows with the 64B swizzle; a stage's fixed costs -- barrier waits, commits,
+// proxy fences -- then cover twice the work) and 8 for T = 2, 4 (one K step,
+// 32-byte rows with the 32B swizzle; their 16-token stages would not fit
+// twice in shared memory):
 //   warp 16    (producer)  TMA of the stage's raw rows (M side, N side) into
 //              the raw ring, L2 prefetches ahead
 //   warps 0-15 (transform) two groups of eight warps on alternate stages, so
 //              two stages are in flight; in a group 4 A warps (one M channel
-//              per thread) and 4 B warps (one N channel per thread): the
+//              per thread) and 4 B warps (one or two N channels per thread): the
 //              channel's T values of the stage's 8 tokens, the group DFT in
 //              FP32, db sums of G_0 on the gy side, the hi/lo split, two
 //              16-byte chunks per plane; after the loop the A warps read the
@@ -60,10 +61,17 @@ struct Cfg {
   using G = Group<T>;
   static_assert(T == 1 || T == 2 || T == 4, "3xTF32 tiles for T in {1, 2, 4}");
   static constexpr int BM = 128;                          // M channels per tile (MMA M)
-  static constexpr int BKN = T <= 2 ? 16 : 8;             // tokens per stage (BKN / 8 TF32 K steps)
+  // N channels per tile: 256 for T = 1, 2 (T * 256 <= 512 TMEM columns), 128
+  // for T = 4 (its complex block products are N = 2 * BC MMAs).  Wide N keeps
+  // the operand reads per FLOP down: an N = 128 TF32 MMA already reads its
+  // operands at the SM's shared-memory rate.
+  static constexpr int BC_MAX = T <= 2 ? 256 : 128;
+  static constexpr int NRB = BC_MAX / 128;                // N channels per B-side transform thread
+  // tokens per stage: 16 for T = 1 (two TF32 K steps), 8 otherwise (the
+  // operands of a 16-token stage would not fit twice beside the raw ring)
+  static constexpr int BKN = T == 1 ? 16 : 8;
   static constexpr int KSTEPS = BKN / 8;
   static constexpr int ROWB = BKN * 4;                    // K-major rows of 64 or 32 bytes
-  static constexpr int BC_MAX = 128;                      // N channels per tile (T * 128 <= 512 columns)
   static constexpr int Q = G::nreal + 3 * G::ncomplex;    // B planes per part (hi / lo)
   static constexpr int A_PLANE_BYTES = BM * ROWB;
   static constexpr int A_BYTES = 2 * T * A_PLANE_BYTES;   // hi planes 0..T-1, lo planes T..2T-1
@@ -76,7 +84,7 @@ struct Cfg {
   static constexpr int NB_ROWB_MAX = BC_MAX * T * 4;
   static constexpr int RAW_BYTES = BKN * (MA_ROWB + NB_ROWB_MAX);
   static constexpr int BUDGET = 220 * 1024;
-  static constexpr int OP_STAGES = (BUDGET - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3 : 2;
+  static constexpr int OP_STAGES = (BUDGET - 3 * OP_BYTES) / RAW_BYTES >= 4 ? 3 : 2;
   static constexpr int RAW_FIT = (BUDGET - OP_STAGES * OP_BYTES) / RAW_BYTES;
   // even: the transform groups take alternate stages, and both uses of a raw
   // slot k and k + RAW_STAGES then belong to the same group, which consumes
@@ -92,7 +100,7 @@ struct Cfg {
     return (NMMA == 1 || 2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
   }
   static constexpr int NBAR = 2 * RAW_STAGES + 2 * OP_STAGES + 1 + NMMA;
-  static constexpr int SMEM_BYTES = OP_STAGES * OP_BYTES + RAW_STAGES * RAW_BYTES + NBAR * 8 + 16 + BM * 4 + 1024;
+  static constexpr int SMEM_BYTES = OP_STAGES * OP_BYTES + RAW_STAGES * RAW_BYTES + NBAR * 8 + 16 + BC_MAX * 4 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
   static constexpr int TR_WARPS = 16;
@@ -162,7 +170,7 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
   uint64_t* drain_bar = acc_full + 1;           // [NMMA]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* db_half = reinterpret_cast<float*>(tmem_slot + 4);       // [BM] token group 1's db sums
+  float* db_half = reinterpret_cast<float*>(tmem_slot + 4);       // [BC_MAX] group 1's db sums
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tiles = p.n_mt * p.n_nt;
@@ -208,26 +216,35 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
     // --------------------------------------------------- transform warps
     const int grp = warp >> 3;                             // stages grp, grp + 2, ...
     const bool is_a = (warp & 7) < 4;
-    const int r = (warp & 3) * 32 + lane;                  // operand row: M channel (A) or N channel (B)
-    const bool active = is_a || r < BC;
+    const int r = (warp & 3) * 32 + lane;                  // first operand row: M channel (A) or N channel (B)
+    const int nrows = is_a ? 1 : C::NRB;                   // rows r, r + 128, ... of this thread
     const bool sums_db = is_a != swap;                     // the side that holds gy
-    const uint32_t raw_col = is_a ? (uint32_t)((r / (C::MA_BOX / T)) * C::BKN * C::MA_BOX * 4 +
-                                               (r % (C::MA_BOX / T)) * T * 4)
-                                  : (uint32_t)((r * T / p.nb_box) * C::BKN * p.nb_box * 4 +
-                                               ((r * T) % p.nb_box) * 4);
     const uint32_t raw_rowb = is_a ? (uint32_t)(C::MA_BOX * 4) : (uint32_t)(p.nb_box * 4);
-    const uint32_t raw_base = (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col;
-    float dbacc = 0.f;
+    // this thread's channels in the raw tile rows
+    uint32_t raw_base[C::NRB];
+#pragma unroll
+    for (int i = 0; i < C::NRB; ++i) {
+      const int rr = r + 128 * i;
+      raw_base[i] = is_a ? (uint32_t)((rr / (C::MA_BOX / T)) * C::BKN * C::MA_BOX * 4 + (rr % (C::MA_BOX / T)) * T * 4)
+                         : (uint32_t)(C::BKN * C::MA_ROWB + (rr * T / p.nb_box) * C::BKN * p.nb_box * 4 +
+                                      ((rr * T) % p.nb_box) * 4);
+    }
+    float dbacc[C::NRB];
+#pragma unroll
+    for (int i = 0; i < C::NRB; ++i) dbacc[i] = 0.f;
     int rs = grp % C::RAW_STAGES, os = grp % C::OP_STAGES;
     uint32_t rph = 0, oph = 0;
     bool ok = true;
     for (int st = grp; st < nst; st += 2) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_DW, 1, 1), (uint32_t)st)) { ok = false; break; }
       if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
-      if (active) {
-        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base;
-        uint8_t* a_st = op_buf + os * C::OP_BYTES;
-        uint8_t* b_st = a_st + C::A_BYTES;
+      uint8_t* a_st = op_buf + os * C::OP_BYTES;
+      uint8_t* b_st = a_st + C::A_BYTES;
+#pragma unroll
+      for (int i = 0; i < C::NRB; ++i) {
+        const int rr = r + 128 * i;
+        if (i >= nrows || (!is_a && rr >= BC)) continue;
+        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base[i];
         // the stage's tokens as 16-byte chunks of 4 tokens per plane row
 #pragma unroll
         for (int c4 = 0; c4 < C::BKN / 4; ++c4) {
@@ -237,14 +254,14 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
             float v[T], P[T];
             load_group<T>(raw + (4 * c4 + j) * raw_rowb, v);
             G::dft(v, P);
-            if (sums_db) dbacc += P[0];
+            if (sums_db) dbacc[i] += P[0];
 #pragma unroll
             for (int q = 0; q < T; ++q) {
               hi[q][j] = f32_to_tf32(P[q]);
               lo[q][j] = f32_to_tf32(P[q] - __uint_as_float(hi[q][j]));
             }
           }
-          const uint32_t off = kmajor_off<C::ROWB>(r, c4);
+          const uint32_t off = kmajor_off<C::ROWB>(rr, c4);
           auto put = [&](uint8_t* plane_base, const uint32_t (&w)[4], uint32_t sign) {
             *reinterpret_cast<uint4*>(plane_base + off) =
                 make_uint4(w[0] ^ sign, w[1] ^ sign, w[2] ^ sign, w[3] ^ sign);
@@ -296,19 +313,24 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
     grid_dep_launch();
 
     // db: the side that sums G_0 writes (or adds) its channels' sums; group 1
-    // (the odd stages) hands its sums to group 0 through shared memory.  Only the tiles of the
-    // other side's first tile write, so each d is written once per chunk.
+    // (the odd stages) hands its sums to group 0 through shared memory.  Only
+    // the tiles of the other side's first tile write, so each d is written
+    // once per chunk.
     const bool db_tile = swap ? (mt == 0) : (nt == 0);
     if (sums_db && db_tile) {
       const int bar_id = is_a ? 1 : 2;
       named_bar_sync(bar_id, 256);
-      if (grp == 1) db_half[r] = dbacc;
+      if (grp == 1)
+        for (int i = 0; i < nrows; ++i) db_half[r + 128 * i] = dbacc[i];
       named_bar_sync(bar_id, 256);
-      const int d = (swap ? n0 : m0) + r;
-      if (grp == 0 && active && d < p.Dp) {
-        float* dst = p.dbpart + (int64_t)z * p.Dp + d;
-        const float v = dbacc + db_half[r];
-        *dst = p.accumulate ? *dst + v : v;
+      for (int i = 0; i < nrows; ++i) {
+        const int rr = r + 128 * i;
+        const int d = (swap ? n0 : m0) + rr;
+        if (grp == 0 && (is_a || rr < BC) && d < p.Dp) {
+          float* dst = p.dbpart + (int64_t)z * p.Dp + d;
+          const float v = dbacc[i] + db_half[rr];
+          *dst = p.accumulate ? *dst + v : v;
+        }
       }
     }
 

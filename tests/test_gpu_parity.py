@@ -108,6 +108,10 @@ SMALL = [  # (T, C', D', N, dtype)
     (1, 256, 512, 20000, "f32"), (4, 20, 36, 300, "f32"), (2, 6, 10, 130, "f32"), (1, 12, 20, 99, "f32"),
     # FP32 dW with c on the MMA's M side (C' a multiple of 128, D' not)
     (2, 128, 72, 5000, "f32"), (4, 128, 40, 9000, "f32"),
+    # FP32 dW N sides wider than 128 channels (two per transform thread; with
+    # d on the N side, db from rows past 128), and token ranges of two passes
+    (2, 256, 128, 5000, "f32"), (2, 128, 200, 3000, "f32"),
+    (2, 128, 128, 160000, "f32"), (1, 128, 128, 160000, "f32"),
 ]
 
 
