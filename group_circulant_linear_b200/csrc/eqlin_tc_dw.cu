@@ -21,13 +21,15 @@
 //   warp 16    (producer)  TMA: the stage's rows of the M-side input (gy or x)
 //              for the 128 M channels and of the N-side input for the BC N
 //              channels into a raw ring, and L2 prefetches of later stages
-//   warps 0-15 (transform) two groups of eight warps, group g taking tokens
-//              8g .. 8g+7 of every stage.  In a group, warps 0-3 take one M
-//              channel each (A planes) and warps 4-7 one N channel each (B
-//              planes): read the channel's T group values of the 8 tokens,
-//              take the group DFT (packed token pairs for T <= 4, FP32 for
-//              T = 8), keep sum_n G_0 in FP32 for db on the side that holds gy,
-//              and write K-major (token-contiguous) operand planes.  After the
+//   warps 0-15 (transform) two groups of eight warps: on alternate stages
+//              (two stages in flight), or in the small-channel configuration
+//              on the two halves of every stage's tokens.  In a group, warps
+//              0-3 take one M channel each (A planes) and warps 4-7 one N
+//              channel each (B planes): read the channel's T group values of
+//              its tokens, 8 at a time, take the group DFT (packed token
+//              pairs for T <= 4, FP32 for T = 3, 6, 8), keep sum_n G_0 in FP32
+//              for db on the side that holds gy, and write K-major
+//              (token-contiguous) operand planes.  After the
 //              main loop the A warps of both groups read the accumulators out
 //              of TMEM, each group half of the N columns
 //   warp 17    allocates TMEM; the warp runs the MMA loop and one lane issues
@@ -65,7 +67,11 @@ struct Cfg {
   using G = Group<T>;
   static constexpr int BM = 128;                          // M channels per tile (MMA M)
   static constexpr int BKN = BCM <= 32 && T <= 4 ? 32 : 16;   // tokens per stage (BKN / 16 MMA K steps)
-  static constexpr int NSB = BKN / 16;                    // 8-token blocks per transform thread and stage
+  // ALT: the two transform groups take alternate stages (two stages in
+  // flight); otherwise (the small-channel configuration, where that measured
+  // slower) they split each stage's tokens
+  static constexpr bool ALT = BCM > 32;
+  static constexpr int NSB = ALT ? BKN / 8 : BKN / 16;    // 8-token blocks per transform thread and stage
   static constexpr int ROWB = BKN * 2;                    // K-major rows of 32 or 64 bytes, swizzled as wide
   // T * BC_MAX TMEM columns; tile widths are multiples of 16
   static constexpr int BC_MAX = (512 / T / 16 * 16) < BCM ? (512 / T / 16 * 16) : BCM;
@@ -82,11 +88,15 @@ struct Cfg {
   // stage k + 2 while the MMAs of k and k + 1 are in flight), four where four
   // raw slots still fit beside them, else two; the rest of 220 KB for raw
   // slots (memory latency)
-  static constexpr int OP_STAGES = (220 * 1024 - 4 * OP_BYTES) / RAW_BYTES >= 4   ? 4
+  static constexpr int OP_STAGES = ALT ? ((220 * 1024 - 3 * OP_BYTES) / RAW_BYTES >= 4 ? 3 : 2)
+                                   : (220 * 1024 - 4 * OP_BYTES) / RAW_BYTES >= 4 ? 4
                                    : (220 * 1024 - 3 * OP_BYTES) / RAW_BYTES >= 3 ? 3
                                                                                   : 2;
   static constexpr int RAW_FIT = (220 * 1024 - OP_STAGES * OP_BYTES) / RAW_BYTES;
-  static constexpr int RAW_STAGES = RAW_FIT > 6 ? 6 : RAW_FIT;
+  // with alternate stages the depth is even, so both uses of a raw slot k and
+  // k + RAW_STAGES belong to the same group (an mbarrier parity wait cannot
+  // tell a phase from the one two ahead)
+  static constexpr int RAW_STAGES = (RAW_FIT > 6 ? 6 : RAW_FIT) & (ALT ? ~1 : ~0);
   static_assert(RAW_STAGES >= 2, "two raw stages must fit");
   // MMA issuers: an accumulator group (a real frequency's plane, or a
   // complex frequency's [Re | Im] block, two MMAs) belongs to one issuer; in
@@ -101,7 +111,8 @@ struct Cfg {
   static constexpr int SMEM_BYTES = OP_STAGES * OP_BYTES + RAW_STAGES * RAW_BYTES + NBAR * 8 + 16 +
                                     BM * 4 + 1024;
   static constexpr int TMEM_COLS = T * BC_MAX <= 256 ? 256 : 512;
-  static constexpr int TR_WARPS = 16;                     // two token groups x (4 A + 4 B warps)
+  static constexpr int TR_WARPS = 16;                     // two groups x (4 A + 4 B warps)
+  static constexpr int STAGE_ARRIVALS = ALT ? 8 : 16;     // transform warps that fill one stage
   static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;   // MMA warps MMA_WARP .. + NMMA - 1
   static constexpr int THREADS = (TR_WARPS + 1 + NMMA) * 32;
   static constexpr int PF_STAGES = 12;                    // L2 prefetch distance (stages)
@@ -182,10 +193,10 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::RAW_STAGES; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], C::TR_WARPS);
+      mbar_init(&raw_empty[i], C::STAGE_ARRIVALS);
     }
     for (int i = 0; i < C::OP_STAGES; ++i) {
-      mbar_init(&op_full[i], C::TR_WARPS);
+      mbar_init(&op_full[i], C::STAGE_ARRIVALS);
       mbar_init(&op_empty[i], C::NMMA);   // one commit per MMA issuer
     }
     mbar_init(acc_full, C::NMMA);
@@ -207,7 +218,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
 
   if (warp < C::TR_WARPS) {
     // --------------------------------------------------- transform warps
-    const int grp = warp >> 3;                             // token group: tokens 8*NSB*grp .. 8*NSB*(grp+1)-1
+    const int grp = warp >> 3;                             // ALT: stages grp, grp + 2, ...; else tokens 8*NSB*grp ..
     const bool is_a = (warp & 7) < 4;
     const int r = (warp & 3) * 32 + lane;                  // operand row: M channel (A) or N channel (B)
     const bool active = is_a || r < BC;
@@ -220,43 +231,48 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
                                                ((r * T) % p.nb_box) * 2);
     const uint32_t raw_rowb = is_a ? (uint32_t)(C::MA_BOX * 2) : (uint32_t)(p.nb_box * 2);
     const uint32_t raw_base =
-        (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + grp * C::NSB * 8 * raw_rowb;
+        (is_a ? 0u : (uint32_t)(C::BKN * C::MA_ROWB)) + raw_col + (C::ALT ? 0 : grp * C::NSB * 8 * raw_rowb);
     float dbacc = 0.f;
-    int rs = 0, os = 0;
+    constexpr int STEP = C::ALT ? 2 : 1;                   // stages between a group's turns
+    int rs = C::ALT ? grp % C::RAW_STAGES : 0, os = C::ALT ? grp % C::OP_STAGES : 0;
     uint32_t rph = 0, oph = 0;
     bool ok = true;
-    for (int st = 0; st < nst; ++st) {
+    for (int st = C::ALT ? grp : 0; st < nst; st += STEP) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_DW, 1, 1), (uint32_t)st)) { ok = false; break; }
-      uint32_t Pw[C::NSB][T][4];
+      // the operand slot must have been consumed by the MMAs issued from it
+      if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
+      uint8_t* a_st = op_buf + os * C::OP_BYTES;
+      uint8_t* b_st = a_st + C::A_BYTES;
 #pragma unroll
       for (int sb = 0; sb < C::NSB; ++sb) {
-      uint32_t wv[8][C::W];
-      const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base + sb * 8 * raw_rowb;
-      if (active && (T == 1 || T == 2 || T == 4 || T == 8)) {
+        uint32_t Pw[T][4];
+        uint32_t wv[8][C::W];
+        const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_base + sb * 8 * raw_rowb;
+        if (active && (T == 1 || T == 2 || T == 4 || T == 8)) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint8_t* src = raw + j * raw_rowb;
-          if constexpr (C::W == 4) {
-            const uint4 u = *reinterpret_cast<const uint4*>(src);
-            wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
-          } else if constexpr (C::W == 2) {
-            const uint2 u = *reinterpret_cast<const uint2*>(src);
-            wv[j][0] = u.x; wv[j][1] = u.y;
-          } else if constexpr (T == 2) {
-            wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
-          } else {
-            wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+          for (int j = 0; j < 8; ++j) {
+            const uint8_t* src = raw + j * raw_rowb;
+            if constexpr (C::W == 4) {
+              const uint4 u = *reinterpret_cast<const uint4*>(src);
+              wv[j][0] = u.x; wv[j][1] = u.y; wv[j][2] = u.z; wv[j][3] = u.w;
+            } else if constexpr (C::W == 2) {
+              const uint2 u = *reinterpret_cast<const uint2*>(src);
+              wv[j][0] = u.x; wv[j][1] = u.y;
+            } else if constexpr (T == 2) {
+              wv[j][0] = *reinterpret_cast<const uint32_t*>(src);
+            } else {
+              wv[j][0] = *reinterpret_cast<const unsigned short*>(src);
+            }
           }
         }
-      }
-      if (active) {
+        if (!active) continue;
         if constexpr (T == 1 || T == 2 || T == 4) {
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
             uint32_t P[T];
             packed::dft_pair<T, E>(wv[2 * pr], wv[2 * pr + 1], P);
 #pragma unroll
-            for (int q = 0; q < T; ++q) Pw[sb][q][pr] = P[q];
+            for (int q = 0; q < T; ++q) Pw[q][pr] = P[q];
             if (sums_db) {
               const float2 f = packed::Pair<E>::to_f2(P[0]);
               dbacc += f.x + f.y;
@@ -281,42 +297,30 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
 #pragma unroll
             for (int q = 0; q < T; ++q) {
               E two[2] = {Elem<E>::from_f(Pa[q]), Elem<E>::from_f(Pb[q])};
-              Pw[sb][q][pr] = *reinterpret_cast<const uint32_t*>(two);
+              Pw[q][pr] = *reinterpret_cast<const uint32_t*>(two);
             }
           }
         }
-      }
-      }
-      // the operand slot must have been consumed by the MMAs issued from it
-      if (!wwait(&op_empty[os], oph ^ 1, limit, abort_flag, lane, p.err, site(K_DW, 1, 4), (uint32_t)st)) { ok = false; break; }
-      if (active) {
-        uint8_t* a_st = op_buf + os * C::OP_BYTES;
-        uint8_t* b_st = a_st + C::A_BYTES;
+        const uint32_t off = kmajor_off<C::ROWB>(r, (C::ALT ? 0 : grp * C::NSB) + sb);
+        if (is_a) {
 #pragma unroll
-        for (int sb = 0; sb < C::NSB; ++sb) {
-          const uint32_t off = kmajor_off<C::ROWB>(r, grp * C::NSB + sb);
-          if (is_a) {
+          for (int q = 0; q < T; ++q)
+            *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) = make_uint4(Pw[q][0], Pw[q][1], Pw[q][2], Pw[q][3]);
+        } else {
 #pragma unroll
-            for (int q = 0; q < T; ++q)
-              *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + off) =
-                  make_uint4(Pw[sb][q][0], Pw[sb][q][1], Pw[sb][q][2], Pw[sb][q][3]);
-          } else {
+          for (int f = 0; f < G::nreal; ++f)
+            *reinterpret_cast<uint4*>(b_st + f * b_plane + off) = make_uint4(Pw[f][0], Pw[f][1], Pw[f][2], Pw[f][3]);
 #pragma unroll
-            for (int f = 0; f < G::nreal; ++f)
-              *reinterpret_cast<uint4*>(b_st + f * b_plane + off) =
-                  make_uint4(Pw[sb][f][0], Pw[sb][f][1], Pw[sb][f][2], Pw[sb][f][3]);
-#pragma unroll
-            for (int k = 1; k <= G::ncomplex; ++k) {
-              const int pr = G::nreal + 2 * (k - 1);
-              const int q = G::nreal + 3 * (k - 1);
-              // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G)
-              const uint32_t* u0 = swap ? Pw[sb][pr] : Pw[sb][pr + 1];
-              const uint32_t* u1 = swap ? Pw[sb][pr + 1] : Pw[sb][pr];
-              *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-              *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-              *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
-                  make_uint4(packed::neg2(u0[0]), packed::neg2(u0[1]), packed::neg2(u0[2]), packed::neg2(u0[3]));
-            }
+          for (int k = 1; k <= G::ncomplex; ++k) {
+            const int pr = G::nreal + 2 * (k - 1);
+            const int q = G::nreal + 3 * (k - 1);
+            // M = d: (Im X, Re X, -Im X);  M = c: (Re G, Im G, -Re G)
+            const uint32_t* u0 = swap ? Pw[pr] : Pw[pr + 1];
+            const uint32_t* u1 = swap ? Pw[pr + 1] : Pw[pr];
+            *reinterpret_cast<uint4*>(b_st + (q + 0) * b_plane + off) = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+            *reinterpret_cast<uint4*>(b_st + (q + 1) * b_plane + off) = make_uint4(u1[0], u1[1], u1[2], u1[3]);
+            *reinterpret_cast<uint4*>(b_st + (q + 2) * b_plane + off) =
+                make_uint4(packed::neg2(u0[0]), packed::neg2(u0[1]), packed::neg2(u0[2]), packed::neg2(u0[3]));
           }
         }
       }
@@ -328,8 +332,10 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ 
         mbar_arrive(&raw_empty[rs]);
         mbar_arrive(&op_full[os]);
       }
-      if (++rs == C::RAW_STAGES) { rs = 0; rph ^= 1; }
-      if (++os == C::OP_STAGES) { os = 0; oph ^= 1; }
+      rs += STEP;
+      if (rs >= C::RAW_STAGES) { rs -= C::RAW_STAGES; rph ^= 1; }
+      os += STEP;
+      if (os >= C::OP_STAGES) { os -= C::OP_STAGES; oph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
     // The next kernel (the split reduction) may be scheduled once every role
