@@ -364,12 +364,12 @@ cudaError_t launch_tc_apply_gauss(const Handle& h, const void* in, void* out, in
 // FP32 handles on the tensor cores, 3xTF32 (eqlin_tc32.cu): T in {1, 2, 4};
 // forward and input gradient, and the pretransform into the hi/lo images.
 // tc32_pass_ok: the pass's reduction is short enough for the FP32-level
-// error bound (at most 384 MMAs into one accumulator: K <= 1024 for T = 1,
-// 2 and K <= 512 for T = 4, whose complex accumulators take two block
+// error bound (at most 256 MMAs into one accumulator: K <= 680 for T = 1,
+// 2 and K <= 336 for T = 4, whose complex accumulators take two block
 // products per stage).
 bool tc32_supported(const Handle& h);
 bool tc32_pass_ok(const Handle& h, bool backward);
-// dW, db (eqlin_tc32_dw.cu), token chunks of at most 384 MMAs per accumulator
+// dW, db (eqlin_tc32_dw.cu), token chunks of at most 256 MMAs per accumulator
 bool tc32_dw_supported(const Handle& h);
 size_t tc32_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);
 cudaError_t launch_tc32_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db, int64_t N,

@@ -13,13 +13,15 @@
 //
 // The tensor core adds each MMA's products into the accumulator with a
 // rounding of its own, whose error grows with the number of MMAs that feed
-// one accumulator.  So one accumulator takes at most 384 MMAs, as in the
-// forward: 1024 tokens for T = 1, 2 (three MMAs per 8-token stage), 512 for
-// T = 4 (six into a complex accumulator).  A token range longer than
-// (splits x that) runs as several launches ("passes") over consecutive
-// token ranges, the first writing the per-split partial planes and the later
-// ones adding to them in IEEE FP32 (each split's slot belongs to one CTA per
-// pass, so the sums are deterministic).  The
+// one accumulator (measured: about 1.5e-8 to 1.9e-8 relative error per MMA).
+// So one accumulator takes at most 256 MMAs, as in the forward: 672 tokens
+// for T = 1, 680 for T = 2 (three MMAs per 8 tokens), 336 for T = 4 (six into
+// a complex accumulator).  A token range longer than
+// (splits x that) runs as more waves of CTAs, each split with its own partial
+// slot, up to four per SM and tile; beyond that as several launches
+// ("passes") over consecutive token ranges, the first writing the per-split
+// partial planes and the later ones adding to them in IEEE FP32 (each split's
+// slot belongs to one CTA per pass, so the sums are deterministic).  The
 // fixed-order reduction over splits and the inverse DFT then follow
 // (launch_dw_reduce).
 //
@@ -107,10 +109,9 @@ struct Cfg {
   static constexpr int PRODUCER = TR_WARPS, MMA_WARP = TR_WARPS + 1;
   static constexpr int THREADS = (TR_WARPS + 1 + NMMA) * 32;
   static constexpr int PF_STAGES = 16;
-  // tokens one accumulator takes: 384 MMAs (three, or six into a complex
-  // accumulator, per 8-token K step)
-  static constexpr int CHUNK_MAX = 384 / (3 * (G::ncomplex > 0 ? 2 : 1)) * 8;
-  static_assert(CHUNK_MAX % BKN == 0, "whole stages per chunk");
+  // tokens one accumulator takes: at most 256 MMAs (three, or six into a
+  // complex accumulator, per 8-token K step), whole stages
+  static constexpr int CHUNK_MAX = 256 / (3 * (G::ncomplex > 0 ? 2 : 1)) * 8 / BKN * BKN;
 };
 
 struct Params {
@@ -364,16 +365,22 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
           }
           tmem_wait_ld();
           if (row_ok) {
+            // a later pass adds to the partials: the chunk's T x 8 loads go out
+            // together, before any of its stores, so they wait one memory
+            // latency rather than one each
+            float add[T][8];
+#pragma unroll
+            for (int q = 0; q < T; ++q)
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                add[q][i] = (p.accumulate && n0 + cc + i < ndim) ? base[q * plane + (int64_t)(n0 + cc + i) * p.mdim]
+                                                                 : 0.f;
 #pragma unroll
             for (int q = 0; q < T; ++q)
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const int n = n0 + cc + i;
-                if (n < ndim) {
-                  float* dst = base + q * plane + (int64_t)n * p.mdim;
-                  const float v = __uint_as_float(rg[q][i]);
-                  *dst = p.accumulate ? *dst + v : v;
-                }
+                if (n < ndim) base[q * plane + (int64_t)n * p.mdim] = add[q][i] + __uint_as_float(rg[q][i]);
               }
           }
         }
@@ -481,6 +488,8 @@ tc32_dw_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant_
   }
 }
 
+constexpr int MAX_WAVES = 4;
+
 struct Plan {
   int BC, n_mt, n_nt, splits;   // splits: partial slots (CTAs per tile in a full pass)
   bool swap;
@@ -489,8 +498,9 @@ struct Plan {
 };
 
 // M side: d, unless c pads less to a multiple of 128.  N side: tiles of BC
-// channels (a multiple of 16, at most 128) that split it evenly.  Splits:
-// the SMs per tile; passes: as many as keep every chunk within CHUNK_MAX.
+// channels (a multiple of 16, at most BC_MAX) that split it evenly.  Splits:
+// the SMs per tile, times the waves (at most MAX_WAVES) that keep every chunk
+// within CHUNK_MAX; passes: as many more as that still needs.
 template <int T>
 static Plan plan(int64_t Cp, int64_t Dp, int64_t N, int sm_count) {
   using C = Cfg<T>;
@@ -507,9 +517,15 @@ static Plan plan(int64_t Cp, int64_t Dp, int64_t N, int sm_count) {
   int s = sm_count / tiles;
   if (s < 1) s = 1;
   if (N < 1) N = 1;
-  pl.passes = (int)((N + (int64_t)s * C::CHUNK_MAX - 1) / ((int64_t)s * C::CHUNK_MAX));
+  // up to MAX_WAVES waves of CTAs in one launch, each split with a partial
+  // slot of its own (the reduction sums them); passes only beyond that
+  const int64_t per_wave = (int64_t)s * C::CHUNK_MAX;
+  int64_t waves = (N + per_wave - 1) / per_wave;
+  if (waves > MAX_WAVES) waves = MAX_WAVES;
+  const int64_t sp = s * waves;               // splits per pass
+  pl.passes = (int)((N + sp * C::CHUNK_MAX - 1) / (sp * C::CHUNK_MAX));
   const int64_t per_pass = (N + pl.passes - 1) / pl.passes;
-  pl.chunk = ((per_pass + s - 1) / s + C::BKN - 1) / C::BKN * C::BKN;
+  pl.chunk = ((per_pass + sp - 1) / sp + C::BKN - 1) / C::BKN * C::BKN;
   pl.splits = (int)((per_pass + pl.chunk - 1) / pl.chunk);
   return pl;
 }

@@ -112,6 +112,9 @@ SMALL = [  # (T, C', D', N, dtype)
     # d on the N side, db from rows past 128), and token ranges of two passes
     (2, 256, 128, 5000, "f32"), (2, 128, 200, 3000, "f32"),
     (2, 128, 128, 160000, "f32"), (1, 128, 128, 160000, "f32"),
+    # FP32 dW over more than four waves of token chunks: two passes, the
+    # second adding to the first's partial planes
+    (2, 16, 24, 700000, "f32"),
 ]
 
 
@@ -138,8 +141,9 @@ def test_small_parity(T, Cp, Dp, N, dt):
 # exact in the FP32 accumulator.
 EXACT = [
     (4, 64, 64, 1024, "f32", 4), (2, 64, 48, 515, "f32", 4), (1, 32, 64, 300, "f32", 4),
-    # FP32 dW over two token passes (the second adds to the first's partials)
-    (4, 64, 64, 100000, "f32", 1),
+    # FP32 dW over three waves of token chunks, and over two passes (the
+    # second adds to the first's partials)
+    (4, 64, 64, 100000, "f32", 1), (4, 16, 16, 250000, "f32", 1),
     (4, 16, 16, 700, "f16", 4), (2, 16, 16, 300, "f16", 4), (4, 16, 8, 129, "f16", 4),
     (4, 8, 8, 400, "bf16", 2), (2, 8, 8, 200, "bf16", 2),
     # 512 token tiles: 3-4 output tiles per persistent CTA of the forward and
@@ -534,10 +538,10 @@ def test_backend_is_reported_per_pass():
     for T in (3, 6, 8):
         assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt", T
     # FP32 passes whose reduction is too long for the 3xTF32 error bound
-    # (more than 384 MMAs into one accumulator) run on the SIMT kernels
-    assert eqlin.create(4, 520, 16, "f32").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
-    assert eqlin.create(2, 16, 1032, "f32").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
-    assert eqlin.create(1, 1024, 1024, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
+    # (more than 256 MMAs into one accumulator) run on the SIMT kernels
+    assert eqlin.create(4, 344, 16, "f32").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
+    assert eqlin.create(2, 16, 688, "f32").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
+    assert eqlin.create(1, 680, 680, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05"
     assert eqlin.create(4, 6, 16, "f16").backend() == "fwd=simt dx=tcgen05 dw=tcgen05"
     assert eqlin.create(4, 16, 6, "bf16").backend() == "fwd=tcgen05 dx=simt dw=tcgen05"
 
