@@ -600,20 +600,34 @@ def main(argv=None):
         dbuf = [{k: torch.empty_like(s["sets"][0][k]) for k in ("x", "gy")} for s in st]
         h2d = sum(host[i][k].numel() * host[i][k].element_size() for i in range(len(st)) for k in ("x", "gy", "W", "b"))
         d2h = sum(host[i][k].numel() * host[i][k].element_size() for i in range(len(st)) for k in ("y", "dx", "dW", "db"))
-        # host->device copies and kernels on the main streams, device->host
-        # copies of each layer's results on a third stream, so that they overlap
-        # the next layer's uploads and kernels; a layer's outputs are
-        # overwritten (next step) only after its copies have run
+        # Host->device copies of every layer's inputs on an upload stream,
+        # kernels on the main streams, device->host copies of each layer's
+        # results on a download stream, so that both copy directions and the
+        # kernels overlap.  A layer's input buffers are overwritten (next step)
+        # only after its kernels have read them, and its outputs only after
+        # their copies have run.
+        h2d_stream = torch.cuda.Stream(device=dev)
         d2h_stream = torch.cuda.Stream(device=dev)
         copied = [None] * len(st)
+        consumed = [None] * len(st)
 
         def e2e_step():
+            uploaded = []
             for i, s in enumerate(st):
                 hb, db_ = host[i], dbuf[i]
-                db_["x"].copy_(hb["x"], non_blocking=True)
-                db_["gy"].copy_(hb["gy"], non_blocking=True)
-                s["W"].copy_(hb["W"], non_blocking=True)
-                s["b"].copy_(hb["b"], non_blocking=True)
+                with torch.cuda.stream(h2d_stream):
+                    if consumed[i] is not None:
+                        h2d_stream.wait_event(consumed[i])
+                    db_["x"].copy_(hb["x"], non_blocking=True)
+                    db_["gy"].copy_(hb["gy"], non_blocking=True)
+                    s["W"].copy_(hb["W"], non_blocking=True)
+                    s["b"].copy_(hb["b"], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d_stream)
+                    uploaded.append(ev)
+            for i, s in enumerate(st):
+                hb, db_ = host[i], dbuf[i]
+                stream.wait_event(uploaded[i])
                 if copied[i] is not None:
                     stream.wait_event(copied[i])
                 eqlin.set_weights(s["h"], s["W"], s["b"])
@@ -628,6 +642,8 @@ def main(argv=None):
                     stream.wait_stream(side)
                 if dist:
                     dp.allreduce_grads((s["dW"], s["db"]))
+                consumed[i] = torch.cuda.Event()
+                consumed[i].record(stream)
                 d2h_stream.wait_stream(stream)
                 with torch.cuda.stream(d2h_stream):
                     for k in ("y", "dx", "dW", "db"):
@@ -646,6 +662,7 @@ def main(argv=None):
         for _ in range(ke):
             e2e_step()
         stream.wait_stream(d2h_stream)      # the last results are on the host
+        stream.wait_stream(h2d_stream)
         b.record(stream)
         torch.cuda.synchronize()
         ems = a.elapsed_time(b) / ke
