@@ -38,11 +38,14 @@
  * - Supported T: 1, 2, 3, 4, 6, 8.  Other values give EQLIN_ERR_UNSUPPORTED.
  *   The tensor-core kernels serve f16/bf16 for every supported T (T = 3 and 6
  *   with FP32 butterflies and the sqrt(3)/2 twiddles).  FP32 handles of
- *   order T = 1, 2, 4 run the forward and dx on the tensor cores as 3xTF32
- *   (each operand split into two TF32 terms, three TF32 products per real
- *   product, FP32 accumulation; an FP32-level result), and their weight
- *   gradient on the CUDA cores; FP32 handles of order 3, 6, 8 run every pass
- *   on the CUDA cores.  The stash forms (fused backward) take T = 1, 2, 4, 8.
+ *   order T = 1, 2, 4 run every pass on the tensor cores as 3xTF32 (each
+ *   operand split into two TF32 terms, three TF32 products per real product,
+ *   FP32 accumulation; an FP32-level result, within 1e-5 relative Frobenius
+ *   error), except a forward or dx whose reduction would feed more than 256
+ *   MMAs into one accumulator (K = C' or D' above 680 for T = 1, 2, above
+ *   336 for T = 4), which runs on the CUDA cores; FP32 handles of order 3, 6,
+ *   8 run every pass on the CUDA cores.  The stash forms (fused backward)
+ *   take f16/bf16 and T = 1, 2, 4, 8.
  *   eqlin_backward_dw_noalloc takes T = 1, 2, 4, 8 only.
  * - Nothing is thrown across the ABI; every call returns a status.
  * - A handle may be used from one host thread at a time.
@@ -292,9 +295,9 @@ EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
  * Which kernel family serves each pass of this handle, as
  * "fwd=<k> dx=<k> dw=<k>", where <k> is "tcgen05" (the tensor-core kernels)
  * or "simt" (the FP32 CUDA-core kernels).  f32 handles run tcgen05 (3xTF32)
- * for the forward and dx when T is 1, 2 or 4, and simt for their weight
- * gradient and for every pass of other orders.  f16/bf16 handles run tcgen05
- * except where the shape rules it out:
+ * in every pass when T is 1, 2 or 4, except a forward or dx past the
+ * reduction-length limit above, and simt for every pass of other orders.
+ * f16/bf16 handles run tcgen05 except where the shape rules it out:
  * a forward (dx) whose K = C' (D') is not a multiple of 8 -- the row pitch of
  * that pass's weight tiles would not be a TMA stride.  For logging and tests; the string lives as long as the handle.
  */
