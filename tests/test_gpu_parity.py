@@ -144,6 +144,12 @@ EXACT = [
     # FP32 dW over three waves of token chunks, and over two passes (the
     # second adds to the first's partials)
     (4, 64, 64, 100000, "f32", 1), (4, 16, 16, 250000, "f32", 1),
+    # FP32 dW with N sides past 128 channels (two rows per transform thread;
+    # T = 1 with 16-token stages)
+    (2, 200, 256, 2000, "f32", 2), (1, 160, 256, 1500, "f32", 2),
+    # f16 dW chunks of 27 stages: the two transform groups, on alternate
+    # stages, take 14 and 13
+    (4, 16, 16, 63936, "f16", 2),
     (4, 16, 16, 700, "f16", 4), (2, 16, 16, 300, "f16", 4), (4, 16, 8, 129, "f16", 4),
     (4, 8, 8, 400, "bf16", 2), (2, 8, 8, 200, "bf16", 2),
     # 512 token tiles: 3-4 output tiles per persistent CTA of the forward and
