@@ -321,7 +321,7 @@ def roofline_of(L, kind, us, pk, fused=False):
     r = {"us": round(us, 2), "tflops": flop / t / 1e12 if flop else 0.0, "gbs": byt / t / 1e9,
          "frac_tensor": flop / t / tens if flop else 0.0, "frac_hbm": byt / t / hbm,
          "frac_roofline": max(flop / tens, byt / hbm) / t}
-    if L.dtype == "f32" and L.T in (1, 2, 4) and kind in ("fwd", "dx", "dw"):
+    if L.dtype == "f32" and (L.T in (1, 2, 4) or (L.T == 8 and kind in ("fwd", "dx"))) and kind != "set_weights":
         # 3xTF32: three kind::tf32 MMAs per real product, against the TF32
         # peak (the measured bf16 peak x the nominal TF32/BF16 ratio of 1/2)
         mma_flop, peak = 3 * flop, pk["bf16"] / 2
@@ -449,9 +449,9 @@ def sub_measurements(dev, pk, reps, fused):
         "EQ-Swin-T stage-1 step (f16)": workloads.WORKLOADS["eq-swin-t-s1-f16-fwdbwd"],
         "cyclic T=8 f16 layer": t8,
         "cyclic T=3 and T=6 f16 layers": t36,
-        # FP32: every pass on 3xTF32 tensor cores for T = 2, 4; T = 8 on the
-        # CUDA cores
-        "cyclic FP32 layers (3xTF32 for T = 2, 4)": f32,
+        # FP32: every pass on 3xTF32 tensor cores for T = 2, 4; T = 8's
+        # forward and dx on them, its dW on the CUDA cores
+        "cyclic FP32 layers (3xTF32)": f32,
     }
     stream = torch.cuda.current_stream()
     for name, layers in subs.items():

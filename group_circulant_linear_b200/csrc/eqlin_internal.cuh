@@ -211,10 +211,12 @@ __host__ __device__ inline int64_t wtile_elems(int T, int bo, int64_t rows, int6
 // chunk j ^ ((r >> 2) & 1).  Tile widths: the widest MMAs that fit (an
 // N = 128 TF32 MMA already reads its operands at the SM's shared-memory rate,
 // so narrower tiles are bandwidth-bound): 256 (T = 1), 256 or 128 (T = 2),
-// 128, 64 or 32 (T = 4), the one that pads O least, the wider on a tie.
+// 128, 64 or 32 (T = 4), the one that pads O least, the wider on a tie; 32
+// for T = 8 (its 16 hi/lo A planes fill most of shared memory).
 constexpr int TC32_BK = 8;
 inline int tc32_pick_bo(int T, int64_t O) {
   if (T == 1) return 256;
+  if (T == 8) return 32;
   const int widths2[2] = {256, 128}, widths4[3] = {128, 64, 32};
   const int* w = T == 2 ? widths2 : widths4;
   const int n = T == 2 ? 2 : 3;
@@ -361,15 +363,16 @@ cudaError_t launch_tc_apply(const Handle& h, bool backward, const void* in, void
 // The p4 forward with the complex products in three real GEMMs (Gauss), for
 // comparison; needs the handle's Gauss image (h.wt_gauss).
 cudaError_t launch_tc_apply_gauss(const Handle& h, const void* in, void* out, int64_t N, cudaStream_t st);
-// FP32 handles on the tensor cores, 3xTF32 (eqlin_tc32.cu): T in {1, 2, 4};
+// FP32 handles on the tensor cores, 3xTF32 (eqlin_tc32.cu): T in {1, 2, 4, 8};
 // forward and input gradient, and the pretransform into the hi/lo images.
 // tc32_pass_ok: the pass's reduction is short enough for the FP32-level
 // error bound (at most 256 MMAs into one accumulator: K <= 680 for T = 1,
-// 2 and K <= 336 for T = 4, whose complex accumulators take two block
+// 2 and K <= 336 for T = 4, 8, whose complex accumulators take two block
 // products per stage).
 bool tc32_supported(const Handle& h);
 bool tc32_pass_ok(const Handle& h, bool backward);
-// dW, db (eqlin_tc32_dw.cu), token chunks of at most 256 MMAs per accumulator
+// dW, db (eqlin_tc32_dw.cu) for T in {1, 2, 4}, token chunks of at most 256
+// MMAs per accumulator
 bool tc32_dw_supported(const Handle& h);
 size_t tc32_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count);
 cudaError_t launch_tc32_dw(const Handle& h, const void* x, const void* gy, float* dW, float* db, int64_t N,

@@ -53,7 +53,14 @@ using namespace waits;
 template <int T, int BO_>
 struct Cfg {
   using G = Group<T>;
-  static_assert(T == 1 || T == 2 || T == 4, "3xTF32 tiles for T in {1, 2, 4}");
+  static_assert(T == 1 || T == 2 || T == 4 || T == 8, "3xTF32 tiles for T in {1, 2, 4, 8}");
+  // SPLIT (T = 8): the 16 hi/lo A planes of a stage leave room for one
+  // operand slot, so all eight transform warps work on every stage (four
+  // tokens per thread) instead of two groups on alternate stages; with one
+  // slot, alternating groups would wait on phases an mbarrier parity cannot
+  // tell apart.
+  static constexpr bool SPLIT = (T == 8);
+  static constexpr int TOK = SPLIT ? 4 : 8;            // tokens per transform thread and stage
   static constexpr int BM = 128;                       // tokens per tile (MMA M)
   static constexpr int BK = TC32_BK;                   // input channels per stage (one MMA K step)
   static constexpr int BO = BO_;
@@ -89,12 +96,13 @@ struct Cfg {
   // the same transform group)
   static constexpr int BIAS_BYTES = 2 * BO * 4;        // per epilogue half, the tile's bias (FP32)
   static constexpr int BUDGET = 225 * 1024 - BIAS_BYTES;
-  static constexpr int AB_ST = (BUDGET - 2 * OUT_TILE_BYTES - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 3 : 2;
+  static constexpr int AB_ST =
+      SPLIT ? 1 : (BUDGET - 2 * OUT_TILE_BYTES - 3 * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 3 : 2;
   static constexpr int NSTG = (BUDGET - 4 * OUT_TILE_BYTES - AB_ST * (A_BYTES + B_BYTES)) / RAW_BYTES >= 4 ? 2 : 1;
   static constexpr int STAGING = 2 * NSTG * OUT_TILE_BYTES;
   static constexpr int RAW_FIT = (BUDGET - STAGING - AB_ST * (A_BYTES + B_BYTES)) / RAW_BYTES;
-  static constexpr int RAW_ST = (RAW_FIT > 8 ? 8 : RAW_FIT) & ~1;
-  static_assert(RAW_ST >= 2 && AB_ST >= 2, "two slots per ring (the transform groups take alternate stages)");
+  static constexpr int RAW_ST = (RAW_FIT > 8 ? 8 : RAW_FIT) & (SPLIT ? ~0 : ~1);
+  static_assert(RAW_ST >= 2 && (SPLIT || AB_ST >= 2), "two slots per ring (the transform groups take alternate stages)");
   static_assert((A_BYTES + B_BYTES) % 1024 == 0 && RAW_BYTES % 1024 == 0, "1 KB alignment of the swizzled tiles");
   static constexpr int NMMA = (T == 1) ? 1 : 2;
   static constexpr int MMAS = G::nreal + 2 * G::ncomplex;          // block products per stage
@@ -107,11 +115,12 @@ struct Cfg {
                                     NBAR * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
   static constexpr int CH = OUT_EL / T;                // output channels per store chunk
-  static_assert(CH % 8 == 0, "8 channels at a time");
+  static constexpr int SUBCH = CH < 8 ? CH : 8;        // channels per inverse-DFT batch
+  static_assert(CH % SUBCH == 0 && (SUBCH * T) % 4 == 0, "whole 16-byte output chunks per batch");
   static constexpr int NCHUNK = BO / CH;
   static_assert(NCHUNK % 2 == 0, "chunks alternate between the two epilogue halves");
   static constexpr int TR_WARPS = 8;
-  static constexpr int GRP_WARPS = TR_WARPS / 2;
+  static constexpr int GRP_WARPS = SPLIT ? TR_WARPS : TR_WARPS / 2;   // transform warps that fill one stage
   static constexpr int RAW_PRODUCER = TR_WARPS, B_PRODUCER = TR_WARPS + 1;
   static constexpr int MMA_WARP = TR_WARPS + 2, EPI0 = MMA_WARP + NMMA;
   static constexpr int EPI_WARPS = 8;
@@ -134,7 +143,11 @@ struct Params {
 
 template <int N_>
 __device__ __forceinline__ void load_group(const uint8_t* src, float (&v)[N_]) {
-  if constexpr (N_ == 4) {
+  static_assert(N_ == 1 || N_ == 2 || N_ == 4 || N_ == 8, "a channel's T values");
+  if constexpr (N_ == 8) {
+    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 16);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else if constexpr (N_ == 4) {
     const float4 u = *reinterpret_cast<const float4*>(src);
     v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
   } else if constexpr (N_ == 2) {
@@ -208,30 +221,32 @@ tc32_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_const
   if (warp < C::TR_WARPS) {
     // ----------------------------------------------------- transform warps
     // Thread: channel c of the stage (8 per stage) and 8 consecutive tokens,
-    // one 32-byte chunk of a plane row.
-    const int grp = warp / C::GRP_WARPS;
+    // one 32-byte chunk of a plane row (SPLIT: 4 tokens, a 16-byte half).
+    const int grp = C::SPLIT ? 0 : warp / C::GRP_WARPS;
     const int c = lane & 7;
-    const int m = (warp % C::GRP_WARPS) * 32 + 8 * (lane >> 3);
+    const int m = C::SPLIT ? warp * 16 + 4 * (lane >> 3) : (warp % C::GRP_WARPS) * 32 + 8 * (lane >> 3);
     const uint32_t a_off =
-        (uint32_t)((m >> 5) * C::A_LBO + (c >> 2) * C::A_SBO + (c & 3) * 128 + ((((m & 31) >> 3) ^ (c & 3)) << 5));
+        (uint32_t)((m >> 5) * C::A_LBO + (c >> 2) * C::A_SBO + (c & 3) * 128 + ((((m & 31) >> 3) ^ (c & 3)) << 5) +
+                   (C::SPLIT ? ((m >> 2) & 1) * 16 : 0));
     const uint32_t raw_off = (uint32_t)(m * C::RAW_ROWB + c * T * 4);
+    constexpr int STEP = C::SPLIT ? 1 : 2;               // stages between a thread's turns
     int rs = grp % C::RAW_ST, as = grp % C::AB_ST;
     uint32_t rph = 0, aph = 0;
     bool ok = true;
-    for (int64_t it = grp; it < my_tiles * nk; it += 2) {
+    for (int64_t it = grp; it < my_tiles * nk; it += STEP) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_APPLY, 1, 1), (uint32_t)it)) { ok = false; break; }
       const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_off;
-      float v[8][T];
+      float v[C::TOK][T];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) load_group<T>(raw + j * C::RAW_ROWB, v[j]);
+      for (int j = 0; j < C::TOK; ++j) load_group<T>(raw + j * C::RAW_ROWB, v[j]);
       // generic reads of the slot ordered before its next TMA write
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&raw_empty[rs]);
       // group DFT in FP32, then hi = tf32(P), lo = tf32(P - hi)
-      uint32_t hi[T][8], lo[T][8];
+      uint32_t hi[T][C::TOK], lo[T][C::TOK];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < C::TOK; ++j) {
         float P[T];
         G::dft(v[j], P);
 #pragma unroll
@@ -240,32 +255,42 @@ tc32_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_const
           lo[q][j] = f32_to_tf32(P[q] - __uint_as_float(hi[q][j]));
         }
       }
-      rs += 2;
+      rs += STEP;
       if (rs >= C::RAW_ST) { rs -= C::RAW_ST; rph ^= 1; }
       if (!wwait(&ab_empty[as], aph ^ 1, limit, abort_flag, lane, p.err, site(K_APPLY, 1, 4), (uint32_t)it)) { ok = false; break; }
       uint8_t* a_st = a_buf + as * C::A_BYTES;
-      // The 16-byte halves of the 32-byte chunk go in opposite orders for
-      // channels c and c + 4: one store instruction then covers all eight
-      // 16-byte bank groups of a 128-byte row (the two K groups of a stage
-      // sit 512 bytes apart, on the same banks), four wavefronts per warp.
-      const bool swap_halves = (c >> 2) != 0;
-      auto half = [&](const uint32_t (&w)[8], int b) {
-        return make_uint4(w[4 * b], w[4 * b + 1], w[4 * b + 2], w[4 * b + 3]);
-      };
+      if constexpr (C::SPLIT) {
 #pragma unroll
-      for (int q = 0; q < T; ++q) {
-        uint8_t* ph = a_st + q * C::A_PLANE_BYTES + a_off;
-        uint8_t* pl = a_st + (T + q) * C::A_PLANE_BYTES + a_off;
-        const uint4 h0 = half(hi[q], 0), h1 = half(hi[q], 1), l0 = half(lo[q], 0), l1 = half(lo[q], 1);
-        *reinterpret_cast<uint4*>(ph + (swap_halves ? 16 : 0)) = swap_halves ? h1 : h0;
-        *reinterpret_cast<uint4*>(pl + (swap_halves ? 16 : 0)) = swap_halves ? l1 : l0;
-        *reinterpret_cast<uint4*>(ph + (swap_halves ? 0 : 16)) = swap_halves ? h0 : h1;
-        *reinterpret_cast<uint4*>(pl + (swap_halves ? 0 : 16)) = swap_halves ? l0 : l1;
+        for (int q = 0; q < T; ++q) {
+          *reinterpret_cast<uint4*>(a_st + q * C::A_PLANE_BYTES + a_off) =
+              make_uint4(hi[q][0], hi[q][1], hi[q][2], hi[q][3]);
+          *reinterpret_cast<uint4*>(a_st + (T + q) * C::A_PLANE_BYTES + a_off) =
+              make_uint4(lo[q][0], lo[q][1], lo[q][2], lo[q][3]);
+        }
+      } else {
+        // The 16-byte halves of the 32-byte chunk go in opposite orders for
+        // channels c and c + 4: one store instruction then covers all eight
+        // 16-byte bank groups of a 128-byte row (the two K groups of a stage
+        // sit 512 bytes apart, on the same banks), four wavefronts per warp.
+        const bool swap_halves = (c >> 2) != 0;
+        auto half = [&](const uint32_t (&w)[8], int b) {
+          return make_uint4(w[4 * b], w[4 * b + 1], w[4 * b + 2], w[4 * b + 3]);
+        };
+#pragma unroll
+        for (int q = 0; q < T; ++q) {
+          uint8_t* ph = a_st + q * C::A_PLANE_BYTES + a_off;
+          uint8_t* pl = a_st + (T + q) * C::A_PLANE_BYTES + a_off;
+          const uint4 h0 = half(hi[q], 0), h1 = half(hi[q], 1), l0 = half(lo[q], 0), l1 = half(lo[q], 1);
+          *reinterpret_cast<uint4*>(ph + (swap_halves ? 16 : 0)) = swap_halves ? h1 : h0;
+          *reinterpret_cast<uint4*>(pl + (swap_halves ? 16 : 0)) = swap_halves ? l1 : l0;
+          *reinterpret_cast<uint4*>(ph + (swap_halves ? 0 : 16)) = swap_halves ? h0 : h1;
+          *reinterpret_cast<uint4*>(pl + (swap_halves ? 0 : 16)) = swap_halves ? l0 : l1;
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ab_full[as]);
-      as += 2;
+      as += STEP;
       if (as >= C::AB_ST) { as -= C::AB_ST; aph ^= 1; }
     }
     if (!ok) raise_abort(abort_flag, p.err);
@@ -430,7 +455,9 @@ tc32_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_const
           const uint32_t col = acc + ci * C::CH +
                                (q < G::nreal ? q * C::BO
                                              : G::nreal * C::BO + (k - 1) * 2 * C::BO + ((q - G::nreal) & 1) * C::BO);
-          if constexpr (C::CH == 8) {
+          if constexpr (C::CH == 4) {
+            tmem_ld_32x32b_x4(col, *reinterpret_cast<uint32_t(*)[4]>(&rg[q][0]));
+          } else if constexpr (C::CH == 8) {
             tmem_ld_32x32b_x8(col, *reinterpret_cast<uint32_t(*)[8]>(&rg[q][0]));
           } else {
 #pragma unroll
@@ -443,27 +470,26 @@ tc32_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_const
           mbar_arrive(&acc_empty[ab]);
         }
 #pragma unroll
-        for (int sub = 0; sub < C::CH / 8; ++sub) {
-          const int oc = ci * C::CH + sub * 8;
-          float bo8[8];
-          {
-            const float4 b0 = *reinterpret_cast<const float4*>(s_bias + half * C::BO + oc);
-            const float4 b1 = *reinterpret_cast<const float4*>(s_bias + half * C::BO + oc + 4);
-            bo8[0] = b0.x; bo8[1] = b0.y; bo8[2] = b0.z; bo8[3] = b0.w;
-            bo8[4] = b1.x; bo8[5] = b1.y; bo8[6] = b1.z; bo8[7] = b1.w;
-          }
-          // 8 channels x T outputs = 2T 16-byte chunks of this row's 128 bytes
-          float vals[8 * T];
+        for (int sub = 0; sub < C::CH / C::SUBCH; ++sub) {
+          const int oc = ci * C::CH + sub * C::SUBCH;
+          float bo8[C::SUBCH];
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
+          for (int i4 = 0; i4 < C::SUBCH / 4; ++i4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(s_bias + half * C::BO + oc + 4 * i4);
+            bo8[4 * i4] = b4.x; bo8[4 * i4 + 1] = b4.y; bo8[4 * i4 + 2] = b4.z; bo8[4 * i4 + 3] = b4.w;
+          }
+          // SUBCH channels x T outputs = SUBCH*T/4 16-byte chunks of this row's 128 bytes
+          float vals[C::SUBCH * T];
+#pragma unroll
+          for (int cc = 0; cc < C::SUBCH; ++cc) {
             float Pc[T];
 #pragma unroll
-            for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][sub * 8 + cc]);
+            for (int q = 0; q < T; ++q) Pc[q] = __uint_as_float(rg[q][sub * C::SUBCH + cc]);
             G::idft_scaled(Pc, bo8[cc], vals + cc * T);
           }
 #pragma unroll
-          for (int v = 0; v < 2 * T; ++v) {
-            const int j = sub * 2 * T + v;
+          for (int v = 0; v < C::SUBCH * T / 4; ++v) {
+            const int j = sub * (C::SUBCH * T / 4) + v;
             *reinterpret_cast<float4*>(my_row + ((j ^ (r & 7)) << 4)) =
                 make_float4(vals[4 * v], vals[4 * v + 1], vals[4 * v + 2], vals[4 * v + 3]);
           }
@@ -632,7 +658,7 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
 }  // namespace tc32
 
 bool tc32_supported(const Handle& h) {
-  return h.group == EQLIN_GROUP_CYCLIC && h.dtype == EQLIN_F32 && (h.T == 1 || h.T == 2 || h.T == 4) &&
+  return h.group == EQLIN_GROUP_CYCLIC && h.dtype == EQLIN_F32 && (h.T == 1 || h.T == 2 || h.T == 4 || h.T == 8) &&
          tensor_map_encoder() != nullptr;
 }
 
@@ -643,7 +669,7 @@ bool tc32_supported(const Handle& h) {
 bool tc32_pass_ok(const Handle& h, bool backward) {
   if (!tc32_supported(h)) return false;
   const int64_t K = backward ? h.Dp : h.Cp;
-  const int64_t per_stage = h.T == 4 ? 6 : 3;     // MMAs into one accumulator per 8-channel stage
+  const int64_t per_stage = h.T % 4 == 0 ? 6 : 3;   // MMAs into one accumulator per 8-channel stage
   return per_stage * ((K + TC32_BK - 1) / TC32_BK) <= 256;
 }
 
@@ -662,6 +688,7 @@ cudaError_t launch_tc32_apply(const Handle& h, bool backward, const void* in, vo
              : bo == 64 ? tc32::launch_t<4, 64>(h, backward, in, out, N, st)
              : bo == 32 ? tc32::launch_t<4, 32>(h, backward, in, out, N, st)
                         : cudaErrorInvalidValue;
+    case 8: return bo == 32 ? tc32::launch_t<8, 32>(h, backward, in, out, N, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }
@@ -683,6 +710,10 @@ cudaError_t launch_tc32_pretransform(const Handle& h, const float* W, const floa
       break;
     case 4:
       e = launch_pdl(tc32::tc32_pretransform_kernel<4>, grid, dim3(256), 0, st, W, b, (float*)h.wt_fwd,
+                     (float*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
+      break;
+    case 8:
+      e = launch_pdl(tc32::tc32_pretransform_kernel<8>, grid, dim3(256), 0, st, W, b, (float*)h.wt_fwd,
                      (float*)h.wt_bwd, h.bias, (int)h.Cp, (int)h.Dp, h.bo_fwd, h.bo_bwd);
       break;
   }

@@ -142,6 +142,7 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int j) {
 
 template <int N_>
 __device__ __forceinline__ void load_group(const uint8_t* src, float (&v)[N_]) {
+  static_assert(N_ == 1 || N_ == 2 || N_ == 4, "a channel's T values");
   if constexpr (N_ == 4) {
     const float4 u = *reinterpret_cast<const float4*>(src);
     v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
@@ -603,7 +604,7 @@ static cudaError_t launch_t(const Handle& h, const void* x, const void* gy, floa
 
 }  // namespace tc32dw
 
-bool tc32_dw_supported(const Handle& h) { return tc32_supported(h); }
+bool tc32_dw_supported(const Handle& h) { return tc32_supported(h) && h.T != 8; }
 
 size_t tc32_dw_workspace_bytes(int T, int64_t Cp, int64_t Dp, int sm_count) {
   switch (T) {

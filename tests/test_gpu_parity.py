@@ -115,6 +115,9 @@ SMALL = [  # (T, C', D', N, dtype)
     # FP32 dW over more than four waves of token chunks: two passes, the
     # second adding to the first's partial planes
     (2, 16, 24, 700000, "f32"),
+    # FP32 T = 8 forward and dx on 3xTF32 (one operand slot, all transform
+    # warps on every stage): several tiles per CTA, and K not a multiple of 8
+    (8, 128, 96, 20000, "f32"), (8, 20, 12, 300, "f32"),
 ]
 
 
@@ -541,7 +544,8 @@ def test_backend_is_reported_per_pass():
             h.close()
     for T in (1, 2, 4):      # FP32: 3xTF32 tensor cores
         assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=tcgen05", T
-    for T in (3, 6, 8):
+    assert eqlin.create(8, 16, 16, "f32").backend() == "fwd=tcgen05 dx=tcgen05 dw=simt"
+    for T in (3, 6):
         assert eqlin.create(T, 16, 16, "f32").backend() == "fwd=simt dx=simt dw=simt", T
     # FP32 passes whose reduction is too long for the 3xTF32 error bound
     # (more than 256 MMAs into one accumulator) run on the SIMT kernels
