@@ -41,10 +41,11 @@
  *   order T = 1, 2, 4 run every pass on the tensor cores as 3xTF32 (each
  *   operand split into two TF32 terms, three TF32 products per real product,
  *   FP32 accumulation; an FP32-level result, within 1e-5 relative Frobenius
- *   error), except a forward or dx whose reduction would feed more than 256
- *   MMAs into one accumulator (K = C' or D' above 680 for T = 1, 2, above
- *   336 for T = 4), which runs on the CUDA cores; FP32 handles of order 3, 6,
- *   8 run every pass on the CUDA cores.  The stash forms (fused backward)
+ *   error), and order 8 its forward and dx, except a forward or dx whose
+ *   reduction would feed more than 256 MMAs into one accumulator (K = C' or
+ *   D' above 680 for T = 1, 2, above 336 for T = 4, 8), which runs on the
+ *   CUDA cores; the T = 8 weight gradient and FP32 handles of order 3, 6 run
+ *   on the CUDA cores.  The stash forms (fused backward)
  *   take f16/bf16 and T = 1, 2, 4, 8.
  *   eqlin_backward_dw_noalloc takes T = 1, 2, 4, 8 only.
  * - Nothing is thrown across the ABI; every call returns a status.
@@ -295,8 +296,9 @@ EQLIN_API eqlin_status_t eqlin_set_wait_limit(eqlin_t h, uint32_t iterations);
  * Which kernel family serves each pass of this handle, as
  * "fwd=<k> dx=<k> dw=<k>", where <k> is "tcgen05" (the tensor-core kernels)
  * or "simt" (the FP32 CUDA-core kernels).  f32 handles run tcgen05 (3xTF32)
- * in every pass when T is 1, 2 or 4, except a forward or dx past the
- * reduction-length limit above, and simt for every pass of other orders.
+ * in every pass when T is 1, 2 or 4 and in the forward and dx when T is 8,
+ * except a forward or dx past the reduction-length limit above, and simt
+ * otherwise.
  * f16/bf16 handles run tcgen05 except where the shape rules it out:
  * a forward (dx) whose K = C' (D') is not a multiple of 8 -- the row pitch of
  * that pass's weight tiles would not be a TMA stride.  For logging and tests; the string lives as long as the handle.
