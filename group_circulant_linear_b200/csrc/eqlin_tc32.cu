@@ -141,6 +141,14 @@ struct Params {
   uint32_t wait_limit;
 };
 
+// 32 lanes x 32 bits, 4 consecutive columns per thread (the T = 8 epilogue's
+// 4-channel chunks).
+__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
 template <int N_>
 __device__ __forceinline__ void load_group(const uint8_t* src, float (&v)[N_]) {
   static_assert(N_ == 1 || N_ == 2 || N_ == 4 || N_ == 8, "a channel's T values");
