@@ -25,7 +25,8 @@
 //                    hi/lo split, and 2T frequency planes written as
 //                    token-contiguous (MN-major) operands in the 128-byte
 //                    swizzle with 32-byte atoms: an atom is 4 channels x 32
-//                    tokens, eight atoms per plane
+//                    tokens, eight atoms per plane.  T = 8 (one operand slot):
+//                    all eight warps on every stage, 4 tokens per thread
 //   MMA warps        (10, 11) lane 0 of each issues, for the accumulators it
 //                    owns, three MMAs per real product: real frequency f one
 //                    M=128, N=BO product; complex frequency k the block
@@ -33,7 +34,12 @@
 //                    [-Im W ; Re W], N=2*BO each
 //   epilogue warps   (12-19) tcgen05.ld of the frequency planes, inverse DFT
 //                    (scales carried by the weight planes), bias, f32 rows of
-//                    32 outputs into a 128B-swizzled staging tile, TMA store
+//                    32 outputs (32/T channels) into a 128B-swizzled staging
+//                    tile, TMA store
+//
+// Tiles are as wide as fit (BO = 256 for T = 1, 2; 128 for T = 4; 32 for
+// T = 8): an N = 128 TF32 MMA already reads its operands at the SM's
+// shared-memory rate, so narrower MMAs make the stage bandwidth-bound.
 //
 // Every mbarrier wait is bounded; a wait that runs out records a timeout in
 // the handle's error word, raises the CTA's abort flag, and the kernel drains
