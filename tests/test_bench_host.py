@@ -67,6 +67,30 @@ def test_roofline_arithmetic():
     assert r["bound"] == "hbm" and r["frac"] == pytest.approx(S.bytes_dw() / 100e-6 / 6e12)
 
 
+@pytest.mark.parametrize("T,kind,bound", [(2, "fwd", "tensor"), (4, "dw", "tensor"), (8, "dx", "tensor"),
+                                          (8, "dw", "alu"), (3, "fwd", "alu"), (6, "dw", "alu")])
+def test_roofline_fp32_denominators(T, kind, bound):
+    """FP32 passes on 3xTF32 are measured as three TF32 MMAs per product against
+    half the bf16 peak; FP32 passes on the CUDA cores against the nominal FFMA
+    rate; neither against the bf16 ridge that decides f16/bf16 passes."""
+    pk = {"hbm_gbs": 6000.0, "bf16": 1500.0, "bf16_sustained": 1400.0, "source": "test"}
+    L = workloads.Layer("t", T, 96, 96, 4096, "f32", ("fwd", "dx", "dw"))
+    us = 40.0
+    flop = L.actual_flop()
+    r = bench.roofline_of(L, kind, us, pk)
+    assert r["bound"] == bound
+    if bound == "tensor":
+        assert r["peak"] == 750.0 and r["unit"].startswith("TFLOP/s (tf32")
+        assert r["achieved"] == pytest.approx(3 * flop / 40e-6 / 1e12)
+        assert r["frac"] == pytest.approx(3 * flop / 40e-6 / 750e12)
+        assert r["fp32_equiv_tflops"] == pytest.approx(flop / 40e-6 / 1e12)
+    else:
+        ffma = 148 * 128 * 2 * 1.965e9
+        assert r["unit"] == "TFLOP/s (FFMA)" and r["peak"] == pytest.approx(ffma / 1e12)
+        assert r["frac"] == pytest.approx(flop / 40e-6 / ffma)
+    assert r["frac_roofline"] >= r["frac"]
+
+
 def test_cpu_info():
     info = bench.cpu_info()
     assert info["nproc"] == os.cpu_count() and isinstance(info["cpu_model"], str)
