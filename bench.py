@@ -571,6 +571,16 @@ def main(argv=None):
     for li, L in enumerate(layers):
         for kind in ("set_weights",) + tuple(L.passes):
             per[(li, kind)] = time_calls(state, li, kind, KERNEL_REPS, stream)
+    # the same forward / dx calls with the opt-in tail split (eqlin_set_tail_split):
+    # shorter lone calls where the last wave of tiles would leave SMs idle
+    split_us = {}
+    if not args.no_sub:
+        for li, L in enumerate(layers):
+            h = state.st[li]["h"]
+            state.eqlin.set_tail_split(h, True)
+            for kind in (k for k in L.passes if k in ("fwd", "dx")):
+                split_us[f"{L.name}/{kind}"] = round(time_calls(state, li, kind, KERNEL_REPS, stream), 2)
+            state.eqlin.set_tail_split(h, False)
     clk = clocks.stop()
     assert all(e == 0 for e in state.errors()), "device-side timeout in the per-kernel region"
     dom = max(per, key=per.get)
@@ -696,6 +706,7 @@ def main(argv=None):
         "per_call_roofline": per_call,
         "kernel_us_sampling": f"CUDA events around {KERNEL_REPS} back-to-back launches of each call, "
                               "after the headline region",
+        "kernel_us_tail_split": split_us or None,
     }
     state.close()
     del state, st

@@ -75,6 +75,43 @@ struct DeviceGuard {
   }
 };
 
+void free_split(Handle& h) {
+  for (int pass = 0; pass < 2; ++pass) {
+    cudaFree(h.split_ws[pass]);
+    cudaFree(h.split_flags[pass]);
+    h.split_ws[pass] = nullptr;
+    h.split_flags[pass] = nullptr;
+    h.split_pairs[pass] = h.split_cols[pass] = 0;
+  }
+}
+
+// The tail-split workspaces (tc_split_tiles) of the f16/bf16 tensor-core
+// passes long enough to split: one FP32 accumulator per pair of CTAs, with
+// its flags.
+bool alloc_split(Handle& h) {
+  for (int pass = 0; pass < 2; ++pass) {
+    const int64_t K = pass ? h.Dp : h.Cp;
+    if (h.split_ws[pass] || (K + eqlin::TC_BK - 1) / eqlin::TC_BK < eqlin::kSplitMinStages ||
+        !eqlin::tc_supported(h, pass == 1))
+      continue;
+    int cols = h.T * (pass ? h.bo_bwd : h.bo_fwd);
+    if (pass == 0 && h.bo_gauss && 5 * h.bo_gauss > cols) cols = 5 * h.bo_gauss;
+    const int pairs = h.sm_count / 2;
+    const size_t nflags = (size_t)2 * pairs + 1;
+    const bool ok = cudaMalloc(&h.split_ws[pass], (size_t)pairs * 128 * cols * sizeof(float)) == cudaSuccess &&
+                    cudaMalloc(&h.split_flags[pass], nflags * sizeof(int)) == cudaSuccess &&
+                    cudaMemset(h.split_flags[pass], 0, nflags * sizeof(int)) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      free_split(h);
+      return false;
+    }
+    h.split_pairs[pass] = pairs;
+    h.split_cols[pass] = cols;
+  }
+  return true;
+}
+
 void free_all(Handle& h) {
   cudaFree(h.wf_fwd);
   cudaFree(h.wf_bwd);
@@ -85,6 +122,7 @@ void free_all(Handle& h) {
   cudaFree(h.err);
   cudaFree(h.wt_gauss);
   h.wt_gauss = nullptr;
+  free_split(h);
   h.wf_fwd = h.wf_bwd = nullptr;
   h.wt_fwd = h.wt_bwd = nullptr;
   h.bias = h.ws = nullptr;
@@ -392,6 +430,20 @@ eqlin_status_t eqlin_error_detail(eqlin_t hh, uint32_t detail[4]) {
   if (!hh || !detail) return EQLIN_ERR_INVALID_ARG;
   for (int i = 0; i < 4; ++i) detail[i] = hh->h.last_error[i];
   return EQLIN_OK;
+}
+
+eqlin_status_t eqlin_set_tail_split(eqlin_t hh, int enable) {
+  if (!hh) return EQLIN_ERR_INVALID_ARG;
+  Handle& h = hh->h;
+  DeviceGuard g(h.device);
+  // the workspaces may still be in use by this handle's queued launches
+  if (cudaDeviceSynchronize() != cudaSuccess) return EQLIN_ERR_CUDA;
+  if (!enable) {
+    free_split(h);
+    return EQLIN_OK;
+  }
+  if (h.group != EQLIN_GROUP_CYCLIC || h.dtype == EQLIN_F32) return EQLIN_OK;   // no tensor-core split there
+  return alloc_split(h) ? EQLIN_OK : EQLIN_ERR_OOM;
 }
 
 eqlin_status_t eqlin_set_wait_limit(eqlin_t hh, uint32_t iterations) {

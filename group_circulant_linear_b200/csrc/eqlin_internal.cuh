@@ -188,6 +188,24 @@ inline int tc_pick_bo(int T, int64_t O) {
   }
   return best;
 }
+// Tail split of a tc_apply launch.  With ctas persistent CTAs taking tiles
+// round-robin, the last wave holds r = n_tiles mod ctas tiles and leaves the
+// other SMs idle for a whole tile.  When 2r <= ctas, each of those r tiles is
+// split in two along the reduction (stages [0, 3nk/8) and [3nk/8, nk)), so
+// the last wave takes 5/8 of a tile.  The half whose MMAs finish first
+// (usually the shorter) leaves its FP32 accumulator in the handle's
+// workspace; the other adds it before the inverse DFT and stores the tile.
+// Only reductions of at least kSplitMinStages stages are split: the
+// hand-over of a 128 x 384-column accumulator costs a few microseconds.  The
+// split shortens a lone call, but the hand-over is extra work: where other
+// kernels (another stream's) would fill the idle SMs, it costs throughput.
+// So it is off by default (eqlin_set_tail_split).
+constexpr int kSplitMinStages = 16;
+inline int tc_split_tiles(int64_t n_tiles, int ctas, int nk, int pairs) {
+  if (nk < kSplitMinStages || ctas < 2 || n_tiles < 1) return 0;
+  const int64_t r = n_tiles % ctas;
+  return (r > 0 && 2 * r <= ctas && r <= pairs) ? (int)r : 0;
+}
 // Element index of (row, k, plane q) in a tiled weight buffer with tile width
 // bo and n_kb K stages.
 __host__ __device__ inline int64_t wtile_index(int T, int bo, int64_t n_kb, int64_t row, int64_t k, int q) {
@@ -276,6 +294,15 @@ struct Handle {
   float* bias = nullptr;          // [Dp] float32 (zeros when no bias)
   float* ws = nullptr;            // dW split partials
   size_t ws_bytes = 0;
+  // tc_apply tail split (tc_split_tiles), off unless eqlin_set_tail_split
+  // turned it on; then, per pass (0 forward, 1 dx) of at least
+  // kSplitMinStages stages: split_ws [pairs][cols / 4][128 rows][4] FP32
+  // accumulators; split_flags [pairs] claims, [pairs] ready flags and a count
+  // of finished CTAs, all zero between launches.
+  float* split_ws[2] = {nullptr, nullptr};
+  int* split_flags[2] = {nullptr, nullptr};
+  int split_pairs[2] = {0, 0};
+  int split_cols[2] = {0, 0};
   int* err = nullptr;             // device error record, 4 words (eqlin_wait.cuh)
   uint32_t last_error[4] = {0, 0, 0, 0};   // the record eqlin_get_error last read, when not OK
   uint32_t wait_limit = 0;        // 0 = default

@@ -23,11 +23,11 @@
 //                    M=128, N=BO product; for each complex frequency two
 //                    M=128, N=2*BO products that accumulate
 //                    [Re Y | Im Y] = Re X [Re W ; Im W] + Im X [-Im W ; Re W]
-//                    -- R(T) real GEMMs, six for p4.  One thread issues at most
-//                    about one MMA per 160 cycles whatever its size, so two
-//                    issuers split the stage's MMAs (p4: the two real
-//                    frequencies, and the complex block product); an
-//                    accumulator is only ever written by one issuer.
+//                    -- R(T) real GEMMs, six for p4.  Two issuers split the
+//                    stage's MMAs (p4: the two real frequencies, and the
+//                    complex block product), each with its own waits and
+//                    commits; an accumulator is only ever written by one
+//                    issuer.
 //   epilogue warps   (12-19) tcgen05.ld of the frequency planes, inverse DFT
 //                    (the weight planes carry its 1/T and 2/T scales, so this
 //                    is additions only), bias, cast into a 128B-swizzled
@@ -47,6 +47,12 @@
 // transform warps have read it, and an operand slot (the stage's A planes and
 // weight planes) once the MMAs that read it have completed; so loads run
 // ahead of the tensor core by the whole raw ring.
+//
+// Tail split: when the last wave of tiles would leave at least half of the
+// SMs idle, each of its tiles runs as two units on two SMs, each over part of
+// the reduction.  The half that finishes its MMAs first stores its FP32
+// accumulator in the handle's workspace and raises a flag; the other adds it
+// in TMEM and stores the tile (the epilogue warps, below).
 //
 // ("Flash EQ-Linear", technical summary, sections "Abordagem Algoritmica",
 // "Especializacao para o Grupo de Rotacao p4" and "Implementacao": fused data
@@ -165,6 +171,11 @@ struct Cfg {
   static constexpr int THREADS = (EPI0 + EPI_WARPS + (STASH_ ? 1 : 0)) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
   static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
+  // split tiles: float4 per epilogue thread per round of the accumulator
+  // merge, staged in the raw ring (whole 16-column groups, at most 16)
+  static constexpr int SPLIT_RND_FIT = (RAW_ST * RAW_BYTES / (EPI_WARPS * 32 * 16)) & ~3;
+  static constexpr int SPLIT_RND = SPLIT_RND_FIT > 16 ? 16 : SPLIT_RND_FIT;
+  static_assert(SPLIT_RND >= 4 && ACC_COLS % 16 == 0, "one 16-column group per round at least");
 };
 
 struct Params {
@@ -180,6 +191,12 @@ struct Params {
   int* err;
   uint32_t wait_limit;
   uint32_t ab_fmt;     // 0 f16, 1 bf16
+  // tail split (tc_split_tiles): the last n_split tiles run as two halves
+  int n_split;
+  float* split_ws;     // [n_split][ACC_COLS / 4][128 rows][4] FP32 accumulators
+  int* split_claim;    // [n_split] halves that have finished their MMAs
+  int* split_ready;    // [n_split] 1 once the first half's accumulator is stored
+  int* split_done;     // CTAs finished (the last one zeroes the flags)
 };
 
 // Eight floats to eight 16-bit values (round to nearest even), two per conversion.
@@ -226,20 +243,52 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   uint64_t* drain_bar = acc_empty + C::NACC;    // [NMMA]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* split_mode = abort_flag + 1;   // the epilogue's role in a split tile
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t limit = p.wait_limit;
   const int nk = (p.K + C::BK - 1) / C::BK;
-  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...  Tile t covers
-  // (token block, output tile) = (t / n_otiles, t % n_otiles): the output tiles
-  // of one token block run side by side and share its input tile in L2.  The
-  // stash forms order them (t % n_tb, t / n_tb) instead: only output tile 0
-  // stores, and with the first order a CTA's tiles b, b + grid, ... all have
-  // the same output tile whenever n_otiles divides the grid, so half of the
-  // CTAs would do every store.
-  const int64_t my_tiles = p.n_tiles > blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  auto tile_tb = [&](int tile) { return STASH ? tile % p.n_tb : tile / p.n_otiles; };
-  auto tile_ot = [&](int tile) { return STASH ? tile / p.n_tb : tile % p.n_otiles; };
+  // Work units of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...  Tiles
+  // are numbered t = token block * n_otiles + output tile.  Tiles t < n_whole
+  // are whole units (all nk stages); the last n_split tiles are split in two
+  // along the reduction, into units n_whole + 2j (stages [0, mid)) and
+  // n_whole + 2j + 1 (stages [mid, nk)) of pair j, mid = 3 nk / 8: the
+  // shorter half usually finishes first and hands its accumulator over while
+  // the longer one still runs its MMAs.  n_whole is a multiple of
+  // the grid, so the halves fill part of the last wave side by side.  Whole
+  // units follow the tile numbering, so the output tiles of one token block
+  // run side by side and share its input tile in L2.  The stash forms take
+  // the same whole tiles output tile by output tile instead: only output
+  // tile 0 stores, and in the first order a CTA's tiles b, b + grid, ... all
+  // have the same output tile whenever n_otiles divides the grid, so half of
+  // the CTAs would do every store.  Both forms split the same tiles, so their
+  // outputs are identical.
+  struct Unit {
+    int tb, ot, kb0, kb1, pair;   // token block, output tile, stages; pair -1: a whole tile
+  };
+  const int n_whole = (int)p.n_tiles - p.n_split;
+  const int n_units = n_whole + 2 * p.n_split;
+  const int my_units = n_units > (int)blockIdx.x ? (n_units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto unit = [&](int i) -> Unit {
+    const int u = (int)blockIdx.x + i * (int)gridDim.x;
+    if (u >= n_whole) {
+      const int v = u - n_whole, j = v >> 1, mid = (nk * 3) >> 3, t = n_whole + j;
+      return (v & 1) ? Unit{t / p.n_otiles, t % p.n_otiles, mid, nk, j}
+                     : Unit{t / p.n_otiles, t % p.n_otiles, 0, mid, j};
+    }
+    if (!STASH) return Unit{u / p.n_otiles, u % p.n_otiles, 0, nk, -1};
+    // output tile ot holds q + (ot < rem) of the whole tiles
+    const int q = n_whole / p.n_otiles, rem = n_whole % p.n_otiles;
+    if (u < rem * (q + 1)) return Unit{u % (q + 1), u / (q + 1), 0, nk, -1};
+    const int k = u - rem * (q + 1);
+    return Unit{k % q, rem + k / q, 0, nk, -1};
+  };
+  // stages of this CTA: nk per whole tile, mid or nk - mid per split half
+  int my_stages = 0;
+  for (int i = 0; i < my_units; ++i) {
+    const Unit un = unit(i);
+    my_stages += un.kb1 - un.kb0;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::RAW_ST; ++i) {
@@ -293,7 +342,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     int rs = grp % C::RAW_ST, as = grp % C::AB_ST;
     uint32_t rph = 0, aph = 0;
     bool ok = true;
-    for (int64_t it = grp; it < my_tiles * nk; it += 2) {
+    for (int it = grp; it < my_stages; it += 2) {
       if (!wwait_all(&raw_full[rs], rph, limit, abort_flag, p.err, site(K_APPLY, 1, 1), (uint32_t)it)) { ok = false; break; }
       const uint8_t* raw = raw_buf + rs * C::RAW_BYTES + raw_off;
       uint32_t Pw[2][T][4];
@@ -419,19 +468,20 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       int64_t n_raw = 0;
       bool ok = true;
       // L2 prefetch of the raw input tiles PF_STAGES stages ahead of their loads
-      int64_t pf_ti = 0;
+      int pf_ti = 0;
       int pf_kb = 0;
       auto prefetch_next = [&]() {
-        if (pf_ti >= my_tiles) return;
-        const int tile = (int)(blockIdx.x + pf_ti * gridDim.x);
-        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, tile_tb(tile) * C::BM);
-        if (++pf_kb == nk) { pf_kb = 0; ++pf_ti; }
+        if (pf_ti >= my_units) return;
+        const Unit un = unit(pf_ti);
+        if (pf_kb < un.kb0) pf_kb = un.kb0;
+        tma_prefetch_2d(&map_in, pf_kb * C::BK * T, un.tb * C::BM);
+        if (++pf_kb == un.kb1) { pf_kb = 0; ++pf_ti; }
       };
       for (int i = 0; i < C::PF_STAGES; ++i) prefetch_next();
-      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const int m0 = tile_tb(tile) * C::BM;
-        for (int kb = 0; kb < nk; ++kb) {
+      for (int ti = 0; ti < my_units && ok; ++ti) {
+        const Unit un = unit(ti);
+        const int m0 = un.tb * C::BM;
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           prefetch_next();
           if (!bwait(&raw_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 2, 2), (uint32_t)n_raw)) { ok = false; break; }
           mbar_arrive_expect_tx(&raw_full[s], C::RAW_BYTES);
@@ -453,10 +503,10 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       uint32_t ph = 0;
       int64_t n_b = 0;
       bool ok = true;
-      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)tile_ot(tile) * nk * C::B_BYTES;
-        for (int kb = 0; kb < nk; ++kb) {
+      for (int ti = 0; ti < my_units && ok; ++ti) {
+        const Unit un = unit(ti);
+        const uint8_t* wt = reinterpret_cast<const uint8_t*>(p.wtiles) + (int64_t)un.ot * nk * C::B_BYTES;
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!bwait(&ab_empty[s], ph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 3, 4), (uint32_t)n_b)) { ok = false; break; }
           // the stage's Q weight planes are one contiguous, pre-swizzled tile
           mbar_arrive_expect_tx(&ab_full[s], C::B_BYTES);
@@ -490,14 +540,15 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       // moves the 14-bit start-address field by d >> 4 without a carry out.
       const uint64_t a_desc0 = smem_desc_mn(smem_u32(a_buf), C::A_LBO, C::A_SBO);
       const uint64_t b_desc0 = smem_desc(smem_u32(b_buf), C::B_ROWB);
-      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
+      for (int ti = 0; ti < my_units && ok; ++ti) {
+        const Unit un = unit(ti);
         if (!bwait(&acc_empty[ab], acph ^ 1, limit, abort_flag, p.err, site(K_APPLY, 4, 6), (uint32_t)ti)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t acc = tmem_base + ab * C::ACC_COLS;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!bwait(&ab_full[s], ph, limit, abort_flag, p.err, site(K_APPLY, 4, 3), (uint32_t)(ti * nk + kb))) {
             ok = false;
             break;
@@ -505,7 +556,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           tc_fence_after();
           const uint64_t a_d = a_desc0 + (uint64_t)((s * C::A_BYTES) >> 4);
           const uint64_t b_d = b_desc0 + (uint64_t)((s * C::B_BYTES) >> 4);
-          const uint32_t first = kb > 0 ? 1u : 0u;
+          const uint32_t first = kb > un.kb0 ? 1u : 0u;
 #pragma unroll
           for (int f = 0; f < G::nreal; ++f)
             if (C::own_real(f) == mi)
@@ -550,7 +601,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       // after the CTA has left would write into the shared memory of whatever
       // the SM runs next.  (On an aborted run, with fewer commits, the
       // wall-time cap ends the wait.)
-      const int64_t n_st = my_tiles * nk;
+      const int n_st = my_stages;
       for (int i = 0; i < C::AB_ST; ++i)
         if (n_st > i) mbar_wait(&ab_empty[i], (uint32_t)(((n_st - 1 - i) / C::AB_ST) & 1), kDefaultWaitLimit);
     }
@@ -565,11 +616,11 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       int s = 0, pend = -1;
       uint32_t ph = 0;
       bool ok = true;
-      for (int64_t ti = 0; ti < my_tiles && ok; ++ti) {
-        const int tile = (int)(blockIdx.x + ti * gridDim.x);
-        const bool store = tile_ot(tile) == 0;
-        const int m0 = tile_tb(tile) * C::BM;
-        for (int kb = 0; kb < nk; ++kb) {
+      for (int ti = 0; ti < my_units && ok; ++ti) {
+        const Unit un = unit(ti);
+        const bool store = un.ot == 0;
+        const int m0 = un.tb * C::BM;
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!bwait(&a_ready[s], ph, limit, abort_flag, p.err, site(K_APPLY, 6, 7), (uint32_t)(ti * nk + kb))) {
             ok = false;
             break;
@@ -619,22 +670,111 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     int ab = 0;
     uint32_t aph = 0;
     bool ok = true;
-    for (int64_t ti = 0; ti < my_tiles; ++ti) {
-      const int tile = (int)(blockIdx.x + ti * gridDim.x);
+    for (int ti = 0; ti < my_units; ++ti) {
+      const Unit un = unit(ti);
       // this half's copy of the tile's bias, loaded while the MMAs run (the
       // half's previous tile has finished reading it)
       {
-        const int ob = tile_ot(tile) * C::BO;
+        const int ob = un.ot * C::BO;
         for (int i = (e & 3) * 32 + lane; i < C::BO; i += 128)
           s_bias[half * C::BO + i] = (p.bias && ob + i < p.O) ? __ldg(p.bias + ob + i) : 0.f;
       }
-      // the four warps of a half share named barriers, so they decide together
-      const bool got = named_bar_and(
-          1 + half, 128, wwait(&acc_full[ab], aph, limit, abort_flag, lane, p.err, site(K_APPLY, 5, 5), (uint32_t)ti));
+      // the four warps of a half share named barriers, so they decide together.
+      // In a launch with split tiles all eight decide together on every tile:
+      // a split tile's hand-over synchronizes both halves (barrier 3), so
+      // neither half may have left the loop while the other goes on.
+      const bool w = wwait(&acc_full[ab], aph, limit, abort_flag, lane, p.err, site(K_APPLY, 5, 5), (uint32_t)ti);
+      const bool got = p.n_split > 0 ? named_bar_and(3, C::EPI_WARPS * 32, w) : named_bar_and(1 + half, 128, w);
       if (!got) { ok = false; break; }
       tc_fence_after();
-      const int m0 = tile_tb(tile) * C::BM;
-      const int o0 = tile_ot(tile) * C::BO;
+      if (un.pair >= 0) {
+        // Half of a split tile.  The first of the pair to get here (mode 1)
+        // stores its FP32 accumulator in the pair's workspace and raises the
+        // pair's ready flag; the second (mode 2) waits for that flag and adds
+        // the stored accumulator to its own in TMEM, then stores the tile as
+        // usual.  Neither waits for a CTA that has not reached this point.
+        if (e == 0 && lane == 0) {
+          int md = atomicAdd(p.split_claim + un.pair, 1) == 0 ? 1 : 2;
+          if (md == 2 && !flag_wait(p.split_ready + un.pair, 1, limit, abort_flag, p.err, site(K_APPLY, 5, 8),
+                                    (uint32_t)un.pair))
+            md = -1;
+          *split_mode = md;
+        }
+        named_bar_sync(3, C::EPI_WARPS * 32);
+        const int mode = *split_mode;
+        if (mode < 0) { ok = false; break; }
+        // the pair's accumulator image: [ACC_COLS / 4][128 rows][4 columns].
+        // Half h takes the 16-column groups h, h + 2, ... of its rows.
+        float4* part = reinterpret_cast<float4*>(p.split_ws) + (size_t)un.pair * (C::ACC_COLS / 4) * C::BM + r;
+        const uint32_t acc0 = tmem_base + lane_addr + ab * C::ACC_COLS;
+        if (mode == 1) {
+#pragma unroll 1
+          for (int g = half; g < C::ACC_COLS / 16; g += 2) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(acc0 + 16 * g, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              __stcg(part + (4 * g + j) * C::BM, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+          // every thread's stores are ordered before the flag that hands them over
+          __threadfence();
+          named_bar_sync(3, C::EPI_WARPS * 32);
+          if (e == 0 && lane == 0) st_release_gpu(p.split_ready + un.pair, 1);
+          if (++ab == C::NACC) { ab = 0; aph ^= 1; }
+          continue;                    // the partner stores the tile
+        }
+        // mode 2: accumulator += the partner's, in place.  In rounds of
+        // SPLIT_RND float4 per thread: cp.async from L2 into the raw ring,
+        // then a TMEM read-add-write of each 16-column group.  The ring is
+        // idle: a split half is its CTA's last unit (units n_whole and on lie
+        // in the last wave), and once its MMAs are done every load of the
+        // CTA has landed and been read.
+        const int te = e * 32 + lane;
+        constexpr int NG = C::ACC_COLS / 16;
+        constexpr int GPR = C::SPLIT_RND / 4;          // groups per round
+#pragma unroll 1
+        for (int g0 = half; g0 < NG; g0 += 2 * GPR) {
+#pragma unroll
+          for (int x = 0; x < GPR; ++x) {
+            const int g = g0 + 2 * x;
+            if (g < NG) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                cp_async_16(raw_buf + ((4 * x + j) * C::EPI_WARPS * 32 + te) * 16, part + (4 * g + j) * C::BM);
+            }
+          }
+          cp_async_commit();
+          cp_async_wait_all();
+#pragma unroll 1
+          for (int x = 0; x < GPR; ++x) {
+            const int g = g0 + 2 * x;
+            if (g >= NG) break;
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(acc0 + 16 * g, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 a = *reinterpret_cast<const float4*>(raw_buf + ((4 * x + j) * C::EPI_WARPS * 32 + te) * 16);
+              v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + a.x);
+              v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + a.y);
+              v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + a.z);
+              v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + a.w);
+            }
+            tmem_st_32x32b_x16(acc0 + 16 * g, v);
+          }
+        }
+        // both halves' sums are in TMEM before either reads the other's columns
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar_sync(3, C::EPI_WARPS * 32);
+        tc_fence_after();
+      }
+      const int m0 = un.tb * C::BM;
+      const int o0 = un.ot * C::BO;
       const uint32_t acc = tmem_base + lane_addr + ab * C::ACC_COLS;
 #pragma unroll 1
       for (int ci = half; ci < C::NCHUNK; ci += 2) {
@@ -757,6 +897,19 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  if (p.n_split > 0 && threadIdx.x == 0) {
+    // the last CTA to finish (every other one is past its last use of the
+    // pairs' flags) zeroes them for the next launch
+    __threadfence();
+    if (atomicAdd(p.split_done, 1) == (int)gridDim.x - 1) {
+      __threadfence();
+      for (int j = 0; j < p.n_split; ++j) {
+        p.split_claim[j] = 0;
+        p.split_ready[j] = 0;
+      }
+      *p.split_done = 0;
+    }
+  }
 }
 
 // ------------------------------------------------------------------- host
@@ -824,13 +977,29 @@ static cudaError_t launch_t(const Handle& h, bool backward, const void* in, void
   p.err = h.err;
   p.wait_limit = h.wait_limit ? h.wait_limit : kDefaultWaitLimit;
   p.ab_fmt = std::is_same<E, __half>::value ? 0u : 1u;
+  // the tail split, where the handle holds a workspace for this pass
+  const int pass = backward ? 1 : 0;
+  p.n_split = 0;
+  p.split_ws = nullptr;
+  p.split_claim = p.split_ready = p.split_done = nullptr;
+  if (h.split_ws[pass] && C::ACC_COLS <= h.split_cols[pass])
+    p.n_split = tc_split_tiles(p.n_tiles, h.sm_count, (K + C::BK - 1) / C::BK, h.split_pairs[pass]);
+  if (p.n_split > 0) {
+    int* f = h.split_flags[pass];
+    p.split_ws = h.split_ws[pass];
+    p.split_claim = f;
+    p.split_ready = f + h.split_pairs[pass];
+    p.split_done = f + 2 * h.split_pairs[pass];
+  }
 
   {
     const cudaError_t e =
         set_smem_limit(reinterpret_cast<const void*>(tc_apply_kernel<T, BO, E, STASH, GAUSS>), C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
-  int64_t grid = p.n_tiles < h.sm_count ? p.n_tiles : h.sm_count;
+  const int64_t n_units = p.n_tiles + p.n_split;
+  if (n_units > 0x7FFFFFFF) return cudaErrorInvalidValue;     // the kernel counts tiles in 32 bits
+  int64_t grid = n_units < h.sm_count ? n_units : h.sm_count;
   if (grid < 1) grid = 1;
   const cudaError_t e = launch_pdl(tc_apply_kernel<T, BO, E, STASH, GAUSS>, dim3((unsigned)grid), dim3(C::THREADS),
                                    C::SMEM_BYTES, st, map_in, map_out, map_stash, p);

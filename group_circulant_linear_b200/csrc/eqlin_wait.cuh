@@ -60,6 +60,26 @@ __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, uint32_t l
   return false;
 }
 
+// Wait until the global flag reads `want` (GPU-scope acquire), bounded and
+// recorded as the mbarrier waits are.
+__device__ __forceinline__ bool flag_wait(const int* flag, int want, uint32_t limit, volatile int* abort_flag,
+                                          int* err, uint32_t where, uint32_t iter) {
+  const uint64_t t0 = cycles_now();
+  uint64_t t = t0;
+  uint32_t i = 0;
+  for (; i < limit; ++i) {
+    if (ld_acquire_gpu(flag) == want) return true;
+    __nanosleep(32);
+    if ((i & 15u) == 15u) {
+      if (*abort_flag) return false;
+      t = cycles_now();
+      if (t - t0 > kWaitCycles) break;
+    }
+  }
+  record_timeout(err, where, iter, i, t - t0);
+  return false;
+}
+
 // Lane 0 waits; the warp then agrees on the outcome (and is ordered after the
 // wait), so no lane leaves a loop that holds warp-synchronous operations.
 __device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, uint32_t limit, volatile int* abort_flag,

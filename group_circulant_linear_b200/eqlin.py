@@ -41,6 +41,7 @@ SIGNATURES = {
     "eqlin_get_error": ([_vp], _int),
     "eqlin_error_detail": ([_vp, ctypes.POINTER(ctypes.c_uint32)], _int),
     "eqlin_set_wait_limit": ([_vp, _u32], _int),
+    "eqlin_set_tail_split": ([_vp, _int], _int),
     "eqlin_backend_name": ([_vp], ctypes.c_char_p),
     "eqlin_status_string": ([_int], ctypes.c_char_p),
     "eqlin_launch_count": ([], ctypes.c_uint64),
@@ -283,6 +284,12 @@ def error_detail(h: Handle) -> dict:
     _check(lib().eqlin_error_detail(h.ptr, d), "eqlin_error_detail")
     return {"status": d[0], "kernel": d[1] >> 8, "role": (d[1] >> 4) & 15, "barrier": d[1] & 15,
             "cta": d[2] & 0xFFF, "iteration": d[2] >> 12, "polls": d[3] & 0xFFFFF, "ms": d[3] >> 20}
+
+
+def set_tail_split(h: Handle, enable: bool):
+    """Split the last wave's tiles of the f16/bf16 forward and dx over two SMs
+    each (off by default): shorter lone calls, at the price of extra work."""
+    _check(lib().eqlin_set_tail_split(h.ptr, 1 if enable else 0), "eqlin_set_tail_split")
 
 
 def set_wait_limit(h: Handle, iterations: int):

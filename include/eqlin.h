@@ -286,6 +286,30 @@ EQLIN_API eqlin_status_t eqlin_get_error(eqlin_t h);
 EQLIN_API eqlin_status_t eqlin_error_detail(eqlin_t h, uint32_t detail[4]);
 
 /*
+ * Tail split of the f16/bf16 forward and dx (off by default; enable != 0
+ * turns it on, 0 off).  The tensor-core kernel gives each SM whole tiles of
+ * 128 tokens in turn.  When a call's last wave of tiles would occupy at most
+ * half of the SMs, and its reduction (C' for the forward, D' for dx) spans 256
+ * channels or more, each of those tiles then runs as two parts of the
+ * reduction on two SMs; the part that finishes first hands its FP32
+ * accumulator to the other through a workspace of the handle.  That shortens
+ * a call that runs alone (the EQ-ViT-B fc1 dx and fc2 forward, 198 tiles: 53
+ * -> 50 us), but the hand-over is extra work: where other kernels, on other
+ * streams, would use the idle SMs anyway, it lowers throughput.
+ *
+ * Turning it on allocates, for each such pass, SMs / 2 accumulators of
+ * 128 x T x tile-width floats (at most 256 KB each) and a few flags;
+ * turning it off frees them.  Both synchronize the device.  While it is on,
+ * two calls of the same pass on one handle must not overlap on the GPU
+ * (eqlin_forward, eqlin_forward_stash and eqlin_forward_gauss are one pass;
+ * eqlin_backward_dx and eqlin_backward_dx_stash the other): order them on one
+ * stream.  Results do not depend on which part finishes first; they may
+ * differ from the unsplit call's in the last bit (two partial sums added).
+ * FP32 and dihedral handles accept the call and do not split.
+ */
+EQLIN_API eqlin_status_t eqlin_set_tail_split(eqlin_t h, int enable);
+
+/*
  * Cap, in polling iterations, on every wait inside this handle's kernels
  * (0 restores the default).  A wait that reaches the cap records
  * EQLIN_ERR_TIMEOUT and its kernel returns early instead of spinning.

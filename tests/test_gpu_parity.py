@@ -67,9 +67,11 @@ def _spectrum(v: np.ndarray, ch: int, T: int) -> np.ndarray:
     return np.stack(planes).transpose(0, 2, 1)
 
 
-def _run_all(T, Cp, Dp, dt, inp, passes=("fwd", "dx", "dw")):
+def _run_all(T, Cp, Dp, dt, inp, passes=("fwd", "dx", "dw"), split=False):
     g = _dev(inp)
     layer = eqlin.EQLinear(g["W"], g["b"])
+    if split:
+        eqlin.set_tail_split(layer.h, True)
     out = {}
     if "fwd" in passes:
         out["y"] = layer.forward(g["x"])
@@ -281,6 +283,97 @@ def test_fused_backward(T, Cp, Dp, N, dt):
     check_exact(f"{tag} dW_spectra vs eqlin_backward", dW2, f["dW"])
     check_exact(f"{tag} db_spectra vs eqlin_backward", db2, f["db"])
     assert eqlin.get_error(layer.h) == 0
+
+
+# Tail split (eqlin_set_tail_split; reductions of 16+ stages): the last
+# wave's tiles run as two parts of the reduction, stages [0, 3K/8) and the
+# rest, and the part that finishes second adds the other's FP32 accumulator.
+# (T, C', D', N, dtype, amp): amp > 0 integer inputs, compared bit for bit
+# (bounds as for EXACT); amp = 0 random inputs within the dtype's tolerance.
+# 160 tiles = one wave + 12 split tiles; 40-71 tiles all split; odd stage
+# counts (K = 264: 17 stages, parts of 6 and 11); T = 3, 6 (no stash form).
+SPLIT = [
+    (4, 256, 96, 20480, "f16", 1), (4, 256, 16, 5120, "f16", 1), (4, 16, 256, 5120, "f16", 1),
+    (4, 264, 16, 3000, "f16", 1), (2, 512, 16, 9000, "f16", 1), (1, 512, 32, 4000, "f16", 1),
+    (4, 256, 96, 20480, "bf16", 0), (4, 96, 264, 6000, "bf16", 0), (2, 320, 128, 9000, "f16", 0),
+    (8, 256, 32, 3000, "bf16", 0), (3, 768, 192, 3000, "f16", 0), (6, 256, 64, 3000, "bf16", 0),
+]
+
+
+@pytest.mark.parametrize("T,Cp,Dp,N,dt,amp", SPLIT, ids=lambda v: str(v))
+def test_tail_split(T, Cp, Dp, N, dt, amp):
+    inp = (inputs.make_integer_inputs(T, Cp, Dp, N, dt, seed=3, amp=amp) if amp
+           else inputs.make_inputs(T, Cp, Dp, N, dt, seed=0))
+    layer, out = _run_all(T, Cp, Dp, dt, inp, passes=("fwd", "dx"), split=True)
+    y = oracle.forward(inp["x"], inp["W"], inp["b"])
+    dx = oracle.backward_dx(inp["gy"], inp["W"])
+    tag = f"split T={T} C'={Cp} D'={Dp} N={N} {dt}"
+    if amp:
+        check_exact(f"{tag} y", out["y"], y)
+        check_exact(f"{tag} dx", out["dx"], dx)
+    else:
+        check(f"{tag} y", out["y"], y, TOL[dt])
+        check(f"{tag} dx", out["dx"], dx, TOL[dt])
+    if _fused_capable(T, Cp, Dp, dt):
+        # the stash forms split the same tiles: identical outputs
+        g = _dev(inp)
+        f = _run_fused(layer, g)
+        check_exact(f"{tag} stash y vs split forward", f["y"], out["y"])
+        check_exact(f"{tag} stash dx vs split dx", f["dx"], out["dx"])
+    # switched off again, the same handle computes whole tiles
+    eqlin.set_tail_split(layer.h, False)
+    g = _dev(inp)
+    y0 = layer.forward(g["x"])
+    torch.cuda.synchronize()
+    if amp:
+        check_exact(f"{tag} y unsplit", y0, y)
+    else:
+        check(f"{tag} y unsplit", y0, y, TOL[dt])
+
+
+@pytest.mark.parametrize("T,Cp,Dp,N,dt", [(4, 768, 192, 12608, "bf16"), (4, 264, 96, 3000, "f16"),
+                                          (3, 768, 192, 3000, "f16")], ids=lambda v: str(v))
+def test_split_tiles_repeatable(T, Cp, Dp, N, dt):
+    # the split tiles' hand-over state is reset by each launch: back-to-back
+    # forwards and dx give identical results, whichever part of a pair
+    # finished first
+    inp = inputs.make_inputs(T, Cp, Dp, N, dt, seed=21)
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    eqlin.set_tail_split(layer.h, True)
+    ys = [layer.forward(g["x"]) for _ in range(6)]
+    dxs = [layer.backward_dx(g["gy"]) for _ in range(4)]
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    for i in range(1, len(ys)):
+        check_exact(f"split forward run {i}", ys[i], ys[0])
+    for i in range(1, len(dxs)):
+        check_exact(f"split dx run {i}", dxs[i], dxs[0])
+    # the split tiles are the last ones (the last token blocks): the oracle on
+    # the last 300 rows
+    tail = slice(N - 300, N)
+    check("split forward", ys[0][tail], oracle.forward(inp["x"][tail], inp["W"], inp["b"]), TOL[dt])
+    if T in (1, 2, 4, 8):
+        f = _run_fused(layer, g)
+        check_exact("split forward, stash form", f["y"], ys[0])
+
+
+def test_tail_split_switch():
+    # FP32 and dihedral handles accept the switch and compute as before; an
+    # f16 handle switches on and off repeatedly
+    for T, dt, grp in ((4, "f32", "cyclic"), (2, "bf16", "dihedral"), (4, "f16", "cyclic")):
+        inp = inputs.make_inputs(T, 256, 32, 700, dt, seed=2)
+        g = _dev(inp)
+        layer = eqlin.EQLinear(g["W"], g["b"], group=grp) if grp == "dihedral" else eqlin.EQLinear(g["W"], g["b"])
+        for on in (True, False, True, True, False):
+            eqlin.set_tail_split(layer.h, on)
+        eqlin.set_tail_split(layer.h, True)
+        y = layer.forward(g["x"])
+        torch.cuda.synchronize()
+        assert eqlin.get_error(layer.h) == 0
+        if grp == "cyclic":
+            check(f"switch T={T} {dt} y", y, oracle.forward(inp["x"], inp["W"], inp["b"]), TOL[dt])
+        layer.h.close()
 
 
 def test_stash_forms_reject_what_they_cannot_serve():
