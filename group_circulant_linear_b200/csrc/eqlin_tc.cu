@@ -151,7 +151,7 @@ struct Cfg {
   __host__ __device__ static constexpr int own_cplx(int k) {
     return NMMA == 1 ? 0 : GAUSS ? 1 : (2 * (G::nreal + 2 * (k - 1)) < MMAS) ? 0 : 1;
   }
-  static constexpr int NBAR = 2 * RAW_ST + 3 * AB_ST + 2 * NACC + NMMA;
+  static constexpr int NBAR = 2 * RAW_ST + 3 * AB_ST + 2 * NACC + NMMA + 2;
   // per epilogue half, the bias of the tile's BO channels (FP32)
   static constexpr int BIAS_BYTES = 2 * BO * 4;
   static constexpr int SMEM_BYTES = RAW_ST * RAW_BYTES + AB_ST * (A_BYTES + B_BYTES) + STAGING +
@@ -171,11 +171,14 @@ struct Cfg {
   static constexpr int THREADS = (EPI0 + EPI_WARPS + (STASH_ ? 1 : 0)) * 32;
   static constexpr int W = packed::Words<T>::n;        // 32-bit words per token and channel
   static constexpr int PF_STAGES = 10;                 // L2 prefetch distance of the input tiles
-  // split tiles: float4 per epilogue thread per round of the accumulator
-  // merge, staged in the raw ring (whole 16-column groups, at most 16)
-  static constexpr int SPLIT_RND_FIT = (RAW_ST * RAW_BYTES / (EPI_WARPS * 32 * 16)) & ~3;
-  static constexpr int SPLIT_RND = SPLIT_RND_FIT > 16 ? 16 : SPLIT_RND_FIT;
-  static_assert(SPLIT_RND >= 4 && ACC_COLS % 16 == 0, "one 16-column group per round at least");
+  // split tiles: accumulator columns per round of the merge (a contiguous
+  // MERGE_COLS x 128 x 4 bytes of the stored image), bulk-copied into one
+  // half of the raw ring while the other half's round is added in
+  static constexpr int RAW_HALF = RAW_ST * RAW_BYTES / 2;
+  static constexpr int MERGE_COLS = (ACC_COLS % 64 == 0 && 64 * BM * 4 <= RAW_HALF)   ? 64
+                                    : (ACC_COLS % 32 == 0 && 32 * BM * 4 <= RAW_HALF) ? 32
+                                                                                      : 16;
+  static_assert(ACC_COLS % MERGE_COLS == 0 && MERGE_COLS * BM * 4 <= RAW_HALF, "merge rounds fit half the raw ring");
 };
 
 struct Params {
@@ -241,7 +244,8 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
   uint64_t* acc_full = a_ready + C::AB_ST;
   uint64_t* acc_empty = acc_full + C::NACC;
   uint64_t* drain_bar = acc_empty + C::NACC;    // [NMMA]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + C::NMMA);
+  uint64_t* merge_bar = drain_bar + C::NMMA;    // [2] split tiles: a merge round's bytes landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* split_mode = abort_flag + 1;   // the epilogue's role in a split tile
 
@@ -305,6 +309,7 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
       mbar_init(&acc_empty[i], C::EPI_WARPS * 32);
     }
     for (int i = 0; i < C::NMMA; ++i) mbar_init(&drain_bar[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&merge_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&map_in);
@@ -727,45 +732,68 @@ tc_apply_kernel(const __grid_constant__ CUtensorMap map_in, const __grid_constan
           if (++ab == C::NACC) { ab = 0; aph ^= 1; }
           continue;                    // the partner stores the tile
         }
-        // mode 2: accumulator += the partner's, in place.  In rounds of
-        // SPLIT_RND float4 per thread: cp.async from L2 into the raw ring,
-        // then a TMEM read-add-write of each 16-column group.  The ring is
-        // idle: a split half is its CTA's last unit (units n_whole and on lie
-        // in the last wave), and once its MMAs are done every load of the
-        // CTA has landed and been read.
-        const int te = e * 32 + lane;
-        constexpr int NG = C::ACC_COLS / 16;
-        constexpr int GPR = C::SPLIT_RND / 4;          // groups per round
+        // mode 2: accumulator += the partner's, in place.  The stored image
+        // comes in rounds of MERGE_COLS columns, each one bulk copy into one
+        // half of the raw ring, so that a round lands while the previous one
+        // is added in (TMEM read, add, TMEM write).  The ring is idle: a
+        // split half is its CTA's last unit (units n_whole and on lie in the
+        // last wave), and once its MMAs are done every load of the CTA has
+        // landed and been read.
+        constexpr int RC = C::MERGE_COLS;
+        constexpr int NR = C::ACC_COLS / RC;
+        constexpr int RB = RC * C::BM * 4;
+        const uint8_t* src =
+            reinterpret_cast<const uint8_t*>(p.split_ws) + (size_t)un.pair * C::ACC_COLS * C::BM * 4;
+        const bool lead = e == 0 && lane == 0;
+        int issued = 0;
+        auto issue = [&](int rd) {
+          mbar_arrive_expect_tx(&merge_bar[rd & 1], RB);
+          bulk_load(raw_buf + (rd & 1) * RB, src + (size_t)rd * RB, RB, &merge_bar[rd & 1]);
+          ++issued;
+        };
+        if (lead) {
+          // the partner's generic-proxy stores, acquired through the flag,
+          // are read by the async proxy (bulk copies)
+          fence_proxy_async_all();
+          issue(0);
+          if (NR > 1) issue(1);
+        }
+        bool mok = true;
 #pragma unroll 1
-        for (int g0 = half; g0 < NG; g0 += 2 * GPR) {
-#pragma unroll
-          for (int x = 0; x < GPR; ++x) {
-            const int g = g0 + 2 * x;
-            if (g < NG) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                cp_async_16(raw_buf + ((4 * x + j) * C::EPI_WARPS * 32 + te) * 16, part + (4 * g + j) * C::BM);
-            }
-          }
-          cp_async_commit();
-          cp_async_wait_all();
+        for (int rd = 0; rd < NR; ++rd) {
+          // every thread reads the copied bytes, so every thread waits (acquire)
+          const bool w2 = bwait(&merge_bar[rd & 1], (uint32_t)((rd >> 1) & 1), limit, abort_flag, p.err,
+                                site(K_APPLY, 5, 9), (uint32_t)rd);
+          mok = named_bar_and(3, C::EPI_WARPS * 32, w2);
+          if (!mok) break;
+          const float4* buf = reinterpret_cast<const float4*>(raw_buf + (rd & 1) * RB);
 #pragma unroll 1
-          for (int x = 0; x < GPR; ++x) {
-            const int g = g0 + 2 * x;
-            if (g >= NG) break;
+          for (int g = half; g < RC / 16; g += 2) {
             uint32_t v[16];
-            tmem_ld_32x32b_x16(acc0 + 16 * g, v);
+            tmem_ld_32x32b_x16(acc0 + rd * RC + 16 * g, v);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float4 a = *reinterpret_cast<const float4*>(raw_buf + ((4 * x + j) * C::EPI_WARPS * 32 + te) * 16);
+              const float4 a = buf[(4 * g + j) * C::BM + r];
               v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + a.x);
               v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + a.y);
               v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + a.z);
               v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + a.w);
             }
-            tmem_st_32x32b_x16(acc0 + 16 * g, v);
+            tmem_st_32x32b_x16(acc0 + rd * RC + 16 * g, v);
           }
+          // this buffer's generic reads are done before the next bulk copy into it
+          fence_proxy_async_smem();
+          named_bar_sync(3, C::EPI_WARPS * 32);
+          if (lead && rd + 2 < NR) issue(rd + 2);
+        }
+        if (!mok) {
+          // no copy may land after the CTA has left
+          if (lead)
+            for (int q = 0; q < 2; ++q)
+              if (issued > q) mbar_wait(&merge_bar[q], (uint32_t)(((issued - 1 - q) / 2) & 1), kDefaultWaitLimit);
+          ok = false;
+          break;
         }
         // both halves' sums are in TMEM before either reads the other's columns
         tmem_wait_st();

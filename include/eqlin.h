@@ -293,9 +293,9 @@ EQLIN_API eqlin_status_t eqlin_error_detail(eqlin_t h, uint32_t detail[4]);
  * channels or more, each of those tiles then runs as two parts of the
  * reduction on two SMs; the part that finishes first hands its FP32
  * accumulator to the other through a workspace of the handle.  That shortens
- * a call that runs alone (the EQ-ViT-B fc1 dx and fc2 forward, 198 tiles: 53
- * -> 50 us), but the hand-over is extra work: where other kernels, on other
- * streams, would use the idle SMs anyway, it lowers throughput.
+ * a call that runs alone (the EQ-ViT-B fc1 dx and fc2 forward, 198 tiles:
+ * 51-54 -> 49 us), but the hand-over is extra work: where other kernels, on
+ * other streams, would use the idle SMs anyway, it lowers throughput.
  *
  * Turning it on allocates, for each such pass, SMs / 2 accumulators of
  * 128 x T x tile-width floats (at most 256 KB each) and a few flags;
