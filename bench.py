@@ -71,6 +71,8 @@ def parse(argv=None):
     ap.add_argument("--order", choices=("layer", "training"), default="layer",
                     help="layer: each layer's forward and backward in turn; training: every forward, "
                          "then the backward passes in reverse layer order")
+    ap.add_argument("--tail-split", action="store_true",
+                    help="switch the forward / dx tail split on for every layer (eqlin_set_tail_split)")
     return ap.parse_args(argv)
 
 
@@ -353,7 +355,7 @@ class Layers:
     X = DFT(x) and G = DFT(gy)) and dW/db come from the spectra; otherwise
     dW/db transform x and gy themselves."""
 
-    def __init__(self, layers, dev, rank, seed_base=0, fused=True):
+    def __init__(self, layers, dev, rank, seed_base=0, fused=True, tail_split=False):
         from group_circulant_linear_b200 import eqlin
         self.eqlin = eqlin
         self.layers = layers
@@ -367,6 +369,8 @@ class Layers:
                                        with_gy=("dx" in L.passes or "dw" in L.passes), device=dev)
                     for s in range(N_SETS)]
             h = eqlin.create(L.T, L.Cp, L.Dp, dt)
+            if tail_split:
+                eqlin.set_tail_split(h, True)
             entry = dict(L=L, h=h, W=w["W"], b=w["b"], sets=sets,
                          y=torch.empty((L.N, L.D), dtype=dt, device=dev),
                          dx=torch.empty((L.N, L.C), dtype=dt, device=dev),
@@ -494,7 +498,7 @@ def main(argv=None):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     fused = args.path == "fused"
-    state = Layers(layers, dev, rank, fused=fused)
+    state = Layers(layers, dev, rank, fused=fused, tail_split=args.tail_split)
     eqlin = state.eqlin
     st = state.st
 
@@ -574,7 +578,7 @@ def main(argv=None):
     # the same forward / dx calls with the opt-in tail split (eqlin_set_tail_split):
     # shorter lone calls where the last wave of tiles would leave SMs idle
     split_us = {}
-    if not args.no_sub:
+    if not args.no_sub and not args.tail_split:
         for li, L in enumerate(layers):
             h = state.st[li]["h"]
             state.eqlin.set_tail_split(h, True)
@@ -689,6 +693,7 @@ def main(argv=None):
         "layers": [dict(name=L.name, T=L.T, Cp=L.Cp, Dp=L.Dp, N=L.N, passes=list(L.passes)) for L in layers],
         "path": args.path,
         "order": args.order,
+        "tail_split": args.tail_split,
         "step": ("per layer: set_weights (weight DFT), forward"
                  + (" writing X = DFT(x)" if fused else "")
                  + ", dx" + (" writing G = DFT(gy)" if fused else "")

@@ -91,6 +91,12 @@ def test_roofline_fp32_denominators(T, kind, bound):
     assert r["frac_roofline"] >= r["frac"]
 
 
+def test_tail_split_flag():
+    # off unless asked for: the bench's step keeps the library's default
+    assert bench.parse([]).tail_split is False
+    assert bench.parse(["--tail-split"]).tail_split is True
+
+
 def test_cpu_info():
     info = bench.cpu_info()
     assert info["nproc"] == os.cpu_count() and isinstance(info["cpu_model"], str)
