@@ -77,6 +77,8 @@ def test_null_handle_calls():
     assert L.eqlin_backward_dx_stash(None, None, None, None, 0, None) == -1
     assert L.eqlin_backward_dw_spectra(None, None, None, None, None, 0, None) == -1
     assert L.eqlin_backward(None, None, None, None, None, None, None, 0, None) == -1
+    assert L.eqlin_set_tail_split(None, 1) == -1
+    assert L.eqlin_set_wait_limit(None, 1) == -1
     L.eqlin_destroy(None)
 
 
