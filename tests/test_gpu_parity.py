@@ -235,6 +235,21 @@ def test_gauss_forward_integer_exact(Cp, Dp, N, dt, amp):
     check_exact(f"gauss integer T=4 C'={Cp} D'={Dp} N={N} {dt} y", y3, oracle.forward(inp["x"], inp["W"], inp["b"]))
 
 
+@pytest.mark.parametrize("Cp,Dp,N", [(256, 96, 3000), (272, 64, 20000)], ids=lambda v: str(v))
+def test_gauss_forward_tail_split(Cp, Dp, N):
+    # the three-product forward with the tail split on (five accumulator planes,
+    # 480 or 320 columns handed over): integer inputs, bit for bit
+    inp = inputs.make_integer_inputs(4, Cp, Dp, N, "f16", seed=17, amp=1)
+    g = _dev(inp)
+    layer = eqlin.EQLinear(g["W"], g["b"])
+    eqlin.set_tail_split(layer.h, True)
+    y = torch.empty((N, Dp * 4), dtype=torch.float16, device="cuda")
+    eqlin.forward_gauss(layer.h, g["x"], y)
+    torch.cuda.synchronize()
+    assert eqlin.get_error(layer.h) == 0
+    check_exact(f"gauss split C'={Cp} D'={Dp} N={N} y", y, oracle.forward(inp["x"], inp["W"], inp["b"]))
+
+
 def test_gauss_forward_rejects_what_it_cannot_serve():
     for T, dt in ((2, torch.bfloat16), (8, torch.float16), (4, torch.float32)):
         h = eqlin.create(T, 16, 16, dt)
